@@ -1,0 +1,513 @@
+#!/usr/bin/env python
+"""Throughput of the masked block-diffusion denoise step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 8b_b1]
+    python bench.py --impl reference ...        # the CPU oracle, same line format
+
+One "step" is one denoising step over the whole batch: embed, QKV + RoPE,
+attention, output projection, fused LM-head reduction, cross-tile reduce,
+commit / re-noise.  Steps run as CUDA-graph replays of whole blocks
+(``dlm_decode_block``); a block of the 8B-shaped batch-1 workload is 32 steps.
+K steps are timed with CUDA events on the launch stream between a barrier and
+device synchronisation on both sides; with N ranks each rank decodes its own
+batch (weak scaling, no collective on the data path) and the time is the
+maximum over ranks.  Rank 0 prints one JSON line.
+
+Inputs exceed L2: the LM head streams its 1.07 GB weight every step, so no
+L2 flush is needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+from masked_block_diffusion_denoise_b200 import roofline as RL  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1280)
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="8b_b1", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="a few eager steps only, for ncu captures")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_init(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit("WORLD_SIZE %d != --gpus %d" % (world, n_gpus))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return world, rank, local, pg
+
+
+def barrier(pg, device):
+    import torch
+    if pg is not None:
+        t = torch.zeros(1, device=device)
+        pg.all_reduce(t)
+    torch.cuda.synchronize(device)
+
+
+def max_over_ranks(pg, value, device):
+    import torch
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(a):
+    import torch
+    import masked_block_diffusion_denoise_b200 as dlm
+    from masked_block_diffusion_denoise_b200 import build as B
+    from masked_block_diffusion_denoise_b200.session import Session, sampler_params
+
+    world, rank, local, pg = dist_init(a.gpus)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if rank == 0:
+        B.build()
+    if pg is not None:
+        barrier(pg, device)
+    wl = W.WORKLOADS[a.workload]
+    sh = wl.shape
+    weights = W.make_weights(sh, seed=wl.seed)
+    lens, toks, kp, vp = W.make_prefix(wl)
+    sess = Session(sh, weights, max_batch=wl.batch, max_prefix=wl.prefix_cap,
+                   max_canvas=wl.canvas, device=device)
+    for b in range(wl.batch):
+        if toks is not None:
+            sess.kv_append_tokens(b, toks[b])
+        else:
+            n = int(lens[b])
+            sess.kv_append_kv(b, np.ascontiguousarray(kp[b][:, :n]),
+                              np.ascontiguousarray(vp[b][:, :n]))
+    del kp, vp
+    p = sampler_params(canvas=wl.canvas, steps=wl.steps, threshold=wl.threshold,
+                       quota=wl.quota, corruption=wl.corruption,
+                       entropy_bound=wl.entropy_bound, temperature=wl.temperature,
+                       t_max=wl.t_max, t_min=wl.t_min, seed=wl.seed)
+    S = wl.steps
+    stream = torch.cuda.Stream(device)
+    # template canvas: initial state (+ EOS plant), copied in before every block
+    tmpl = sess.new_canvas(wl.batch, wl.canvas)
+    with torch.cuda.stream(stream):
+        sess.init(tmpl, p, stream=stream)
+        for (b, slot) in W.make_eos_plant(wl):
+            tmpl.tokens[b, slot] = sh.eos_id
+            tmpl.committed[b, slot] = 1
+    stream.synchronize()
+    cv = sess.new_canvas(wl.batch, wl.canvas)
+
+    def reset(canvas):
+        for dst, src in ((canvas.tokens, tmpl.tokens), (canvas.committed, tmpl.committed),
+                         (canvas.step, tmpl.step), (canvas.done, tmpl.done),
+                         (canvas.eos_pos, tmpl.eos_pos)):
+            dst.copy_(src, non_blocking=True)
+
+    def run_steps(k, canvas):
+        """k steps: whole blocks as graph replays, the rest as single steps."""
+        full, rest = divmod(k, S)
+        with torch.cuda.stream(stream):
+            for _ in range(full):
+                reset(canvas)
+                sess.block(canvas, p, stream=stream)
+            if rest:
+                reset(canvas)
+                for _ in range(rest):
+                    sess.step(canvas, p, stream=stream)
+
+    if a.profile:
+        with torch.cuda.stream(stream):
+            reset(cv)
+            for _ in range(max(1, a.steps)):
+                sess.step(cv, p, stream=stream)
+        stream.synchronize()
+        sess.check(stream)
+        if rank == 0:
+            print(json.dumps({"profile": a.workload, "steps": a.steps}))
+        return
+
+    K, Wm = a.steps, max(a.warmup, 3)
+    run_steps(max(Wm, S), cv)            # warm-up (also captures the block graph)
+    stream.synchronize()
+    sess.check(stream)
+    launches_per_step = dlm.dlm_launches_per_step(sess.ctx)
+
+    # ---- timed region ----
+    clocks = Clocks(local) if rank == 0 else None
+    stats0 = cv.stats.clone()
+    cv.stats.zero_()
+    barrier(pg, device)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg, device)
+    e0.record(stream)
+    run_steps(K, cv)
+    e1.record(stream)
+    stream.synchronize()
+    barrier(pg, device)
+    ck = clocks.stop() if clocks else None
+    sess.check(stream)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(pg, ms, device)
+    committed = int(cv.stats[:, 1].sum().item())
+    committed_all = max_over_ranks(pg, committed, device) * world
+    del stats0
+
+    # ---- roofline of the dominant kernel: LM-head launches of the timed pass
+    # configuration, events recorded inside the replayed graph ----
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * S)]
+    for e in evs:            # torch creates the CUDA event on its first record
+        e.record(stream)
+    stream.synchronize()
+    dlm.dlm_set_stage_events(sess.ctx, dlm.DLM_STAGE_LM_HEAD, [e.cuda_event for e in evs])
+    n_roof_blocks = max(3, min(20, K // S))
+    run_steps(n_roof_blocks * S, cv)
+    stream.synchronize()
+    lm_ms = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(S)]
+    stages = {}
+    names = ["embed", "qkv", "attention", "wo", "lm_head", "reduce", "commit"]
+    for st, name in enumerate(names):
+        dlm.dlm_set_stage_events(sess.ctx, st, [e.cuda_event for e in evs])
+        run_steps(2 * S, cv)
+        stream.synchronize()
+        stages[name] = 1e3 * statistics.mean(evs[2 * i].elapsed_time(evs[2 * i + 1])
+                                             for i in range(S))
+    dlm.dlm_set_stage_events(sess.ctx, 0, [])
+
+    # ---- end to end through the host-buffer entry point ----
+    e2e = None
+    if not a.no_e2e:
+        host = {k: getattr(tmpl, k).cpu().pin_memory() for k in
+                ("tokens", "committed", "step", "done", "eos_pos")}
+        hstats = torch.zeros((wl.batch, 4), dtype=torch.int32).pin_memory()
+        work = {k: v.clone().pin_memory() for k, v in host.items()}
+        n_blocks = max(1, K // S)
+        h2d = sum(v.numel() * v.element_size() for v in host.values()) + hstats.numel() * 4
+        d2h = h2d
+        barrier(pg, device)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n_blocks):
+            for k in work:
+                work[k].copy_(host[k])
+            dlm.dlm_decode_block_host(sess.ctx, work["tokens"], work["committed"], work["step"],
+                                      work["done"], work["eos_pos"], wl.batch, p, stats=hstats,
+                                      stream=stream)
+        f1.record(stream)
+        stream.synchronize()
+        e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), device)
+        e2e = {"value": world * n_blocks * S / (e2e_ms / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": h2d / S, "d2h_bytes_per_step": d2h / S,
+               "blocks": n_blocks, "call": "dlm_decode_block_host"}
+
+    if rank == 0:
+        pk = peaks()
+        shape = RL.StepShape(sh.d_model, sh.n_heads, sh.n_kv_heads, sh.head_dim, sh.vocab, 2,
+                             wl.canvas, [int(x) for x in lens])
+        work_ = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256)
+        lm_avg_s = statistics.mean(lm_ms) / 1e3
+        bound = "hbm" if work_["lm_head"]["flop"] / work_["lm_head"]["bytes"] < 250 else "tensor"
+        if bound == "hbm":
+            ach = work_["lm_head"]["bytes"] / lm_avg_s / 1e9
+            peak = pk["hbm_gbs"]
+            unit = "GB/s"
+        else:
+            ach = work_["lm_head"]["flop"] / lm_avg_s / 1e12
+            peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+            unit = "TFLOP/s"
+        roof = {"kernel": "gemm_tc_kernel<EPI_LM> (LM head + fused vocab reduction)",
+                "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+                "frac": round(ach / peak, 4), "traffic": None,
+                "peak_source": pk.get("source", "measured") + (" hbm_gbs" if bound == "hbm"
+                                                               else " bf16_tflops_sustained"),
+                "launch_us": round(lm_avg_s * 1e6, 2),
+                "algorithmic_bytes_per_launch": work_["lm_head"]["bytes"],
+                "algorithmic_flop_per_launch": work_["lm_head"]["flop"],
+                "launches_timed": len(lm_ms)}
+        traffic = _ncu_traffic(a.workload)
+        if traffic is not None:
+            roof["traffic"] = traffic
+        step_s = ms_max / 1e3 / K
+        line = {
+            "metric": "denoise steps/s", "value": round(world * K / (ms_max / 1e3), 2),
+            "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": max(Wm, S),
+            "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if sh.dtype == "bf16" else "f32",
+            "data": "synthetic: seeded random-init weights N(0,0.02), embeddings and prefix "
+                    "K/V N(0,1), all-mask canvas",
+            "config": {"workload": a.workload, "batch": wl.batch, "canvas": wl.canvas,
+                       "prefix": [int(lens.min()), int(lens.max())], "steps_per_block": S,
+                       "threshold": wl.threshold, "quota": wl.quota_eff,
+                       "corruption": wl.corruption, "d_model": sh.d_model,
+                       "heads": [sh.n_heads, sh.n_kv_heads, sh.head_dim], "vocab": sh.vocab,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (the LM head streams 1.07 GB of weights "
+                             "every step); no flush"},
+            "committed_tokens_per_s": round(committed_all / (ms_max / 1e3), 1),
+            "stages_us": {k: round(v, 2) for k, v in stages.items()},
+            "step_algorithmic_bytes": work_["step"]["bytes"],
+            "step_hbm_frac": round(work_["step"]["bytes"] / step_s / 1e9 / pk["hbm_gbs"], 4),
+            "roofline": roof,
+            "gpu_launches": int(launches_per_step * K),
+            "e2e": e2e,
+            "clocks": ck,
+        }
+        if world == 1 and not a.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    sess.close()
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def _ncu_traffic(workload):
+    """DRAM bytes per LM-head launch from the committed ncu summary, if it
+    describes this workload and the current kernel."""
+    path = os.path.join(ROOT, "profiles", "lm_head_%s.json" % workload)
+    try:
+        with open(path) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle
+# ---------------------------------------------------------------------------
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_setup(wl, vocab_slice=None):
+    from oracle import dlm_oracle as O
+    sh = wl.shape
+    w = W.make_weights(sh, seed=wl.seed)
+    if vocab_slice is not None:
+        w = dict(w)
+        w["w_lm"] = np.ascontiguousarray(w["w_lm"][:vocab_slice])
+    dims = O.ModelDims.of(sh)
+    if vocab_slice is not None:
+        dims.vocab = vocab_slice
+    om = O.OracleModel(dims, w)
+    lens, toks, kp, vp = W.make_prefix(wl)
+    conv = O.bf16_bits_to_f64 if sh.dtype == "bf16" else (lambda x: np.asarray(x, np.float64))
+    for b in range(wl.batch):
+        if toks is not None:
+            om.kv_append_tokens(b, toks[b])
+        else:
+            n = int(lens[b])
+            om.kv_append_kv(b, conv(kp[b][:, :n]), conv(vp[b][:, :n]))
+    p = O.SamplerParams(canvas=wl.canvas, steps=wl.steps, threshold=wl.threshold,
+                        quota=wl.quota, corruption=wl.corruption,
+                        entropy_bound=wl.entropy_bound, temperature=wl.temperature,
+                        t_max=wl.t_max, t_min=wl.t_min, seed=wl.seed)
+    st = O.init_canvas(wl.batch, p, sh.mask_id, sh.vocab)
+    return O, om, p, st
+
+
+def _oracle_step_timed(O, om, p, st, vocab_full):
+    """One oracle step; returns (seconds of forward-to-y, of LM head + scores,
+    of selection).  The LM head may cover a vocabulary slice."""
+    t_fwd = t_lm = t_sel = 0.0
+    for b in range(st.tokens.shape[0]):
+        if st.done[b]:
+            continue
+        t0 = time.perf_counter()
+        x = om.embed(st.tokens[b])
+        L = om.kv_len(b)
+        q, k, v = om.project_qkv(x, np.arange(L, L + len(x)))
+        o = om.attend(b, q, k, v)
+        y = om.out_proj(x, o)
+        t1 = time.perf_counter()
+        lg = om.logits(y)
+        mask = om.dims.mask_id if p.corruption == "mask" else -1
+        cand, conf, H, _ = O.scores(lg, mask if mask < lg.shape[1] else -1)
+        t2 = time.perf_counter()
+        O.select_canvas(st, b, cand, conf, H, p, vocab=vocab_full, mask_id=om.dims.mask_id,
+                        eos_id=om.dims.eos_id)
+        t3 = time.perf_counter()
+        t_fwd += t1 - t0
+        t_lm += t2 - t1
+        t_sel += t3 - t2
+    return t_fwd, t_lm, t_sel
+
+
+def cpu_baseline(wl):
+    """The oracle, as it stands, timed on this host over full steps for about
+    10-30 s (at least two steps)."""
+    O, om, p, st = _oracle_setup(wl)
+    times = []
+    t_start = time.perf_counter()
+    while len(times) < 2 or (time.perf_counter() - t_start < 10.0 and len(times) < 32):
+        if st.done.all():
+            st = O.init_canvas(wl.batch, p, wl.shape.mask_id, wl.shape.vocab)
+        f, l, s = _oracle_step_timed(O, om, p, st, wl.shape.vocab)
+        times.append(f + l + s)
+    return {"value": round(len(times) / sum(times), 4), "unit": "steps/s",
+            "cores": _threads(), "host_cpus": os.cpu_count(), "kind": "oracle",
+            "sample": "%d full oracle steps of the %s block (float64 NumPy)" % (len(times),
+                                                                            wl.name)}
+
+
+def run_reference(a):
+    """--impl reference: the oracle on this host, K timed steps after W
+    warm-up steps; each step computes the full forward to the LM-head input
+    and the LM head + scores on a vocabulary slice of 1/f of the rows of W_lm,
+    whose time is scaled by f (every other stage in full)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[a.workload]
+    V = wl.shape.vocab
+    f = 32
+    O, om, p, st = _oracle_setup(wl, vocab_slice=V // f)
+    K, Wm = a.steps, max(a.warmup, 3)
+    total = 0.0
+    for i in range(Wm + K):
+        if st.done.all():
+            st = O.init_canvas(wl.batch, p, wl.shape.mask_id, V)
+        fw, lm, sel = _oracle_step_timed(O, om, p, st, V)
+        if i >= Wm:
+            total += fw + lm * f + sel
+    value = K / total
+    line = {"metric": "denoise steps/s", "value": round(value, 4), "unit": "steps/s",
+            "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": round(1e3 * total / K, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": a.workload, "batch": wl.batch, "canvas": wl.canvas,
+                       "vocab": V},
+            "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": _threads(),
+                             "kind": "oracle",
+                             "sample": "each step: full forward to the LM-head input, LM head "
+                                       "and scores on 1/%d of the vocabulary, time scaled "
+                                       "by %d" % (f, f)},
+            "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * dlm.h -- C ABI of the masked block-diffusion denoise-step library
+ * (NVIDIA B200, sm_100a).
+ *
+ * One denoising step of masked block-diffusion decoding over a fixed canvas of
+ * C positions per sequence:
+ *   1. bidirectional attention of every canvas position over the cached
+ *      prefix K/V plus all canvas positions (Nemotron Labs Diffusion guide,
+ *      section 6: the whole block is denoised with a bidirectional mask;
+ *      course "Diffusion LLMs", section 14: the current block reads the
+ *      finished prefix and all of its own positions);
+ *   2. the LM-head projection to vocabulary logits (same guide, section 7:
+ *      an untied diffusion head over a 131072-token vocabulary), whose
+ *      per-position softmax maximum, argmax, normaliser and entropy are
+ *      reduced inside the GEMM, so full logits never reach HBM (same guide,
+ *      section 5.3: non-materialised chunked scoring);
+ *   3. per-position confidence = probability of the candidate and entropy
+ *      (course section 12 and section 9);
+ *   4. the sampler: commit every uncommitted position whose confidence is at
+ *      least the threshold, at least a uniform per-step quota of the most
+ *      confident, and everything left on the last step of the budget; keep
+ *      the mask id or re-noise the rest with uniform random ids; or, with an
+ *      entropy bound, commit the lowest-entropy positions whose summed
+ *      entropy stays under the bound (diffusers DiffusionGemma page,
+ *      BlockRefinementScheduler and EntropyBoundScheduler; Nemotron guide,
+ *      sections 3.2 and 6).
+ *
+ * Conventions for every call:
+ *   - Pointers named *_dev / documented "device" are CUDA device pointers
+ *     owned by the caller; pointers documented "host" are host memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).  The int result reports argument
+ *     and launch errors synchronously; it is DLM_OK (0) or a negative code.
+ *   - Device-detected errors (a bounded wait that ran out) set an error word
+ *     in the context; dlm_check() synchronises `stream` and returns it.
+ *   - A context is not thread-safe: one host thread drives it at a time.
+ *   - On any error, dlm_last_error() describes the first one.
+ */
+#ifndef DLM_H_
+#define DLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+enum {
+  DLM_OK = 0,
+  DLM_EINVAL = -1,    /* an argument is out of range or inconsistent          */
+  DLM_ENOMEM = -2,    /* device or host allocation failed                     */
+  DLM_ECUDA = -3,     /* a CUDA runtime call failed                           */
+  DLM_ECAP = -4,      /* KV capacity (max_prefix) would be exceeded           */
+  DLM_ETIMEOUT = -5,  /* a device-side bounded wait ran out                   */
+  DLM_EBOUNDS = -6,   /* a device-side index check failed                     */
+  DLM_ESTATE = -7     /* the call does not fit the context's current state    */
+};
+
+enum { DLM_F32 = 0, DLM_BF16 = 1 };          /* model / weight element type  */
+enum { DLM_MASK = 0, DLM_UNIFORM = 1 };      /* corruption of uncommitted slots */
+
+typedef struct dlm_ctx dlm_ctx;
+
+/* Shape of the single-attention-layer denoiser.  Weights are row-major,
+ * out-features x in-features.  mask_id 100 and eos_id 11 are the Nemotron
+ * ids (guide, section 7); rope_theta 1e6 likewise; rope_theta <= 0 turns RoPE
+ * off.  eos_id < 0 disables EOS handling.  head_dim must be 64 or 128 for
+ * DLM_BF16 (128 only for bf16 attention) and <= 128 for DLM_F32. */
+typedef struct {
+  int d_model, n_heads, n_kv_heads, head_dim, vocab, dtype;
+  float rope_theta;
+  int mask_id, eos_id;
+  int max_batch;    /* sequences (canvases) per call                       */
+  int max_prefix;   /* KV capacity per sequence for the finished prefix    */
+  int max_canvas;   /* largest canvas length, <= 1024                       */
+} dlm_model_desc;
+
+/* Device pointers, caller-owned, valid for the life of the context; element
+ * type per dlm_model_desc.dtype (bf16 bit patterns or float32).
+ *   emb [vocab][d], w_q [H*Dh][d], w_k, w_v [Hkv*Dh][d], w_o [d][H*Dh],
+ *   w_lm [vocab][d].  w_q/w_k/w_v are copied into one fused matrix at
+ *   dlm_create; emb, w_o and w_lm are read in place. */
+typedef struct { const void *emb, *w_q, *w_k, *w_v, *w_o, *w_lm; } dlm_weights;
+
+/* Sampler parameters (DiffusionGemma page, __call__ and scheduler config;
+ * Nemotron guide, sections 3.2 and 5.5).
+ *   canvas      canvas length C, 1 <= C <= max_canvas
+ *   steps       step budget S >= 1; the step with index S-1 commits all
+ *   threshold   confidence threshold (>= is a hit); 0 commits everything
+ *   quota       minimum commits per step; <= 0 means ceil(C / S)
+ *   corruption  DLM_MASK: uncommitted slots hold mask_id (which is excluded
+ *               from the argmax, softmax and entropy); DLM_UNIFORM: they are
+ *               re-noised with uniform random ids after every step
+ *   editing     must be 0 (re-editing committed tokens is not supported)
+ *   entropy_bound  >= 0 selects the entropy-bound rule (temperature annealed
+ *               linearly from t_max at step 0 to t_min at step S-1, Gumbel
+ *               sampling); < 0 selects threshold + quota
+ *   temperature 0: greedy argmax; > 0: Gumbel sampling at this temperature
+ *               (threshold + quota rule only)
+ *   seed        key of the counter-based generator (Philox4x32-10)        */
+typedef struct {
+  int canvas, steps;
+  float threshold;
+  int quota;
+  int corruption;
+  int editing;
+  float entropy_bound;
+  float temperature, t_max, t_min;
+  unsigned long long seed;
+} dlm_sampler_params;
+
+/* Canvas state of `batch` sequences, device, caller-owned, updated in place:
+ *   tokens [B][C] int32, committed [B][C] uint8 (0/1), step [B] int32 (steps
+ *   taken), done [B] uint8, eos_pos [B] int32 (first committed EOS or -1).
+ * Canvas b attends to KV sequence b. */
+typedef struct {
+  int32_t *tokens;
+  uint8_t *committed;
+  int32_t *step;
+  uint8_t *done;
+  int32_t *eos_pos;
+} dlm_canvas;
+
+/* Per-canvas counters, device, caller-owned and caller-zeroed; every step
+ * adds to them.  committed_by_sampler counts positions the selection chose
+ * (forced ones included); forced_at_budget those committed only because the
+ * budget ran out; eos_autofill the uncommitted positions filled with EOS
+ * after the first committed EOS. */
+typedef struct {
+  int32_t steps_used;
+  int32_t committed_by_sampler;
+  int32_t forced_at_budget;
+  int32_t eos_autofill;
+} dlm_canvas_stats;
+
+/* Create a context: validates the descriptor, allocates the KV cache
+ * [max_batch][Hkv][max_prefix + max_canvas][Dh] (K and V), the activations
+ * and scratch, the fused QKV weight and the RoPE table on the current device.
+ * Returns DLM_EINVAL / DLM_ENOMEM / DLM_ECUDA; *out is NULL on failure. */
+int dlm_create(const dlm_model_desc *desc, const dlm_weights *weights, dlm_ctx **out);
+
+/* Free everything the context owns (synchronises the device first). */
+void dlm_destroy(dlm_ctx *ctx);
+
+/* Append n finished tokens to KV sequence `seq` (course section 14: the
+ * finished prefix is cached; the clean pass over a finished block supplies
+ * its states).  Either `tokens` (device int32[n]) is given and K = RoPE(E[t]
+ * W_k^T), V = E[t] W_v^T are computed at absolute positions len..len+n-1,
+ * or tokens == NULL and `k`, `v` (device, [Hkv][n][Dh], already rotated, in
+ * the model's element type) are copied in.  DLM_ECAP if len + n >
+ * max_prefix; the length is tracked on the host and on the device. */
+int dlm_kv_append(dlm_ctx *ctx, int seq, int n, const int32_t *tokens, const void *k,
+                  const void *v, void *stream);
+
+/* Set the length of KV sequence `seq` to 0 (no device work). */
+int dlm_reset_kv(dlm_ctx *ctx, int seq);
+
+/* Current length of KV sequence `seq`, or a negative code. */
+int dlm_kv_length(const dlm_ctx *ctx, int seq);
+
+/* Initialise `batch` canvases: all mask_id (DLM_MASK) or uniform random ids
+ * from Philox counter (b, 0, i, 0xFFFFFFFF) (DLM_UNIFORM); committed = 0,
+ * step = 0, done = 0, eos_pos = -1. */
+int dlm_canvas_init(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+                    const dlm_sampler_params *params, void *stream);
+
+/* One denoising step over the canvases that are not done: embed, QKV+RoPE,
+ * attention, output projection, fused LM-head reduction, cross-tile reduce,
+ * commit/re-noise, one kernel launch each.  Canvas K/V of
+ * the step occupy cache slots len..len+C-1 of each sequence (not appended).
+ * `stats` (device, [batch]) may be NULL. */
+int dlm_denoise_step(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+                     const dlm_sampler_params *params, dlm_canvas_stats *stats, void *stream);
+
+/* `params->steps` denoising steps (the whole block; steps of canvases that
+ * are already done do no work), captured once per configuration into a CUDA
+ * graph and replayed on `stream`.  Same arguments as dlm_denoise_step. */
+int dlm_decode_block(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+                     const dlm_sampler_params *params, dlm_canvas_stats *stats, void *stream);
+
+/* dlm_decode_block with HOST buffers: copies the canvas state in (host
+ * arrays shaped as in dlm_canvas), runs the block, copies the canvas state
+ * and `stats` (host, may be NULL) back, and synchronises `stream`.  The
+ * device copies live in the context. */
+int dlm_decode_block_host(dlm_ctx *ctx, int32_t *tokens, uint8_t *committed, int32_t *step,
+                          uint8_t *done, int32_t *eos_pos, int batch,
+                          const dlm_sampler_params *params, dlm_canvas_stats *stats,
+                          void *stream);
+
+/* Kernel (c) alone: the sampler update of dlm_denoise_step applied to given
+ * per-position candidates (device int32 [B][C]), confidences and entropies
+ * (device float32 [B][C]).  Used to check the selection bit for bit. */
+int dlm_commit(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+               const dlm_sampler_params *params, const int32_t *cand, const float *conf,
+               const float *entropy, dlm_canvas_stats *stats, void *stream);
+
+/* Read-only views of the context's buffers after a step, for inspection.
+ * which: DLM_BUF_X [M][d], DLM_BUF_Q [M][H][Dh], DLM_BUF_O [M][H*Dh],
+ * DLM_BUF_Y [M][d] (model element type; M = batch * C, row b*C + i),
+ * DLM_BUF_CAND int32 [M], DLM_BUF_CONF float [M], DLM_BUF_ENTROPY float [M],
+ * DLM_BUF_K_CACHE / DLM_BUF_V_CACHE [max_batch][Hkv][max_prefix+max_canvas][Dh].
+ * *ptr receives a device pointer owned by the context, *bytes its size. */
+enum { DLM_BUF_X = 0, DLM_BUF_Q = 1, DLM_BUF_O = 2, DLM_BUF_Y = 3, DLM_BUF_CAND = 4,
+       DLM_BUF_CONF = 5, DLM_BUF_ENTROPY = 6, DLM_BUF_K_CACHE = 7, DLM_BUF_V_CACHE = 8 };
+int dlm_debug_buffer(dlm_ctx *ctx, int which, void **ptr, size_t *bytes);
+
+/* Full float32 logits of the rows in DLM_BUF_Y: `logits` (device float
+ * [batch*canvas][vocab]) receives y W_lm^T from the same GEMM main loop as
+ * the fused reduction (the store epilogue instead of the reduction). */
+int dlm_debug_logits(dlm_ctx *ctx, int batch, int canvas, float *logits, void *stream);
+
+/* Stages of a step, for dlm_set_stage_events. */
+enum { DLM_STAGE_EMBED = 0, DLM_STAGE_QKV = 1, DLM_STAGE_ATTENTION = 2, DLM_STAGE_WO = 3,
+       DLM_STAGE_LM_HEAD = 4, DLM_STAGE_REDUCE = 5, DLM_STAGE_COMMIT = 6, DLM_NUM_STAGES = 7 };
+
+/* Measurement hook: record caller-created CUDA events (cudaEvent_t passed as
+ * void*, created with timing enabled, owned by the caller) on the launch
+ * stream immediately before and after `stage` of the steps issued from now
+ * on: step s of a dlm_decode_block (or the s-th dlm_denoise_step call since
+ * this call) uses events[2*(s % n_pairs)] and events[2*(s % n_pairs) + 1].
+ * Inside a CUDA graph the records are graph nodes, so after a replay each
+ * pair brackets that stage of one step.  n_pairs = 0 (events may be NULL)
+ * turns the hook off.  The array is copied; the events must outlive their
+ * use.  DLM_EINVAL for a bad stage or n_pairs < 0. */
+int dlm_set_stage_events(dlm_ctx *ctx, int stage, void *const *events, int n_pairs);
+
+/* Synchronise `stream` and return the device error word (DLM_OK, or
+ * DLM_ETIMEOUT / DLM_EBOUNDS set by a kernel); clears it. */
+int dlm_check(dlm_ctx *ctx, void *stream);
+
+/* Number of kernel launches one dlm_denoise_step made for this batch and
+ * configuration (the last one issued), for launch accounting. */
+int dlm_launches_per_step(const dlm_ctx *ctx);
+
+/* Text of the first error since the last successful call, or "". */
+const char *dlm_last_error(const dlm_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DLM_H_ */

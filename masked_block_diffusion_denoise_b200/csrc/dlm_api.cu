@@ -1,0 +1,852 @@
+// Host side of the C ABI declared in include/dlm.h: context, argument
+// validation, work plans, TMA tensor maps, the kernel sequence of one
+// denoising step and the CUDA-graph replay of a block.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "kernels.h"
+
+using namespace dlm;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+struct GraphEntry {
+  std::vector<uint8_t> key;
+  cudaGraphExec_t exec = nullptr;
+  int launches = 0;
+};
+
+}  // namespace
+
+struct dlm_ctx {
+  dlm_model_desc d{};
+  ModelDims md{};
+  int dev = 0, num_sms = 148;
+  bool bf16 = true;
+  size_t es = 2;
+  const void *emb = nullptr, *w_o = nullptr, *w_lm = nullptr;
+  void* w_qkv = nullptr;
+  int Nqkv = 0;
+  void *kc = nullptr, *vc = nullptr;
+  int Lcap = 0;
+  std::vector<int> lens_h;
+  int32_t* lens_d = nullptr;
+  int Mmax = 0;
+  void *x = nullptr, *q = nullptr, *o = nullptr, *y = nullptr;
+  float* part = nullptr;
+  size_t part_floats = 0;
+  float* opart = nullptr;
+  size_t opart_floats = 0;
+  float2* ml = nullptr;
+  size_t ml_count = 0;
+  LmPart* lmpart = nullptr;
+  int32_t* cand = nullptr;
+  float *conf = nullptr, *ent = nullptr;
+  float2* rope = nullptr;
+  int* n_active = nullptr;
+  int* err = nullptr;
+  // device copies of a canvas for the host-buffer entry point
+  int32_t *h_tok = nullptr, *h_step = nullptr, *h_eos = nullptr;
+  uint8_t *h_com = nullptr, *h_done = nullptr;
+  dlm_canvas_stats* h_stats = nullptr;
+  std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> maps;
+  CUtensorMap tmK{}, tmV{};
+  std::vector<GraphEntry> graphs;
+  cudaStream_t cap = nullptr;
+  std::string msg;
+  int launches = 0;
+  // measurement hook: events around one stage
+  int ev_stage = -1;
+  std::vector<cudaEvent_t> ev;
+  int ev_step = 0;
+  std::vector<void*> owned;
+};
+
+namespace {
+
+int fail(dlm_ctx* c, int code, const std::string& what) {
+  if (c) {
+    if (c->msg.empty()) c->msg = what;
+  } else {
+    g_create_error = what;
+  }
+  return code;
+}
+
+int cuda_fail(dlm_ctx* c, const char* where, cudaError_t e) {
+  return fail(c, DLM_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(call)                                            \
+  do {                                                      \
+    cudaError_t e_ = (call);                                \
+    if (e_ != cudaSuccess) return cuda_fail(ctx, #call, e_); \
+  } while (0)
+
+template <typename T>
+int dalloc(dlm_ctx* ctx, T** p, size_t bytes) {
+  void* v = nullptr;
+  cudaError_t e = cudaMalloc(&v, bytes < 256 ? 256 : bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ctx, DLM_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+  }
+  ctx->owned.push_back(v);
+  *p = reinterpret_cast<T*>(v);
+  return DLM_OK;
+}
+
+const CUtensorMap* map2d(dlm_ctx* ctx, const void* ptr, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows) {
+  auto key = std::make_tuple(ptr, rows, cols, box_rows);
+  auto it = ctx->maps.find(key);
+  if (it != ctx->maps.end()) return &it->second;
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return nullptr;
+  CUtensorMap m;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return nullptr;
+  return &(ctx->maps[key] = m);
+}
+
+bool map_kv(CUtensorMap* m, void* base, uint64_t planes, uint64_t Lcap, uint64_t Dh) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {Dh, Lcap, planes};
+  cuuint64_t strides[2] = {Dh * 2, Lcap * Dh * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------
+// work plans
+// ---------------------------------------------------------------------------
+
+// splits of K that keep the most SMs busy (units = tiles * splits over
+// whole waves of num_sms), fewer splits preferred on near ties
+int pick_splits(int tiles, int kblocks, int num_sms, int max_splits) {
+  if (tiles >= num_sms) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  const int lim = std::min(max_splits, std::max(1, kblocks / 2));
+  for (int s = 1; s <= lim; ++s) {
+    const int units = tiles * s;
+    const int waves = cdiv(units, num_sms);
+    const double eff = (double)units / ((double)waves * num_sms);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
+  GemmPlan p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.epi = epi;
+  p.splits = 1;
+  if (!ctx->bf16) {
+    p.BN = 64;
+    if (epi == EPI_F32) {
+      const int tiles = cdiv(M, 64) * cdiv(N, 64);
+      p.splits = pick_splits(tiles, cdiv(K, 16) / 4, ctx->num_sms, 8);
+    }
+    return p;
+  }
+  const int mt = cdiv(M, 128);
+  if (epi == EPI_LM) {
+    p.BN = mt > 1 ? 256 : 128;
+    return p;
+  }
+  p.BN = (mt > 1 && mt * cdiv(N, 128) >= 4 * ctx->num_sms) ? 256 : 128;
+  if (mt == 1) p.splits = pick_splits(cdiv(N, p.BN), cdiv(K, 64), ctx->num_sms, 16);
+  return p;
+}
+
+AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, int max_keys) {
+  AttnPlan a{};
+  a.B = B;
+  a.C = C;
+  a.G = ctx->md.H / ctx->md.Hkv;
+  a.R = a.G * C;
+  a.rtiles = cdiv(a.R, 128);
+  const int nbg = B * ctx->md.Hkv * a.rtiles;
+  long best_cost = -1;
+  for (int ns = 1; ns <= 64; ++ns) {
+    const int chunk = cdiv(cdiv(max_keys, ns), 64) * 64;
+    const int nse = cdiv(max_keys, chunk);
+    if (nse != ns) continue;
+    const long waves = cdiv(nbg * nse, ctx->num_sms);
+    const long cost = waves * chunk + 16L * nse;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      a.chunk = chunk;
+      a.nsplit = nse;
+    }
+  }
+  return a;
+}
+
+int max_len(const dlm_ctx* ctx, int batch) {
+  int m = 0;
+  for (int b = 0; b < batch; ++b) m = std::max(m, ctx->lens_h[b]);
+  return m;
+}
+
+int ensure_attn_scratch(dlm_ctx* ctx, const AttnPlan& ap) {
+  if (ap.nsplit <= 1) return DLM_OK;
+  const size_t slots = (size_t)ap.B * ctx->md.Hkv * ap.nsplit * ap.R;
+  if (slots * ctx->md.Dh > ctx->opart_floats) {
+    if (ctx->opart) {
+      cudaFree(ctx->opart);
+      ctx->owned.erase(std::find(ctx->owned.begin(), ctx->owned.end(), (void*)ctx->opart));
+      ctx->opart = nullptr;
+    }
+    if (int rc = dalloc(ctx, &ctx->opart, slots * ctx->md.Dh * sizeof(float))) return rc;
+    ctx->opart_floats = slots * ctx->md.Dh;
+  }
+  if (slots > ctx->ml_count) {
+    if (ctx->ml) {
+      cudaFree(ctx->ml);
+      ctx->owned.erase(std::find(ctx->owned.begin(), ctx->owned.end(), (void*)ctx->ml));
+      ctx->ml = nullptr;
+    }
+    if (int rc = dalloc(ctx, &ctx->ml, slots * sizeof(float2))) return rc;
+    ctx->ml_count = slots;
+  }
+  return DLM_OK;
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+
+int check_params(dlm_ctx* ctx, const dlm_sampler_params* p, int batch) {
+  if (p == nullptr) return fail(ctx, DLM_EINVAL, "params is NULL");
+  if (batch < 1 || batch > ctx->d.max_batch)
+    return fail(ctx, DLM_EINVAL, "batch must be in [1, max_batch]");
+  if (p->canvas < 1 || p->canvas > ctx->d.max_canvas)
+    return fail(ctx, DLM_EINVAL, "canvas must be in [1, max_canvas]");
+  if (p->steps < 1) return fail(ctx, DLM_EINVAL, "steps must be >= 1");
+  if (!(p->threshold >= 0.0f)) return fail(ctx, DLM_EINVAL, "threshold must be >= 0");
+  if (p->corruption != DLM_MASK && p->corruption != DLM_UNIFORM)
+    return fail(ctx, DLM_EINVAL, "corruption must be DLM_MASK or DLM_UNIFORM");
+  if (p->editing != 0) return fail(ctx, DLM_EINVAL, "editing mode is not supported");
+  if (p->corruption == DLM_MASK && (ctx->d.mask_id < 0 || ctx->d.mask_id >= ctx->d.vocab))
+    return fail(ctx, DLM_EINVAL, "mask corruption needs mask_id in [0, vocab)");
+  if (!(p->temperature >= 0.0f)) return fail(ctx, DLM_EINVAL, "temperature must be >= 0");
+  if (p->entropy_bound >= 0.0f && !(p->t_min > 0.0f && p->t_max >= p->t_min))
+    return fail(ctx, DLM_EINVAL, "entropy bound needs 0 < t_min <= t_max");
+  return DLM_OK;
+}
+
+int check_canvas(dlm_ctx* ctx, const dlm_canvas* c) {
+  if (c == nullptr || !c->tokens || !c->committed || !c->step || !c->done || !c->eos_pos)
+    return fail(ctx, DLM_EINVAL, "canvas buffers must all be non-NULL");
+  return DLM_OK;
+}
+
+LmEpi make_epi(const dlm_ctx* ctx, const dlm_sampler_params* p, const dlm_canvas* c) {
+  LmEpi e{};
+  e.V = ctx->d.vocab;
+  e.mask_id = p->corruption == DLM_MASK ? ctx->d.mask_id : -1;
+  e.C = p->canvas;
+  e.S = p->steps;
+  e.t_max = p->t_max;
+  e.t_min = p->t_min;
+  if (p->entropy_bound >= 0.0f) {
+    e.mode = LM_SAMPLE_ANNEAL;
+  } else if (p->temperature > 0.0f) {
+    e.mode = LM_SAMPLE_FIXED;
+    e.inv_temp = 1.0f / p->temperature;
+  } else {
+    e.mode = LM_GREEDY;
+  }
+  e.seed_lo = (uint32_t)(p->seed & 0xFFFFFFFFull);
+  e.seed_hi = (uint32_t)(p->seed >> 32);
+  e.step = c->step;
+  return e;
+}
+
+SelectArgs make_select(const dlm_ctx* ctx, const dlm_sampler_params* p, int batch) {
+  SelectArgs a{};
+  a.B = batch;
+  a.C = p->canvas;
+  a.S = p->steps;
+  a.V = ctx->d.vocab;
+  a.quota = p->quota > 0 ? p->quota : cdiv(p->canvas, p->steps);
+  a.threshold = p->threshold;
+  a.eb = p->entropy_bound >= 0.0f;
+  a.bound = p->entropy_bound;
+  a.uniform = p->corruption == DLM_UNIFORM;
+  a.mask_id = ctx->d.mask_id;
+  a.eos_id = ctx->d.eos_id;
+  a.seed_lo = (uint32_t)(p->seed & 0xFFFFFFFFull);
+  a.seed_hi = (uint32_t)(p->seed >> 32);
+  return a;
+}
+
+// one GEMM through the engine of the model's element type
+int run_gemm(dlm_ctx* ctx, const void* A, const void* B, int Brows, const GemmPlan& plan,
+             const GemmIO& io, cudaStream_t st) {
+  cudaError_t e;
+  if (ctx->bf16) {
+    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K, 128);
+    const CUtensorMap* tb = map2d(ctx, B, (uint64_t)Brows, (uint64_t)plan.K, (uint32_t)plan.BN);
+    if (ta == nullptr || tb == nullptr)
+      return fail(ctx, DLM_ECUDA, "cuTensorMapEncodeTiled failed");
+    e = gemm_tc(*ta, *tb, plan, io, ctx->num_sms, st);
+  } else {
+    e = gemm_f32((const float*)A, (const float*)B, plan, io, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(ctx, "gemm launch", e);
+  ++ctx->launches;
+  return DLM_OK;
+}
+
+// record the measurement event of `stage` (begin or end) for the current step
+int stage_event(dlm_ctx* ctx, int stage, bool end, cudaStream_t st) {
+  if (ctx->ev_stage != stage || ctx->ev.empty()) return DLM_OK;
+  const int pairs = (int)ctx->ev.size() / 2;
+  // external: under stream capture the record becomes an event-record node of the graph
+  cudaError_t e = cudaEventRecordWithFlags(ctx->ev[2 * (ctx->ev_step % pairs) + (end ? 1 : 0)],
+                                           st, cudaEventRecordExternal);
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaEventRecord (stage events)", e);
+  return DLM_OK;
+}
+
+#define STAGE(s, end)                                                  \
+  do {                                                                 \
+    if (int rc_ = stage_event(ctx, (s), (end), st)) return rc_;         \
+  } while (0)
+
+// the kernel sequence of one denoising step
+int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                 dlm_canvas_stats* stats, const AttnPlan& ap, cudaStream_t st) {
+  const ModelDims& md = ctx->md;
+  const int C = p->canvas;
+  const int rows = batch * C;
+  cudaError_t e;
+  // a1: embedding gather (+ count of unfinished canvases)
+  STAGE(DLM_STAGE_EMBED, false);
+  e = embed_rows(md, c->tokens, ctx->emb, ctx->x, rows, C, batch, c->done, ctx->n_active,
+                 ctx->err, st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "embed", e);
+  ++ctx->launches;
+  STAGE(DLM_STAGE_EMBED, true);
+  // a2: fused QKV projection, RoPE, q and canvas K/V into the cache
+  STAGE(DLM_STAGE_QKV, false);
+  {
+    GemmPlan pl = plan_gemm(ctx, rows, ctx->Nqkv, md.d, EPI_F32);
+    GemmIO io;
+    io.out = ctx->part;
+    io.n_active = ctx->n_active;
+    io.err = ctx->err;
+    if (int rc = run_gemm(ctx, ctx->x, ctx->w_qkv, ctx->Nqkv, pl, io, st)) return rc;
+    e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
+                     ctx->kc, ctx->vc, c->done, ctx->n_active, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue", e);
+    ++ctx->launches;
+  }
+  STAGE(DLM_STAGE_QKV, true);
+  // a3: attention over [prefix ; canvas]
+  STAGE(DLM_STAGE_ATTENTION, false);
+  if (ctx->bf16) {
+    e = attention_bf16(md, ap, ctx->tmK, ctx->tmV, ctx->q, ctx->o, ctx->opart, ctx->ml,
+                       ctx->lens_d, c->done, ctx->n_active, ctx->err, st);
+    ctx->launches += ap.nsplit > 1 ? 2 : 1;
+  } else {
+    e = attention_f32(md, batch, C, (const float*)ctx->q, (const float*)ctx->kc,
+                      (const float*)ctx->vc, (float*)ctx->o, ctx->lens_d, c->done,
+                      ctx->n_active, st);
+    ++ctx->launches;
+  }
+  if (e != cudaSuccess) return cuda_fail(ctx, "attention", e);
+  STAGE(DLM_STAGE_ATTENTION, true);
+  // a4: output projection + residual
+  STAGE(DLM_STAGE_WO, false);
+  {
+    GemmPlan pl = plan_gemm(ctx, rows, md.d, md.H * md.Dh, EPI_F32);
+    GemmIO io;
+    io.out = ctx->part;
+    io.n_active = ctx->n_active;
+    io.err = ctx->err;
+    if (int rc = run_gemm(ctx, ctx->o, ctx->w_o, md.d, pl, io, st)) return rc;
+    e = wo_epilogue(md, ctx->part, pl.splits, rows, C, ctx->x, ctx->y, c->done, ctx->n_active,
+                    st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "wo epilogue", e);
+    ++ctx->launches;
+  }
+  STAGE(DLM_STAGE_WO, true);
+  // a5: LM head with the fused vocabulary reduction
+  GemmPlan pl = plan_gemm(ctx, rows, md.V, md.d, EPI_LM);
+  STAGE(DLM_STAGE_LM_HEAD, false);
+  {
+    GemmIO io;
+    io.part = ctx->lmpart;
+    io.epi = make_epi(ctx, p, c);
+    io.done = c->done;
+    io.n_active = ctx->n_active;
+    io.err = ctx->err;
+    if (int rc = run_gemm(ctx, ctx->y, ctx->w_lm, md.V, pl, io, st)) return rc;
+  }
+  STAGE(DLM_STAGE_LM_HEAD, true);
+  // a6: cross-tile reduction
+  STAGE(DLM_STAGE_REDUCE, false);
+  e = lm_reduce(ctx->lmpart, rows, cdiv(md.V, pl.BN), C, c->done, ctx->n_active, ctx->cand,
+                ctx->conf, ctx->ent, st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "lm reduce", e);
+  ++ctx->launches;
+  STAGE(DLM_STAGE_REDUCE, true);
+  // a7: commit / re-noise
+  STAGE(DLM_STAGE_COMMIT, false);
+  e = commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
+                  c->eos_pos, ctx->cand, ctx->conf, ctx->ent, stats, ctx->n_active, ctx->err, st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "commit", e);
+  ++ctx->launches;
+  STAGE(DLM_STAGE_COMMIT, true);
+  ++ctx->ev_step;
+  return DLM_OK;
+}
+
+size_t part_floats_needed(const dlm_ctx* ctx) {
+  size_t need = 0;
+  const ModelDims& md = ctx->md;
+  std::vector<int> Ms;
+  for (int m = 1; m <= ctx->Mmax; m = (m < 128 ? m * 2 : m + 128)) Ms.push_back(m);
+  Ms.push_back(ctx->Mmax);
+  for (int M : Ms) {
+    const int uses[3][2] = {{ctx->Nqkv, md.d}, {md.d, md.H * md.Dh}, {2 * md.Hkv * md.Dh, md.d}};
+    for (auto& u : uses) {
+      GemmPlan pl = plan_gemm(ctx, M, u[0], u[1], EPI_F32);
+      need = std::max(need, (size_t)pl.splits * M * u[0]);
+    }
+  }
+  return need;
+}
+
+void destroy_graphs(dlm_ctx* ctx) {
+  for (auto& g : ctx->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  ctx->graphs.clear();
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+
+extern "C" {
+
+int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) {
+  g_create_error.clear();
+  if (out == nullptr) return fail(nullptr, DLM_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (desc == nullptr || w == nullptr) return fail(nullptr, DLM_EINVAL, "desc/weights NULL");
+  const dlm_model_desc& d = *desc;
+  if (d.dtype != DLM_F32 && d.dtype != DLM_BF16)
+    return fail(nullptr, DLM_EINVAL, "dtype must be DLM_F32 or DLM_BF16");
+  if (d.d_model <= 0 || d.n_heads <= 0 || d.n_kv_heads <= 0 || d.vocab <= 0 || d.head_dim <= 0)
+    return fail(nullptr, DLM_EINVAL, "model dimensions must be positive");
+  if (d.n_heads % d.n_kv_heads != 0)
+    return fail(nullptr, DLM_EINVAL, "n_heads must be a multiple of n_kv_heads");
+  if (d.dtype == DLM_BF16 && (d.head_dim != 128 || d.d_model % 64 != 0))
+    return fail(nullptr, DLM_EINVAL, "bf16 model needs head_dim 128 and d_model % 64 == 0");
+  if (d.dtype == DLM_F32 && !(d.head_dim == 32 || d.head_dim == 64 || d.head_dim == 128))
+    return fail(nullptr, DLM_EINVAL, "fp32 model needs head_dim 32, 64 or 128");
+  if (d.dtype == DLM_F32 && d.d_model % 4 != 0)
+    return fail(nullptr, DLM_EINVAL, "fp32 model needs d_model % 4 == 0");
+  if (d.mask_id >= d.vocab || d.eos_id >= d.vocab)
+    return fail(nullptr, DLM_EINVAL, "mask_id / eos_id must be < vocab");
+  if (d.max_batch < 1 || d.max_prefix < 0 || d.max_canvas < 1 || d.max_canvas > 1024)
+    return fail(nullptr, DLM_EINVAL, "need max_batch >= 1, max_prefix >= 0, 1 <= max_canvas <= 1024");
+  if (!w->emb || !w->w_q || !w->w_k || !w->w_v || !w->w_o || !w->w_lm)
+    return fail(nullptr, DLM_EINVAL, "every weight pointer must be non-NULL");
+
+  dlm_ctx* ctx = new dlm_ctx();
+  ctx->d = d;
+  ctx->bf16 = d.dtype == DLM_BF16;
+  ctx->es = ctx->bf16 ? 2 : 4;
+  cudaGetDevice(&ctx->dev);
+  cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->dev);
+  ctx->Lcap = d.max_prefix + d.max_canvas;
+  ctx->md = ModelDims{d.d_model, d.n_heads, d.n_kv_heads, d.head_dim, d.vocab, d.mask_id,
+                      d.eos_id, ctx->Lcap, (int)ctx->es};
+  ctx->Nqkv = (d.n_heads + 2 * d.n_kv_heads) * d.head_dim;
+  ctx->Mmax = d.max_batch * d.max_canvas;
+  ctx->emb = w->emb;
+  ctx->w_o = w->w_o;
+  ctx->w_lm = w->w_lm;
+  ctx->lens_h.assign(d.max_batch, 0);
+
+  auto bail = [&](int rc) {
+    g_create_error = ctx->msg;
+    dlm_destroy(ctx);
+    return rc;
+  };
+  const size_t es = ctx->es;
+  const size_t dm = d.d_model, qd = (size_t)d.n_heads * d.head_dim;
+  const size_t kv_elems = (size_t)d.max_batch * d.n_kv_heads * ctx->Lcap * d.head_dim;
+  int rc = DLM_OK;
+  if ((rc = dalloc(ctx, &ctx->w_qkv, (size_t)ctx->Nqkv * dm * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->kc, kv_elems * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->vc, kv_elems * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->lens_d, d.max_batch * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->x, ctx->Mmax * dm * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->q, ctx->Mmax * qd * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->o, ctx->Mmax * qd * es))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->y, ctx->Mmax * dm * es))) return bail(rc);
+  const int lm_tile = ctx->bf16 ? 128 : 64;
+  if ((rc = dalloc(ctx, &ctx->lmpart, (size_t)ctx->Mmax * cdiv(d.vocab, lm_tile) * sizeof(LmPart))))
+    return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->cand, ctx->Mmax * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->conf, ctx->Mmax * sizeof(float)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->ent, ctx->Mmax * sizeof(float)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->rope, (size_t)ctx->Lcap * (d.head_dim / 2) * sizeof(float2))))
+    return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->n_active, 2 * sizeof(int)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->err, sizeof(int)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_tok, ctx->Mmax * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_com, ctx->Mmax))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_step, d.max_batch * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_done, d.max_batch))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_eos, d.max_batch * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_stats, d.max_batch * sizeof(dlm_canvas_stats)))) return bail(rc);
+  ctx->part_floats = part_floats_needed(ctx);
+  if ((rc = dalloc(ctx, &ctx->part, ctx->part_floats * sizeof(float)))) return bail(rc);
+
+  cudaError_t e = cudaSuccess;
+  auto ck = [&](cudaError_t r, const char* what) {
+    if (r != cudaSuccess && e == cudaSuccess) {
+      e = r;
+      cuda_fail(ctx, what, r);
+    }
+  };
+  ck(cudaMemset(ctx->kc, 0, kv_elems * es), "memset K cache");
+  ck(cudaMemset(ctx->vc, 0, kv_elems * es), "memset V cache");
+  ck(cudaMemset(ctx->lens_d, 0, d.max_batch * sizeof(int32_t)), "memset lens");
+  ck(cudaMemset(ctx->x, 0, ctx->Mmax * dm * es), "memset x");
+  ck(cudaMemset(ctx->o, 0, ctx->Mmax * qd * es), "memset o");
+  ck(cudaMemset(ctx->y, 0, ctx->Mmax * dm * es), "memset y");
+  ck(cudaMemset(ctx->err, 0, sizeof(int)), "memset err");
+  // fused [W_q ; W_k ; W_v]
+  const size_t qb = qd * dm * es, kvb = (size_t)d.n_kv_heads * d.head_dim * dm * es;
+  ck(cudaMemcpy(ctx->w_qkv, w->w_q, qb, cudaMemcpyDeviceToDevice), "copy w_q");
+  ck(cudaMemcpy((uint8_t*)ctx->w_qkv + qb, w->w_k, kvb, cudaMemcpyDeviceToDevice), "copy w_k");
+  ck(cudaMemcpy((uint8_t*)ctx->w_qkv + qb + kvb, w->w_v, kvb, cudaMemcpyDeviceToDevice),
+     "copy w_v");
+  if (d.rope_theta > 0.0f)
+    ck(rope_table_init(ctx->rope, ctx->Lcap, d.head_dim, (double)d.rope_theta, nullptr),
+       "rope table");
+  ck(cudaStreamCreateWithFlags(&ctx->cap, cudaStreamNonBlocking), "capture stream");
+  ck(cudaDeviceSynchronize(), "create sync");
+  if (e != cudaSuccess) return bail(DLM_ECUDA);
+  if (ctx->bf16) {
+    const uint64_t planes = (uint64_t)d.max_batch * d.n_kv_heads;
+    if (!map_kv(&ctx->tmK, ctx->kc, planes, ctx->Lcap, d.head_dim) ||
+        !map_kv(&ctx->tmV, ctx->vc, planes, ctx->Lcap, d.head_dim))
+      return bail(fail(ctx, DLM_ECUDA, "cuTensorMapEncodeTiled (KV cache) failed"));
+  }
+  *out = ctx;
+  return DLM_OK;
+}
+
+void dlm_destroy(dlm_ctx* ctx) {
+  if (ctx == nullptr) return;
+  cudaDeviceSynchronize();
+  destroy_graphs(ctx);
+  if (ctx->cap) cudaStreamDestroy(ctx->cap);
+  for (void* p : ctx->owned) cudaFree(p);
+  delete ctx;
+}
+
+int dlm_kv_append(dlm_ctx* ctx, int seq, int n, const int32_t* tokens, const void* k,
+                  const void* v, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (seq < 0 || seq >= ctx->d.max_batch) return fail(ctx, DLM_EINVAL, "seq out of range");
+  if (n < 0) return fail(ctx, DLM_EINVAL, "n must be >= 0");
+  if (n == 0) return DLM_OK;
+  if ((long)ctx->lens_h[seq] + n > ctx->d.max_prefix)
+    return fail(ctx, DLM_ECAP, "KV capacity exceeded");
+  cudaStream_t st = (cudaStream_t)stream;
+  const ModelDims& md = ctx->md;
+  if (tokens == nullptr) {
+    if (k == nullptr || v == nullptr) return fail(ctx, DLM_EINVAL, "need tokens or k and v");
+    CK(kv_copy_in(md, seq, n, k, v, ctx->lens_d, ctx->kc, ctx->vc, st));
+    CK(add_len(ctx->lens_d, seq, n, st));
+  } else {
+    const int Nkv = 2 * md.Hkv * md.Dh;
+    const void* wkv = (const uint8_t*)ctx->w_qkv + (size_t)md.H * md.Dh * md.d * ctx->es;
+    for (int j0 = 0; j0 < n; j0 += ctx->Mmax) {
+      const int rows = std::min(ctx->Mmax, n - j0);
+      CK(embed_rows(md, tokens + j0, ctx->emb, ctx->x, rows, rows, 1, nullptr, nullptr, ctx->err,
+                    st));
+      GemmPlan pl = plan_gemm(ctx, rows, Nkv, md.d, EPI_F32);
+      GemmIO io;
+      io.out = ctx->part;
+      io.err = ctx->err;
+      if (int rc = run_gemm(ctx, ctx->x, wkv, Nkv, pl, io, st)) return rc;
+      CK(qkv_epilogue(md, ctx->part, pl.splits, rows, rows, seq, md.H, ctx->lens_d, ctx->rope,
+                      nullptr, ctx->kc, ctx->vc, nullptr, nullptr, st));
+      CK(add_len(ctx->lens_d, seq, rows, st));
+    }
+  }
+  ctx->lens_h[seq] += n;
+  return DLM_OK;
+}
+
+int dlm_reset_kv(dlm_ctx* ctx, int seq) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (seq < 0 || seq >= ctx->d.max_batch) return fail(ctx, DLM_EINVAL, "seq out of range");
+  ctx->lens_h[seq] = 0;
+  CK(cudaMemset(ctx->lens_d + seq, 0, sizeof(int32_t)));
+  return DLM_OK;
+}
+
+int dlm_kv_length(const dlm_ctx* ctx, int seq) {
+  if (ctx == nullptr || seq < 0 || seq >= ctx->d.max_batch) return DLM_EINVAL;
+  return ctx->lens_h[seq];
+}
+
+int dlm_canvas_init(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                    void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c)) return rc;
+  CK(canvas_init(ctx->md, batch, p->canvas, p->corruption, p->seed, c->tokens, c->committed,
+                 c->step, c->done, c->eos_pos, (cudaStream_t)stream));
+  return DLM_OK;
+}
+
+int dlm_denoise_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                     dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c)) return rc;
+  AttnPlan ap = plan_attention(ctx, batch, p->canvas, max_len(ctx, batch) + p->canvas);
+  if (ctx->bf16)
+    if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
+  ctx->launches = 0;
+  return enqueue_step(ctx, c, batch, p, stats, ap, (cudaStream_t)stream);
+}
+
+int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                     dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c)) return rc;
+  AttnPlan ap = plan_attention(ctx, batch, p->canvas, max_len(ctx, batch) + p->canvas);
+  if (ctx->bf16)
+    if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
+  // the graph bakes in pointers, sizes, parameters and the attention plan
+  std::vector<uint8_t> key(sizeof(int) * 4 + sizeof(dlm_sampler_params) + sizeof(dlm_canvas) +
+                           sizeof(void*) * 3 + ctx->ev.size() * sizeof(cudaEvent_t));
+  uint8_t* kp = key.data();
+  const int hdr[4] = {batch, ap.chunk, ap.nsplit, ctx->ev_stage};
+  const void* ptrs[3] = {stats, ctx->opart, ctx->ml};
+  std::memcpy(kp, hdr, sizeof(hdr));
+  kp += sizeof(hdr);
+  dlm_sampler_params pc = *p;
+  std::memcpy(kp, &pc, sizeof(pc));
+  kp += sizeof(pc);
+  std::memcpy(kp, c, sizeof(*c));
+  kp += sizeof(*c);
+  std::memcpy(kp, ptrs, sizeof(ptrs));
+  kp += sizeof(ptrs);
+  if (!ctx->ev.empty()) std::memcpy(kp, ctx->ev.data(), ctx->ev.size() * sizeof(cudaEvent_t));
+  GraphEntry* ge = nullptr;
+  for (auto& g : ctx->graphs)
+    if (g.key == key) ge = &g;
+  if (ge == nullptr) {
+    if (ctx->graphs.size() >= 8) {
+      cudaGraphExecDestroy(ctx->graphs.front().exec);
+      ctx->graphs.erase(ctx->graphs.begin());
+    }
+    cudaGraph_t graph = nullptr;
+    CK(cudaStreamBeginCapture(ctx->cap, cudaStreamCaptureModeThreadLocal));
+    ctx->launches = 0;
+    ctx->ev_step = 0;
+    int rc = DLM_OK;
+    for (int s = 0; s < p->steps && rc == DLM_OK; ++s)
+      rc = enqueue_step(ctx, c, batch, p, stats, ap, ctx->cap);
+    cudaError_t ce = cudaStreamEndCapture(ctx->cap, &graph);
+    if (rc != DLM_OK) {
+      if (graph) cudaGraphDestroy(graph);
+      return rc;
+    }
+    if (ce != cudaSuccess) return cuda_fail(ctx, "cudaStreamEndCapture", ce);
+    GraphEntry g;
+    g.key = key;
+    g.launches = ctx->launches / p->steps;
+    ce = cudaGraphInstantiate(&g.exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ce != cudaSuccess) return cuda_fail(ctx, "cudaGraphInstantiate", ce);
+    ctx->graphs.push_back(g);
+    ge = &ctx->graphs.back();
+  }
+  ctx->launches = ge->launches;
+  CK(cudaGraphLaunch(ge->exec, (cudaStream_t)stream));
+  return DLM_OK;
+}
+
+int dlm_decode_block_host(dlm_ctx* ctx, int32_t* tokens, uint8_t* committed, int32_t* step,
+                          uint8_t* done, int32_t* eos_pos, int batch,
+                          const dlm_sampler_params* p, dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (!tokens || !committed || !step || !done || !eos_pos)
+    return fail(ctx, DLM_EINVAL, "host canvas buffers must be non-NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t n = (size_t)batch * p->canvas;
+  CK(cudaMemcpyAsync(ctx->h_tok, tokens, n * sizeof(int32_t), cudaMemcpyHostToDevice, st));
+  CK(cudaMemcpyAsync(ctx->h_com, committed, n, cudaMemcpyHostToDevice, st));
+  CK(cudaMemcpyAsync(ctx->h_step, step, batch * sizeof(int32_t), cudaMemcpyHostToDevice, st));
+  CK(cudaMemcpyAsync(ctx->h_done, done, batch, cudaMemcpyHostToDevice, st));
+  CK(cudaMemcpyAsync(ctx->h_eos, eos_pos, batch * sizeof(int32_t), cudaMemcpyHostToDevice, st));
+  if (stats)
+    CK(cudaMemcpyAsync(ctx->h_stats, stats, batch * sizeof(dlm_canvas_stats),
+                       cudaMemcpyHostToDevice, st));
+  dlm_canvas c{ctx->h_tok, ctx->h_com, ctx->h_step, ctx->h_done, ctx->h_eos};
+  const std::string keep = ctx->msg;
+  if (int rc = dlm_decode_block(ctx, &c, batch, p, stats ? ctx->h_stats : nullptr, stream))
+    return rc;
+  CK(cudaMemcpyAsync(tokens, ctx->h_tok, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(committed, ctx->h_com, n, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(step, ctx->h_step, batch * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(done, ctx->h_done, batch, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(eos_pos, ctx->h_eos, batch * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  if (stats)
+    CK(cudaMemcpyAsync(stats, ctx->h_stats, batch * sizeof(dlm_canvas_stats),
+                       cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  return DLM_OK;
+}
+
+int dlm_commit(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+               const int32_t* cand, const float* conf, const float* entropy,
+               dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c)) return rc;
+  if (!cand || !conf || !entropy) return fail(ctx, DLM_EINVAL, "cand/conf/entropy NULL");
+  CK(commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
+                 c->eos_pos, cand, conf, entropy, stats, nullptr, ctx->err,
+                 (cudaStream_t)stream));
+  return DLM_OK;
+}
+
+int dlm_debug_buffer(dlm_ctx* ctx, int which, void** ptr, size_t* bytes) {
+  if (ctx == nullptr || ptr == nullptr || bytes == nullptr) return DLM_EINVAL;
+  const size_t M = ctx->Mmax, es = ctx->es, dm = ctx->d.d_model;
+  const size_t qd = (size_t)ctx->d.n_heads * ctx->d.head_dim;
+  const size_t kv = (size_t)ctx->d.max_batch * ctx->d.n_kv_heads * ctx->Lcap * ctx->d.head_dim;
+  switch (which) {
+    case DLM_BUF_X: *ptr = ctx->x; *bytes = M * dm * es; break;
+    case DLM_BUF_Q: *ptr = ctx->q; *bytes = M * qd * es; break;
+    case DLM_BUF_O: *ptr = ctx->o; *bytes = M * qd * es; break;
+    case DLM_BUF_Y: *ptr = ctx->y; *bytes = M * dm * es; break;
+    case DLM_BUF_CAND: *ptr = ctx->cand; *bytes = M * 4; break;
+    case DLM_BUF_CONF: *ptr = ctx->conf; *bytes = M * 4; break;
+    case DLM_BUF_ENTROPY: *ptr = ctx->ent; *bytes = M * 4; break;
+    case DLM_BUF_K_CACHE: *ptr = ctx->kc; *bytes = kv * es; break;
+    case DLM_BUF_V_CACHE: *ptr = ctx->vc; *bytes = kv * es; break;
+    default: return fail(ctx, DLM_EINVAL, "unknown buffer id");
+  }
+  return DLM_OK;
+}
+
+int dlm_debug_logits(dlm_ctx* ctx, int batch, int canvas, float* logits, void* stream) {
+  if (ctx == nullptr || logits == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (batch < 1 || canvas < 1 || (long)batch * canvas > ctx->Mmax)
+    return fail(ctx, DLM_EINVAL, "batch * canvas out of range");
+  const int rows = batch * canvas;
+  GemmPlan pl = plan_gemm(ctx, rows, ctx->d.vocab, ctx->d.d_model, EPI_LM);
+  pl.epi = EPI_F32;
+  pl.splits = 1;
+  GemmIO io;
+  io.out = logits;
+  io.err = ctx->err;
+  return run_gemm(ctx, ctx->y, ctx->w_lm, ctx->d.vocab, pl, io, (cudaStream_t)stream);
+}
+
+int dlm_check(dlm_ctx* ctx, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  CK(cudaStreamSynchronize((cudaStream_t)stream));
+  int word = 0;
+  CK(cudaMemcpy(&word, ctx->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word != 0) {
+    CK(cudaMemset(ctx->err, 0, sizeof(int)));
+    return fail(ctx, word, word == DLM_ETIMEOUT ? "device wait timed out"
+                                                : "device index check failed");
+  }
+  return DLM_OK;
+}
+
+int dlm_launches_per_step(const dlm_ctx* ctx) { return ctx ? ctx->launches : DLM_EINVAL; }
+
+int dlm_set_stage_events(dlm_ctx* ctx, int stage, void* const* events, int n_pairs) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (stage < 0 || stage >= DLM_NUM_STAGES || n_pairs < 0 || (n_pairs > 0 && events == nullptr))
+    return fail(ctx, DLM_EINVAL, "bad stage or event array");
+  ctx->ev.clear();
+  ctx->ev_stage = n_pairs > 0 ? stage : -1;
+  for (int i = 0; i < 2 * n_pairs; ++i) ctx->ev.push_back((cudaEvent_t)events[i]);
+  ctx->ev_step = 0;
+  return DLM_OK;
+}
+
+const char* dlm_last_error(const dlm_ctx* ctx) {
+  return ctx ? ctx->msg.c_str() : g_create_error.c_str();
+}
+
+}  // extern "C"

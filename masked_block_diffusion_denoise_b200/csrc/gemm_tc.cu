@@ -1,0 +1,304 @@
+// tcgen05 GEMM engine for sm_100a: D[M][N] = A[M][K] . B[N][K]^T, bf16
+// operands (both K-major, row-major in HBM), f32 accumulators in tensor
+// memory.
+//
+// One persistent CTA per SM, three roles:
+//   warp 0      TMA producer: streams 128x64 A and BNx64 B tiles (128-byte
+//               swizzle) into a STAGES-deep shared-memory ring;
+//   warp 1      MMA issuer: one thread issues tcgen05.mma 128xBNx16 into one
+//               of two TMEM accumulators and frees ring slots with
+//               tcgen05.commit;
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (one TMEM lane = one
+//               output row per thread) while the MMA warp fills the other
+//               accumulator.
+// Work units are (m tile, n tile, k split), m fastest, so that CTAs that run
+// at the same time share the same B (weight) slab through L2.
+//
+// Epilogues:
+//   EPI_F32  store f32 partial sums [split][M][N] (projections, split-K;
+//            full logits for inspection);
+//   EPI_LM   the LM head's fused vocabulary reduction: per (row, n tile) one
+//            LmPart; logits never leave the SM.
+#include <cstdio>
+
+#include "kernels.h"
+#include "lm_epilogue.cuh"
+
+namespace dlm {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 per row
+
+template <int BN>
+struct TcCfg {
+  static constexpr int kStages = (BN == 128) ? 6 : 4;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct TcParams {
+  int M, N, K;
+  int m_tiles, n_tiles, splits, units, kblocks;
+  float* out;
+  LmPart* part;
+  LmEpi epi;
+  const uint8_t* done;   // [B] canvases that are finished (LM rows skipped)
+  const int* n_active;   // whole launch skipped when *n_active == 0
+  int* err;
+};
+
+__device__ __forceinline__ void unit_coords(const TcParams& p, int u, int& m, int& n, int& kb0,
+                                            int& kb1) {
+  m = u % p.m_tiles;
+  const int rest = u / p.m_tiles;
+  n = rest % p.n_tiles;
+  const int split = rest / p.n_tiles;
+  kb0 = (int)(((long long)split * p.kblocks) / p.splits);
+  kb1 = (int)(((long long)(split + 1) * p.kblocks) / p.splits);
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcParams p) {
+  using Cfg = TcCfg<BN>;
+  if (p.n_active != nullptr && *p.n_active == 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kStages * Cfg::kStageBytes);
+  uint64_t* empty = full + Cfg::kStages;
+  uint64_t* tfull = empty + Cfg::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, Cfg::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int m, n, kb0, kb1;
+        unit_coords(p, u, m, n, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * Cfg::kStageBytes;
+          uint8_t* sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+          tma_load_2d(sa, &tmA, &full[stage], kb * kBK, m * kBM);
+          tma_load_2d(sb, &tmB, &full[stage], kb * kBK, n * BN);
+          ++issued;
+          if (++stage == Cfg::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land before the CTA exits
+        int st = stage, ph = phase;
+        for (int i = 0; i < Cfg::kStages && i < issued; ++i) {
+          if (--st < 0) {
+            st = Cfg::kStages - 1;
+            ph ^= 1;
+          }
+          mbar_wait_bounded(&full[st], (uint32_t)ph, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int m, n, kb0, kb1;
+        unit_coords(p, u, m, n, kb0, kb1);
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
+          const uint32_t sb = sa + Cfg::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            umma_bf16(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
+                      (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == Cfg::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // every MMA issued has completed before TMEM is released
+      umma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+      int m, n, kb0, kb1;
+      unit_coords(p, u, m, n, kb0, kb1);
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const int row0 = m * kBM + quad * 32;
+      const int row = row0 + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      if (row0 < p.M) {   // warp-uniform: tcgen05.ld is a warp-wide instruction
+        if constexpr (EPI == EPI_F32) {
+          const int split = (u / p.m_tiles) / p.n_tiles;
+          float* orow = p.out + ((size_t)split * p.M + row) * p.N;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            tmem_ld32(taddr + c, v);
+            const int col0 = n * BN + c;
+            if (row < p.M) {
+              if (col0 + 32 <= p.N) {
+                float4* dst = reinterpret_cast<float4*>(orow + col0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              } else {
+                for (int j = 0; j < 32; ++j)
+                  if (col0 + j < p.N) orow[col0 + j] = v[j];
+              }
+            }
+          }
+        } else {
+          const int canvas = row / p.epi.C;
+          const int pos = row - canvas * p.epi.C;
+          const bool live = row < p.M && (p.done == nullptr || p.done[canvas] == 0);
+          const int step = live ? p.epi.step[canvas] : 0;
+          const float inv_t = lm_inv_temp(p.epi, step);
+          RowState rs;
+          rs_init(rs);
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            tmem_ld32(taddr + c, v);
+            if (live) rs_update<32>(rs, v, n * BN + c, inv_t, p.epi, canvas, pos, step);
+          }
+          if (live) rs_store(p.part + (size_t)row * p.epi.n_tiles + n, rs);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
+}
+
+template <int BN, int EPI>
+cudaError_t launch_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const TcParams& p,
+                      int num_sms, cudaStream_t st) {
+  using Cfg = TcCfg<BN>;
+  static bool attr_set = false;   // per process; one device is used per process
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = p.units < num_sms ? p.units : num_sms;
+  gemm_tc_kernel<BN, EPI><<<grid, 192, Cfg::kSmem, st>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPlan& plan,
+                    const GemmIO& io, int num_sms, cudaStream_t st) {
+  TcParams p{};
+  p.M = plan.M;
+  p.N = plan.N;
+  p.K = plan.K;
+  p.m_tiles = (plan.M + kBM - 1) / kBM;
+  p.n_tiles = (plan.N + plan.BN - 1) / plan.BN;
+  p.splits = plan.splits;
+  p.kblocks = (plan.K + kBK - 1) / kBK;
+  p.units = p.m_tiles * p.n_tiles * p.splits;
+  p.out = io.out;
+  p.part = io.part;
+  p.epi = io.epi;
+  p.epi.n_tiles = p.n_tiles;
+  p.done = io.done;
+  p.n_active = io.n_active;
+  p.err = io.err;
+  if (plan.BN == 128) {
+    return plan.epi == EPI_LM ? launch_tc<128, EPI_LM>(tmA, tmB, p, num_sms, st)
+                              : launch_tc<128, EPI_F32>(tmA, tmB, p, num_sms, st);
+  }
+  return plan.epi == EPI_LM ? launch_tc<256, EPI_LM>(tmA, tmB, p, num_sms, st)
+                            : launch_tc<256, EPI_F32>(tmA, tmB, p, num_sms, st);
+}
+
+int gemm_tc_smem_bytes(int BN) { return BN == 128 ? TcCfg<128>::kSmem : TcCfg<256>::kSmem; }
+
+}  // namespace dlm

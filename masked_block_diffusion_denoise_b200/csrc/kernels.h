@@ -1,0 +1,117 @@
+// Host-side launchers of the library's kernels (one per .cu file section).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lm_epilogue.cuh"
+
+namespace dlm {
+
+enum { EPI_F32 = 0, EPI_LM = 1 };
+
+struct GemmPlan {
+  int M, N, K;
+  int BN;       // 128 or 256 (tcgen05); 64 (fp32 SIMT)
+  int splits;   // K splits (EPI_F32 only)
+  int epi;      // EPI_F32 / EPI_LM
+};
+
+struct GemmIO {
+  float* out = nullptr;        // EPI_F32: [splits][M][N]
+  LmPart* part = nullptr;      // EPI_LM:  [M][n_tiles]
+  LmEpi epi{};
+  const uint8_t* done = nullptr;
+  const int* n_active = nullptr;
+  int* err = nullptr;
+};
+
+// ---- gemm_tc.cu: bf16 tcgen05 GEMM ---------------------------------------
+cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPlan& plan,
+                    const GemmIO& io, int num_sms, cudaStream_t st);
+int gemm_tc_smem_bytes(int BN);
+
+// ---- gemm_simt.cu: fp32 GEMM on the CUDA cores (fp32 model) ----------------
+cudaError_t gemm_f32(const float* A, const float* B, const GemmPlan& plan, const GemmIO& io,
+                     cudaStream_t st);
+
+// ---- misc.cu: embedding, projection epilogues, cache writes, canvas init --
+struct ModelDims {
+  int d, H, Hkv, Dh, V, mask_id, eos_id;
+  int Lcap;      // KV slots per (sequence, KV head)
+  int esize;     // element bytes
+};
+
+cudaError_t rope_table_init(float2* table, int Lcap, int Dh, double theta, cudaStream_t st);
+
+// x[r] = E[tokens[r]] for r < rows; skips rows of finished canvases; block 0
+// also writes *n_active = number of unfinished canvases (done may be null)
+cudaError_t embed_rows(const ModelDims& md, const int32_t* tokens, const void* emb, void* x,
+                       int rows, int C, int B, const uint8_t* done, int* n_active, int* err,
+                       cudaStream_t st);
+
+// Sum split-K partials of the fused QKV projection, rotate q and k, store q
+// ([rows][H][Dh]) and k, v into the cache at slot lens[seq] + position.
+// Row r is (seq = r / C, position = r % C) or, with seq_fixed >= 0, (seq_fixed,
+// position = r).  head0 = first head of the partial columns (0: q, k, v;
+// H: k, v only).
+cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
+                         int seq_fixed, int head0, const int32_t* lens, const float2* rope,
+                         void* q, void* kcache, void* vcache, const uint8_t* done,
+                         const int* n_active, cudaStream_t st);
+
+// y = x + sum of split-K partials of o W_o^T
+cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
+                        const void* x, void* y, const uint8_t* done, const int* n_active,
+                        cudaStream_t st);
+
+// copy caller K/V [Hkv][n][Dh] into the cache of `seq` at slots lens[seq]..
+cudaError_t kv_copy_in(const ModelDims& md, int seq, int n, const void* k, const void* v,
+                       const int32_t* lens, void* kcache, void* vcache, cudaStream_t st);
+
+cudaError_t add_len(int32_t* lens, int seq, int n, cudaStream_t st);
+
+cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint64_t seed,
+                        int32_t* tokens, uint8_t* committed, int32_t* step, uint8_t* done,
+                        int32_t* eos_pos, cudaStream_t st);
+
+// ---- attention.cu ------------------------------------------------------------
+struct AttnPlan {
+  int B, C, G, R, rtiles;   // G = H / Hkv, R = G * C query rows per (seq, kv head)
+  int chunk, nsplit;        // keys per split (multiple of 64), splits per (seq, kv head)
+};
+
+// bf16: TMA-fed mma.sync flash attention over [prefix ; canvas] keys, split-KV
+cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const void* q, void* o, float* opart,
+                           float2* ml, const int32_t* lens, const uint8_t* done,
+                           const int* n_active, int* err, cudaStream_t st);
+// fp32: one thread per query row
+cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,
+                          const float* vcache, float* o, const int32_t* lens,
+                          const uint8_t* done, const int* n_active, cudaStream_t st);
+
+// ---- select.cu ------------------------------------------------------------------
+// combine LM partials of each row into candidate, confidence and entropy
+cudaError_t lm_reduce(const LmPart* part, int rows, int n_tiles, int C, const uint8_t* done,
+                      const int* n_active, int32_t* cand, float* conf, float* ent,
+                      cudaStream_t st);
+
+struct SelectArgs {
+  int B, C, S, V;
+  int quota;             // effective quota (>= 1)
+  float threshold;
+  int eb;                // entropy-bound rule
+  float bound;
+  int uniform;           // re-noise with uniform ids
+  int mask_id, eos_id;
+  uint32_t seed_lo, seed_hi;
+};
+
+cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
+                        uint8_t* done, int32_t* eos_pos, const int32_t* cand, const float* conf,
+                        const float* ent, dlm_canvas_stats* stats, const int* n_active,
+                        int* err, cudaStream_t st);
+
+}  // namespace dlm

@@ -1,0 +1,176 @@
+// Fused vocabulary reduction of the LM head (non-materialised scoring, the
+// "chunked" head scoring of the Nemotron guide, section 5.3): each GEMM tile
+// of logits is reduced, per row, to
+//   m  = max z, s = sum e^(z-m), t = sum e^(z-m) (z-m)
+//   (g, idx, zw): the winning column -- the argmax of z (greedy, lowest index
+//   on ties) or of z + Gumbel noise (sampling) -- and its scaled logit,
+// with z = logit / T (T = 1 for greedy) and the mask id excluded.  Partials of
+// all tiles of a row are combined afterwards; confidence = e^(zw - M) / S and
+// entropy H = log S - T/S (nats).
+#pragma once
+
+#include <math_constants.h>
+
+#include "common.cuh"
+
+namespace dlm {
+
+struct LmPart {
+  float m, s, t, g, zw;
+  int idx;
+};
+
+enum { LM_GREEDY = 0, LM_SAMPLE_FIXED = 1, LM_SAMPLE_ANNEAL = 2 };
+
+struct LmEpi {
+  int V;          // vocabulary (columns >= V are excluded)
+  int mask_id;    // excluded column, < 0 for none
+  int C;          // canvas length: row r is position r % C of canvas r / C
+  int S;          // step budget (anneal)
+  int mode;       // LM_GREEDY / LM_SAMPLE_FIXED / LM_SAMPLE_ANNEAL
+  float inv_temp; // LM_SAMPLE_FIXED
+  float t_max, t_min;
+  uint32_t seed_lo, seed_hi;
+  const int32_t* step;   // [B] steps taken (sampling counter and anneal)
+  int n_tiles;    // partials per row
+};
+
+struct RowState {
+  float m, s, t, g, zw;
+  int idx;
+};
+
+__device__ __forceinline__ void rs_init(RowState& r) {
+  r.m = -CUDART_INF_F;
+  r.s = 0.f;
+  r.t = 0.f;
+  r.g = -CUDART_INF_F;
+  r.zw = -CUDART_INF_F;
+  r.idx = 0x7fffffff;
+}
+
+// 1/T of a row, float32 with explicit rounding so that the host can repeat it
+__device__ __forceinline__ float lm_inv_temp(const LmEpi& e, int step) {
+  if (e.mode == LM_SAMPLE_FIXED) return e.inv_temp;
+  if (e.mode == LM_SAMPLE_ANNEAL) {
+    float T = e.t_max;
+    if (e.S > 1) {
+      const float frac = __fdiv_rn((float)step, (float)(e.S - 1));
+      T = __fadd_rn(e.t_max, __fmul_rn(__fsub_rn(e.t_min, e.t_max), frac));
+    }
+    return __frcp_rn(T);
+  }
+  return 1.f;
+}
+
+// Fold N consecutive logits (columns col0 .. col0+N-1, col0 % 4 == 0) of one
+// row into the row state.  canvas / pos / step locate the row for the
+// sampling counter.
+template <int N>
+__device__ __forceinline__ void rs_update(RowState& r, const float (&v)[N], int col0,
+                                          float inv_t, const LmEpi& e, int canvas, int pos,
+                                          int step) {
+  float z[N];
+  float cmax = -CUDART_INF_F;
+  int carg = 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const int col = col0 + j;
+    float zj = (e.mode == LM_GREEDY) ? v[j] : __fmul_rn(v[j], inv_t);
+    if (col >= e.V || col == e.mask_id) zj = -CUDART_INF_F;
+    z[j] = zj;
+    if (zj > cmax) {
+      cmax = zj;
+      carg = j;
+    }
+  }
+  if (cmax == -CUDART_INF_F) return;
+  if (cmax > r.m) {
+    if (r.m != -CUDART_INF_F) {
+      const float a = __expf(r.m - cmax);
+      r.t = (r.t + r.s * (r.m - cmax)) * a;
+      r.s *= a;
+    }
+    r.m = cmax;
+  }
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    if (z[j] != -CUDART_INF_F) {
+      const float d = z[j] - r.m;
+      const float ex = __expf(d);
+      r.s += ex;
+      r.t = fmaf(ex, d, r.t);
+    }
+  }
+  if (e.mode == LM_GREEDY) {
+    // columns arrive in increasing order: on equal values the earlier wins
+    if (cmax > r.g) {
+      r.g = cmax;
+      r.zw = cmax;
+      r.idx = col0 + carg;
+    }
+  } else {
+#pragma unroll
+    for (int j4 = 0; j4 < N; j4 += 4) {
+      const int col = col0 + j4;
+      const U32x4 w = philox10(U32x4{(uint32_t)canvas, (uint32_t)step, (uint32_t)pos,
+                                     (uint32_t)(col >> 2)},
+                               e.seed_lo, e.seed_hi);
+      const uint32_t ws[4] = {w.a, w.b, w.c, w.d};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float zj = z[j4 + q];
+        if (zj == -CUDART_INF_F) continue;
+        const float gj = zj + gumbel_from_bits(ws[q]);
+        if (gj > r.g) {
+          r.g = gj;
+          r.zw = zj;
+          r.idx = col + q;
+        }
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void rs_store(LmPart* dst, const RowState& r) {
+  LmPart p;
+  p.m = r.m;
+  p.s = r.s;
+  p.t = r.t;
+  p.g = r.g;
+  p.zw = r.zw;
+  p.idx = r.idx;
+  *dst = p;
+}
+
+// combine two partial states (the order of arguments fixes the tie rule:
+// equal winners keep the lower index)
+__device__ __forceinline__ RowState rs_combine(const RowState& a, const RowState& b) {
+  RowState c;
+  const float M = fmaxf(a.m, b.m);
+  if (M == -CUDART_INF_F) {
+    rs_init(c);
+    return c;
+  }
+  float s = 0.f, t = 0.f;
+  if (a.m != -CUDART_INF_F) {
+    const float w = __expf(a.m - M);
+    s += a.s * w;
+    t += (a.t + a.s * (a.m - M)) * w;
+  }
+  if (b.m != -CUDART_INF_F) {
+    const float w = __expf(b.m - M);
+    s += b.s * w;
+    t += (b.t + b.s * (b.m - M)) * w;
+  }
+  c.m = M;
+  c.s = s;
+  c.t = t;
+  const bool take_b = (b.g > a.g) || (b.g == a.g && b.idx < a.idx);
+  c.g = take_b ? b.g : a.g;
+  c.zw = take_b ? b.zw : a.zw;
+  c.idx = take_b ? b.idx : a.idx;
+  return c;
+}
+
+}  // namespace dlm

@@ -1,0 +1,230 @@
+// Element-wise kernels around the GEMMs: RoPE table, embedding gather, the
+// projection epilogues (split-K sum, rotary embedding, KV-cache write,
+// residual), KV copy-in and canvas initialisation.
+#include "kernels.h"
+
+namespace dlm {
+namespace {
+
+// cos/sin of pos * theta^(-2j/Dh), evaluated in double precision (positions
+// reach 32k+, where a float32 angle would already be off by ~1e-3 rad)
+__global__ void rope_table_kernel(float2* table, int Lcap, int half, double theta) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)Lcap * half) return;
+  const int pos = (int)(i / half), j = (int)(i % half);
+  const double inv_freq = pow(theta, -2.0 * (double)j / (double)(2 * half));
+  double s, c;
+  sincos((double)pos * inv_freq, &s, &c);
+  table[i] = make_float2((float)c, (float)s);
+}
+
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ emb,
+                             T* __restrict__ x, int rows, int C, int d, int V, int B,
+                             const uint8_t* __restrict__ done, int* n_active, int* err) {
+  if (blockIdx.x == 0 && n_active != nullptr) {
+    __shared__ int cnt;
+    if (threadIdx.x == 0) cnt = 0;
+    __syncthreads();
+    int mine = 0;
+    for (int b = threadIdx.x; b < B; b += blockDim.x) mine += (done == nullptr || !done[b]);
+    atomicAdd(&cnt, mine);
+    __syncthreads();
+    if (threadIdx.x == 0) *n_active = cnt;
+  }
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  if (done != nullptr && done[r / C]) return;
+  int t = tokens[r];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) raise_error(err, DLM_EBOUNDS);
+    t = 0;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(emb + (size_t)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(x + (size_t)r * d);
+  const int n16 = d * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
+}
+
+template <typename T>
+__global__ void qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part, int splits,
+                                    int rows, int C, int seq_fixed, int head0,
+                                    const int32_t* __restrict__ lens,
+                                    const float2* __restrict__ rope, T* __restrict__ q,
+                                    T* __restrict__ kc, T* __restrict__ vc,
+                                    const uint8_t* __restrict__ done, const int* n_active) {
+  if (n_active != nullptr && *n_active == 0) return;
+  const int r = blockIdx.x;
+  const int hh = blockIdx.y + head0;
+  const int j = threadIdx.x;
+  const int half = md.Dh / 2;
+  int seq, p_in;
+  if (seq_fixed >= 0) {
+    seq = seq_fixed;
+    p_in = r;
+  } else {
+    seq = r / C;
+    p_in = r - seq * C;
+    if (done != nullptr && done[seq]) return;
+  }
+  const int pos = lens[seq] + p_in;
+  const int ncols = (md.H + 2 * md.Hkv - head0) * md.Dh;
+  const int cb = (hh - head0) * md.Dh;
+  float a = 0.f, b = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float* pr = part + ((size_t)s * rows + r) * ncols + cb;
+    a += pr[j];
+    b += pr[j + half];
+  }
+  if (rope != nullptr && hh < md.H + md.Hkv) {
+    const float2 cs = rope[(size_t)pos * half + j];
+    const float a2 = a * cs.x - b * cs.y;
+    const float b2 = b * cs.x + a * cs.y;
+    a = a2;
+    b = b2;
+  }
+  T* dst;
+  if (hh < md.H) {
+    dst = q + ((size_t)r * md.H + hh) * md.Dh;
+  } else if (hh < md.H + md.Hkv) {
+    dst = kc + (((size_t)seq * md.Hkv + (hh - md.H)) * md.Lcap + pos) * md.Dh;
+  } else {
+    dst = vc + (((size_t)seq * md.Hkv + (hh - md.H - md.Hkv)) * md.Lcap + pos) * md.Dh;
+  }
+  dst[j] = from_f32<T>(a);
+  dst[j + half] = from_f32<T>(b);
+}
+
+template <typename T>
+__global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, int rows, int d,
+                                   int C, const T* __restrict__ x, T* __restrict__ y,
+                                   const uint8_t* __restrict__ done, const int* n_active) {
+  if (n_active != nullptr && *n_active == 0) return;
+  const int r = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= d) return;
+  if (done != nullptr && done[r / C]) return;
+  float acc = 0.f;
+  for (int s = 0; s < splits; ++s) acc += part[((size_t)s * rows + r) * d + c];
+  const size_t i = (size_t)r * d + c;
+  y[i] = from_f32<T>(to_f32(x[i]) + acc);
+}
+
+template <typename T>
+__global__ void kv_copy_kernel(int Hkv, int Lcap, int Dh, int seq, int n,
+                               const T* __restrict__ k, const T* __restrict__ v,
+                               const int32_t* __restrict__ lens, T* kc, T* vc) {
+  const int g = blockIdx.x, j = blockIdx.y;
+  const int pos = lens[seq] + j;
+  const size_t src = ((size_t)g * n + j) * Dh;
+  const size_t dst = (((size_t)seq * Hkv + g) * Lcap + pos) * Dh;
+  for (int t = threadIdx.x; t < Dh; t += blockDim.x) {
+    kc[dst + t] = k[src + t];
+    vc[dst + t] = v[src + t];
+  }
+}
+
+__global__ void add_len_kernel(int32_t* lens, int seq, int n) { lens[seq] += n; }
+
+__global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint32_t s0,
+                                   uint32_t s1, int32_t* tokens, uint8_t* committed,
+                                   int32_t* step, uint8_t* done, int32_t* eos_pos) {
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    int32_t t = mask_id;
+    if (uniform) {
+      const U32x4 w = philox10(U32x4{(uint32_t)b, 0u, (uint32_t)i, kRenoiseWord}, s0, s1);
+      t = uniform_id(w.a, V);
+    }
+    tokens[(size_t)b * C + i] = t;
+    committed[(size_t)b * C + i] = 0;
+  }
+  if (threadIdx.x == 0) {
+    step[b] = 0;
+    done[b] = 0;
+    eos_pos[b] = -1;
+  }
+}
+
+}  // namespace
+
+cudaError_t rope_table_init(float2* table, int Lcap, int Dh, double theta, cudaStream_t st) {
+  const int64_t n = (int64_t)Lcap * (Dh / 2);
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(table, Lcap, Dh / 2, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t embed_rows(const ModelDims& md, const int32_t* tokens, const void* emb, void* x,
+                       int rows, int C, int B, const uint8_t* done, int* n_active, int* err,
+                       cudaStream_t st) {
+  if (md.esize == 2)
+    embed_kernel<__nv_bfloat16><<<rows, 128, 0, st>>>(
+        tokens, (const __nv_bfloat16*)emb, (__nv_bfloat16*)x, rows, C, md.d, md.V, B, done,
+        n_active, err);
+  else
+    embed_kernel<float><<<rows, 128, 0, st>>>(tokens, (const float*)emb, (float*)x, rows, C,
+                                              md.d, md.V, B, done, n_active, err);
+  return cudaGetLastError();
+}
+
+cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
+                         int seq_fixed, int head0, const int32_t* lens, const float2* rope,
+                         void* q, void* kcache, void* vcache, const uint8_t* done,
+                         const int* n_active, cudaStream_t st) {
+  dim3 grid(rows, md.H + 2 * md.Hkv - head0);
+  if (md.esize == 2)
+    qkv_epilogue_kernel<__nv_bfloat16><<<grid, md.Dh / 2, 0, st>>>(
+        md, part, splits, rows, C, seq_fixed, head0, lens, rope, (__nv_bfloat16*)q,
+        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active);
+  else
+    qkv_epilogue_kernel<float><<<grid, md.Dh / 2, 0, st>>>(
+        md, part, splits, rows, C, seq_fixed, head0, lens, rope, (float*)q, (float*)kcache,
+        (float*)vcache, done, n_active);
+  return cudaGetLastError();
+}
+
+cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
+                        const void* x, void* y, const uint8_t* done, const int* n_active,
+                        cudaStream_t st) {
+  dim3 grid((md.d + 255) / 256, rows);
+  if (md.esize == 2)
+    wo_epilogue_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        part, splits, rows, md.d, C, (const __nv_bfloat16*)x, (__nv_bfloat16*)y, done, n_active);
+  else
+    wo_epilogue_kernel<float><<<grid, 256, 0, st>>>(part, splits, rows, md.d, C,
+                                                    (const float*)x, (float*)y, done, n_active);
+  return cudaGetLastError();
+}
+
+cudaError_t kv_copy_in(const ModelDims& md, int seq, int n, const void* k, const void* v,
+                       const int32_t* lens, void* kcache, void* vcache, cudaStream_t st) {
+  dim3 grid(md.Hkv, n);
+  const int threads = md.Dh < 128 ? md.Dh : 128;
+  if (md.esize == 2)
+    kv_copy_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
+        md.Hkv, md.Lcap, md.Dh, seq, n, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, lens,
+        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache);
+  else
+    kv_copy_kernel<float><<<grid, threads, 0, st>>>(md.Hkv, md.Lcap, md.Dh, seq, n,
+                                                    (const float*)k, (const float*)v, lens,
+                                                    (float*)kcache, (float*)vcache);
+  return cudaGetLastError();
+}
+
+cudaError_t add_len(int32_t* lens, int seq, int n, cudaStream_t st) {
+  add_len_kernel<<<1, 1, 0, st>>>(lens, seq, n);
+  return cudaGetLastError();
+}
+
+cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint64_t seed,
+                        int32_t* tokens, uint8_t* committed, int32_t* step, uint8_t* done,
+                        int32_t* eos_pos, cudaStream_t st) {
+  const int threads = C < 1024 ? ((C + 31) / 32) * 32 : 1024;
+  canvas_init_kernel<<<B, threads, 0, st>>>(C, md.V, md.mask_id, corruption == DLM_UNIFORM,
+                                            (uint32_t)(seed & 0xFFFFFFFFull),
+                                            (uint32_t)(seed >> 32), tokens, committed, step,
+                                            done, eos_pos);
+  return cudaGetLastError();
+}
+
+}  // namespace dlm

@@ -1,0 +1,226 @@
+// Selection half of the step:
+//   lm_reduce    combines the LM head's per-tile partials of every row into
+//                the candidate token, its confidence and the entropy;
+//   commit_step  kernel (c): one CTA per canvas ranks the uncommitted
+//                positions (bitonic sort in shared memory), applies the
+//                threshold + quota rule or the entropy bound, forces
+//                completion on the last step of the budget, handles EOS,
+//                re-noises the rest and advances step / done.
+// The selection follows the DiffusionGemma page (BlockRefinementScheduler,
+// EntropyBoundScheduler), the course "Diffusion LLMs" section 12 (confidence
+// order, ties to the lower position) and the Nemotron guide, section 6 (the
+// last step fills every remaining mask).
+#include "kernels.h"
+
+namespace dlm {
+namespace {
+
+__global__ void lm_reduce_kernel(const LmPart* __restrict__ part, int rows, int n_tiles, int C,
+                                 const uint8_t* __restrict__ done, const int* n_active,
+                                 int32_t* __restrict__ cand, float* __restrict__ conf,
+                                 float* __restrict__ ent) {
+  if (n_active != nullptr && *n_active == 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  if (done != nullptr && done[row / C]) return;
+  RowState acc;
+  rs_init(acc);
+  const LmPart* pr = part + (size_t)row * n_tiles;
+  for (int j = lane; j < n_tiles; j += 32) {
+    const LmPart q = pr[j];
+    RowState x{q.m, q.s, q.t, q.g, q.zw, q.idx};
+    acc = rs_combine(acc, x);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    RowState o;
+    o.m = __shfl_xor_sync(0xffffffffu, acc.m, off);
+    o.s = __shfl_xor_sync(0xffffffffu, acc.s, off);
+    o.t = __shfl_xor_sync(0xffffffffu, acc.t, off);
+    o.g = __shfl_xor_sync(0xffffffffu, acc.g, off);
+    o.zw = __shfl_xor_sync(0xffffffffu, acc.zw, off);
+    o.idx = __shfl_xor_sync(0xffffffffu, acc.idx, off);
+    acc = rs_combine(acc, o);   // symmetric: every lane ends with the same value
+  }
+  if (lane == 0) {
+    if (acc.idx == 0x7fffffff || !(acc.s > 0.f)) {
+      cand[row] = 0;
+      conf[row] = 0.f;
+      ent[row] = 0.f;
+    } else {
+      cand[row] = acc.idx;
+      conf[row] = expf(acc.zw - acc.m) / acc.s;
+      ent[row] = logf(acc.s) - acc.t / acc.s;
+    }
+  }
+}
+
+// float -> unsigned key with the same order (-0.0 folded onto +0.0)
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t u = __float_as_uint(x + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int kMaxC = 1024;
+
+// positions after the first committed EOS become EOS and committed; returns
+// the EOS position (or -1) and, through *filled, how many were filled
+__device__ int eos_fill(int32_t* tok, uint8_t* com, int C, int eos_id, int* e_s, int* filled) {
+  const int i = threadIdx.x;
+  if (eos_id < 0) {
+    *filled = 0;
+    return -1;
+  }
+  if (i == 0) *e_s = C;
+  __syncthreads();
+  if (i < C && com[i] && tok[i] == eos_id) atomicMin(e_s, i);
+  __syncthreads();
+  const int e = *e_s;
+  const bool f = (i < C && i > e && !com[i]);
+  if (f) {
+    tok[i] = eos_id;
+    com[i] = 1;
+  }
+  *filled = __syncthreads_count(f);
+  return e < C ? e : -1;
+}
+
+__global__ void commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
+                              uint8_t* __restrict__ committed, int32_t* __restrict__ step,
+                              uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
+                              const int32_t* __restrict__ cand, const float* __restrict__ conf,
+                              const float* __restrict__ ent, dlm_canvas_stats* stats,
+                              const int* n_active, int* err) {
+  if (n_active != nullptr && *n_active == 0) return;
+  const int b = blockIdx.x;
+  if (done[b]) return;
+  __shared__ unsigned long long keys[kMaxC];
+  __shared__ int32_t tok[kMaxC];
+  __shared__ uint8_t com[kMaxC];
+  __shared__ int e_s, k_s, krule_s;
+  const int i = threadIdx.x;
+  const int P = blockDim.x;
+  const int C = a.C;
+  const size_t base = (size_t)b * C;
+  const int s = step[b];
+  if (i < C) {
+    tok[i] = tokens[base + i];
+    com[i] = committed[base + i];
+  }
+  __syncthreads();
+
+  int fill0 = 0, fill1 = 0;
+  eos_fill(tok, com, C, a.eos_id, &e_s, &fill0);
+
+  const bool open = (i < C) && !com[i];
+  unsigned long long key = ~0ull;
+  if (open) {
+    const uint32_t hi = a.eb ? ordered_bits(ent[base + i]) : ~ordered_bits(conf[base + i]);
+    key = ((unsigned long long)hi << 32) | (unsigned)i;
+  }
+  keys[i] = key;
+  const int nU = __syncthreads_count(open);
+  const int nthr = __syncthreads_count(open && !a.eb && conf[base + i] >= a.threshold);
+
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int ixj = i ^ j;
+      if (ixj > i) {
+        const unsigned long long x = keys[i], y = keys[ixj];
+        const bool up = (i & k) == 0;
+        if ((x > y) == up) {
+          keys[i] = y;
+          keys[ixj] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  if (i == 0) {
+    int k;
+    if (a.eb) {
+      k = 0;
+      float run = 0.f;
+      for (int j = 0; j < nU; ++j) {
+        const int pos = (int)(keys[j] & 0xffffffffu);
+        run = __fadd_rn(run, ent[base + pos] + 0.0f);
+        if (run <= a.bound)
+          ++k;
+        else
+          break;
+      }
+      if (nU > 0 && k < 1) k = 1;
+    } else {
+      k = nthr > a.quota ? nthr : a.quota;
+      if (k > nU) k = nU;
+    }
+    krule_s = k;
+    if (s >= a.S - 1) k = nU;
+    k_s = k;
+  }
+  __syncthreads();
+  const int k = k_s;
+  if (i < k) {
+    const int pos = (int)(keys[i] & 0xffffffffu);
+    int c = cand[base + pos];
+    if (c < 0 || c >= a.V) {
+      raise_error(err, DLM_EBOUNDS);
+      c = 0;
+    }
+    tok[pos] = c;
+    com[pos] = 1;
+  }
+  __syncthreads();
+
+  const int e = eos_fill(tok, com, C, a.eos_id, &e_s, &fill1);
+
+  if (a.uniform && i < C && !com[i]) {
+    const U32x4 w =
+        philox10(U32x4{(uint32_t)b, (uint32_t)(s + 1), (uint32_t)i, kRenoiseWord}, a.seed_lo,
+                 a.seed_hi);
+    tok[i] = uniform_id(w.a, a.V);
+  }
+  if (i < C) {
+    tokens[base + i] = tok[i];
+    committed[base + i] = com[i];
+  }
+  const int all = __syncthreads_and(i >= C || com[i]);
+  if (i == 0) {
+    done[b] = all ? 1 : 0;
+    step[b] = s + 1;
+    eos_pos[b] = e;
+    if (stats != nullptr) {
+      stats[b].steps_used += 1;
+      stats[b].committed_by_sampler += k;
+      stats[b].forced_at_budget += k - krule_s;
+      stats[b].eos_autofill += fill0 + fill1;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t lm_reduce(const LmPart* part, int rows, int n_tiles, int C, const uint8_t* done,
+                      const int* n_active, int32_t* cand, float* conf, float* ent,
+                      cudaStream_t st) {
+  const int rows_per_block = 8;
+  lm_reduce_kernel<<<(rows + rows_per_block - 1) / rows_per_block, 32 * rows_per_block, 0, st>>>(
+      part, rows, n_tiles, C, done, n_active, cand, conf, ent);
+  return cudaGetLastError();
+}
+
+cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
+                        uint8_t* done, int32_t* eos_pos, const int32_t* cand, const float* conf,
+                        const float* ent, dlm_canvas_stats* stats, const int* n_active,
+                        int* err, cudaStream_t st) {
+  int P = 32;
+  while (P < a.C) P <<= 1;
+  if (P > kMaxC) return cudaErrorInvalidValue;
+  commit_kernel<<<a.B, P, 0, st>>>(a, tokens, committed, step, done, eos_pos, cand, conf, ent,
+                                   stats, n_active, err);
+  return cudaGetLastError();
+}
+
+}  // namespace dlm

@@ -378,10 +378,10 @@ def chunk_partials(z_row: np.ndarray, chunk: int):
         if not np.isfinite(m):
             parts.append((-np.inf, 0.0, 0.0, -1))
             continue
-        e = np.exp(zc - m)
         fin = np.isfinite(zc)
-        parts.append((m, e.sum(), float(np.sum(np.where(fin, e * (zc - m), 0.0))),
-                      c0 + int(np.argmax(zc))))
+        dz = np.where(fin, zc - m, 0.0)
+        e = np.where(fin, np.exp(dz), 0.0)
+        parts.append((m, e.sum(), float(np.sum(e * dz)), c0 + int(np.argmax(zc))))
     return parts
 
 

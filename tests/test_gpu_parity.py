@@ -1,0 +1,401 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on seeded
+inputs.  Every stage is teacher-forced: the oracle is given the GPU's own
+inputs to that stage, so one rounding difference cannot cascade.
+
+Standards (the method's parity bar):
+  * selection on identical float32 inputs: token ids, commit masks, step,
+    done, EOS position and counters bit-exact;
+  * candidates from identical float32 logits bit-exact, confidence within
+    1e-3, entropy within 1e-3;
+  * attention output within 2e-2 absolute of the float64 oracle;
+  * stored bf16 activations equal up to one rounding step;
+  * candidates from the oracle's float64 logits: equal except near ties
+    (top-2 gap < 1e-3), which are counted.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from gpu_util import (abs_terms, assert_storage_close, lib_params, make_pair, near_tie_ok,
+                      oracle_params, state_from, to64)
+from oracle import dlm_oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only hosts
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from masked_block_diffusion_denoise_b200 import (DLM_BUF_CAND, DLM_BUF_CONF, DLM_BUF_ENTROPY,
+                                                 DLM_BUF_K_CACHE, DLM_BUF_O, DLM_BUF_Q,
+                                                 DLM_BUF_V_CACHE, DLM_BUF_X, DLM_BUF_Y)
+
+
+# ---------------------------------------------------------------------------
+# stage-by-stage check of one step
+# ---------------------------------------------------------------------------
+
+def check_one_step(sess, om, wl, cv, p_lib, p_or, *, rows_sample=None, heads_sample=None,
+                   full_logits=True, report=None):
+    sh = wl.shape
+    B, C = cv.tokens.shape
+    M = B * C
+    dt = torch.bfloat16 if sh.dtype == "bf16" else torch.float32
+    pre = cv.numpy()
+    sess.step(cv, p_lib)
+    sess.check()
+    post = cv.numpy()
+    active = [b for b in range(B) if not pre["done"][b]]
+    x = to64(sess.buffer(DLM_BUF_X, (M, sh.d_model), dt))
+    q = to64(sess.buffer(DLM_BUF_Q, (M, sh.n_heads, sh.head_dim), dt))
+    o = to64(sess.buffer(DLM_BUF_O, (M, sh.n_heads * sh.head_dim), dt))
+    y = to64(sess.buffer(DLM_BUF_Y, (M, sh.d_model), dt))
+    Lcap = sess.max_prefix + sess.max_canvas
+    kc = sess.buffer(DLM_BUF_K_CACHE, (sess.max_batch, sh.n_kv_heads, Lcap, sh.head_dim), dt)
+    vc = sess.buffer(DLM_BUF_V_CACHE, (sess.max_batch, sh.n_kv_heads, Lcap, sh.head_dim), dt)
+    cand = sess.buffer(DLM_BUF_CAND, (M,), torch.int32).cpu().numpy()
+    conf = sess.buffer(DLM_BUF_CONF, (M,), torch.float32).cpu().numpy()
+    ent = sess.buffer(DLM_BUF_ENTROPY, (M,), torch.float32).cpu().numpy()
+    logits = sess.logits(B, C).cpu().numpy() if full_logits else None
+    near_ties = 0
+    for b in active:
+        r0 = b * C
+        rows = np.arange(C) if rows_sample is None else np.asarray(rows_sample)
+        L = om.kv_len(b)
+        # a1 embedding: exact
+        assert np.array_equal(x[r0 + rows], om.embed(pre["tokens"][b][rows])), "embed"
+        # a2 projections + RoPE from the GPU's x
+        qo, ko, vo = om.project_qkv(x[r0 + rows], L + rows)
+        xr = x[r0 + rows]
+        half = sh.head_dim // 2
+        rot = lambda t: np.concatenate([t[..., :half] + t[..., half:]] * 2, axis=-1)
+        tq = rot(abs_terms(xr, om.w_q).reshape(qo.shape))
+        tk = rot(abs_terms(xr, om.w_k).reshape(ko.shape))
+        tv = abs_terms(xr, om.w_v).reshape(vo.shape)
+        assert_storage_close(q[r0 + rows], qo, sh.dtype, what="q", terms=tq)
+        kg = to64(kc[b, :, L:L + C]).transpose(1, 0, 2)
+        vg = to64(vc[b, :, L:L + C]).transpose(1, 0, 2)
+        assert_storage_close(kg[rows], ko, sh.dtype, what="canvas k", terms=tk)
+        assert_storage_close(vg[rows], vo, sh.dtype, what="canvas v", terms=tv)
+        # a3 attention from the GPU's q, k, v
+        qb = q[r0:r0 + C]
+        oo = om.attend(b, qb, kg, vg)
+        err = np.abs(o[r0:r0 + C] - oo)
+        if heads_sample is not None:
+            cols = np.concatenate([np.arange(h * sh.head_dim, (h + 1) * sh.head_dim)
+                                   for h in heads_sample])
+            err = err[:, cols]
+        assert err.max() < 2e-2, "attention max abs err %g" % err.max()
+        if report is not None:
+            report.setdefault("attn_max_err", []).append(float(err.max()))
+        # a4 output projection + residual from the GPU's x and o
+        yo = om.out_proj(x[r0 + rows], o[r0 + rows])
+        assert_storage_close(y[r0 + rows], yo, sh.dtype, what="y",
+                             terms=np.abs(xr) + abs_terms(o[r0 + rows], om.w_o))
+        # a5/a6 scores
+        if p_or.entropy_bound >= 0 or p_or.temperature > 0:
+            continue   # sampling modes are checked in their own test
+        mask = sh.mask_id if p_or.corruption == "mask" else -1
+        if logits is not None:
+            lg = logits[r0:r0 + C]
+            lo = om.logits(y[r0:r0 + C])
+            assert np.abs(lg - lo).max() < 2e-3 * max(1.0, np.abs(lo).max()), "logits"
+            c32, f32, h32, _ = O.scores(lg.astype(np.float32), mask)
+            assert np.array_equal(cand[r0:r0 + C], c32), "cand from identical logits"
+            assert np.abs(conf[r0:r0 + C] - f32).max() < 1e-3, "confidence"
+            assert np.abs(ent[r0:r0 + C] - h32).max() < 1e-3, "entropy"
+            c64, _, _, z = O.scores(lo, mask)
+            for i in range(C):
+                if cand[r0 + i] != c64[i]:
+                    assert near_tie_ok(z[i], int(cand[r0 + i]), int(c64[i]), 1e-3), \
+                        "argmax flip outside a near tie"
+                    near_ties += 1
+        else:
+            for i in rows:
+                lo = om.logits(y[r0 + i:r0 + i + 1])
+                c64, f64, h64, z = O.scores(lo, mask)
+                if cand[r0 + i] != c64[0]:
+                    assert near_tie_ok(z[0], int(cand[r0 + i]), int(c64[0]), 1e-3)
+                    near_ties += 1
+                else:
+                    assert abs(conf[r0 + i] - f64[0]) < 1e-3
+                assert abs(ent[r0 + i] - h64[0]) < 1e-3
+    # a7 selection on the GPU's own cand / conf / H: bit-exact
+    st = state_from(pre)
+    stats = [O.CanvasStats() for _ in range(B)]
+    for b in range(B):
+        O.select_canvas(st, b, cand[b * C:(b + 1) * C], conf[b * C:(b + 1) * C],
+                        ent[b * C:(b + 1) * C], p_or, vocab=sh.vocab, mask_id=sh.mask_id,
+                        eos_id=sh.eos_id, stats=stats[b])
+    assert np.array_equal(st.tokens, post["tokens"]), "tokens after commit"
+    assert np.array_equal(st.committed, post["committed"]), "commit mask"
+    assert np.array_equal(st.step, post["step"]) and np.array_equal(st.done, post["done"])
+    assert np.array_equal(st.eos_pos, post["eos_pos"])
+    dstats = post["stats"] - pre["stats"]
+    for b in range(B):
+        assert list(dstats[b]) == [stats[b].steps_used, stats[b].committed_by_sampler,
+                                   stats[b].forced_at_budget, stats[b].eos_autofill]
+    if report is not None:
+        report["near_ties"] = report.get("near_ties", 0) + near_ties
+    return pre, post
+
+
+SMALL = {
+    # GQA 2, vocab with a ragged 96-column tail, ragged prefixes, one M tile
+    "small_gqa2": W.small_workload("small_gqa2", steps=8, quota=4),
+    # GQA 4, two batches of 64 positions: 256 rows -> two M tiles, 256-wide LM tiles
+    "small_mtiles": W.small_workload("small_mtiles", n_heads=8, n_kv_heads=2, batch=4,
+                                     canvas=64, steps=6, quota=0, prefix_len=(64, 300),
+                                     prefix_cap=320, vocab=3000),
+    # canvas not a multiple of 8, single KV head, threshold 0 (all commit in one step)
+    "small_c37": W.small_workload("small_c37", n_heads=2, n_kv_heads=1, canvas=37, batch=3,
+                                  steps=5, threshold=0.0, quota=1, prefix_len=(1, 130),
+                                  prefix_cap=160),
+    # uniform corruption, quota from ceil(C/S)
+    "small_uniform": W.small_workload("small_uniform", corruption="uniform", steps=7, quota=0,
+                                      seed=3),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_block_stagewise(name):
+    wl = SMALL[name]
+    sess, om, _ = make_pair(wl)
+    try:
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        sess.init(cv, p_lib)
+        init = cv.numpy()
+        ref = O.init_canvas(wl.batch, p_or, wl.shape.mask_id, wl.shape.vocab)
+        assert np.array_equal(init["tokens"], ref.tokens)
+        report = {}
+        for s in range(wl.steps):
+            pre, post = check_one_step(sess, om, wl, cv, p_lib, p_or, report=report)
+            if post["done"].all():
+                break
+        assert cv.numpy()["done"].all()
+        print(name, report)
+    finally:
+        sess.close()
+
+
+def test_tiny_fp32_reference_config():
+    """The tiny fp32 configuration: batch 1, d 256, 4 heads of 64, vocab 4096,
+    prefix of 128 random ids appended through the clean pass, canvas 32,
+    8 steps, threshold 0.9, quota 4, seed 0."""
+    wl = W.WORKLOADS["tiny"]
+    sess, om, _ = make_pair(wl)
+    try:
+        # the clean pass wrote the same K/V as the oracle's
+        Lcap = sess.max_prefix + sess.max_canvas
+        kc = to64(sess.buffer(DLM_BUF_K_CACHE, (1, 4, Lcap, 64), torch.float32))
+        assert np.allclose(kc[0, :, :128], om.k_cache[0], atol=1e-4)
+        cv = sess.new_canvas(1, 32)
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        sess.init(cv, p_lib)
+        steps = 0
+        while not cv.numpy()["done"].all():
+            check_one_step(sess, om, wl, cv, p_lib, p_or)
+            steps += 1
+        assert steps == 8    # quota 4 over 32 positions
+        # free-running oracle from the same start reaches the same canvas
+        st = O.init_canvas(1, p_or, 100, 4096)
+        O.decode_block(om, st, p_or)
+        assert np.array_equal(st.tokens, cv.numpy()["tokens"])
+    finally:
+        sess.close()
+
+
+def test_block_graph_equals_steps_and_resume():
+    wl = SMALL["small_gqa2"].replace(eos_frac=0.5, seed=5)
+    sess, om, _ = make_pair(wl)
+    try:
+        p = lib_params(wl)
+        a, b, c = (sess.new_canvas(wl.batch, wl.canvas) for _ in range(3))
+        for cv in (a, b, c):
+            sess.init(cv, p)
+        for (bb, slot) in W.make_eos_plant(wl) or [(0, 7)]:
+            for cv in (a, b, c):
+                cv.tokens[bb, slot] = wl.shape.eos_id
+                cv.committed[bb, slot] = 1
+        sess.block(a, p)
+        for _ in range(wl.steps):
+            sess.step(b, p)
+        for _ in range(3):
+            sess.step(c, p)
+        sess.block(c, p)       # resume: steps of finished canvases do nothing
+        sess.check()
+        na, nb, nc = a.numpy(), b.numpy(), c.numpy()
+        for key in ("tokens", "committed", "step", "done", "eos_pos", "stats"):
+            assert np.array_equal(na[key], nb[key]), key
+            assert np.array_equal(na[key], nc[key]), key
+        assert na["done"].all()
+        assert sess.ctx is not None
+    finally:
+        sess.close()
+
+
+def test_entropy_bound_sampling_stage():
+    """Gumbel sampling at annealed temperature and the entropy-bound rule."""
+    wl = W.small_workload("small_eb", corruption="uniform", entropy_bound=0.5, steps=6,
+                          vocab=2000, seed=11)
+    sess, om, _ = make_pair(wl)
+    try:
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        sess.init(cv, p_lib)
+        C = wl.canvas
+        flips = 0
+        for s in range(wl.steps):
+            pre = cv.numpy()
+            if pre["done"].all():
+                break
+            check_one_step(sess, om, wl, cv, p_lib, p_or)
+            # scores: replay the sampling on the GPU's float32 logits
+            lg = sess.logits(wl.batch, C).cpu().numpy()
+            cand = sess.buffer(DLM_BUF_CAND, (wl.batch * C,), torch.int32).cpu().numpy()
+            conf = sess.buffer(DLM_BUF_CONF, (wl.batch * C,), torch.float32).cpu().numpy()
+            ent = sess.buffer(DLM_BUF_ENTROPY, (wl.batch * C,), torch.float32).cpu().numpy()
+            for b in range(wl.batch):
+                if pre["done"][b]:
+                    continue
+                st = int(pre["step"][b])
+                T = O.annealed_temperature(wl.t_max, wl.t_min, st, wl.steps)
+                inv = np.float32(np.float32(1.0) / T)
+                G = np.stack([O.gumbel_noise(wl.seed, b, st, i, wl.shape.vocab)
+                              for i in range(C)])
+                c64, f64, h64, z = O.scores(lg[b * C:(b + 1) * C], -1, inv_temp=inv, gumbel=G)
+                for i in range(C):
+                    gc = int(cand[b * C + i])
+                    g = z[i] + G[i]
+                    if gc != c64[i]:
+                        assert abs(g[gc] - g[c64[i]]) < 1e-4, "sampled id outside a near tie"
+                        flips += 1
+                    else:
+                        assert abs(conf[b * C + i] - f64[i]) < 1e-3
+                    assert abs(ent[b * C + i] - h64[i]) < 1e-3
+        assert flips <= 2
+    finally:
+        sess.close()
+
+
+# ---------------------------------------------------------------------------
+# kernel (c) alone: bit-exact selection on identical inputs
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("C", [1, 7, 32, 100, 256, 1024])
+@pytest.mark.parametrize("mode", ["greedy", "thr0", "thr_big_q1", "eb", "uniform", "forced"])
+def test_commit_bit_exact(C, mode):
+    from masked_block_diffusion_denoise_b200.session import Session, sampler_params
+    sh = W.ModelShape(d_model=64, n_heads=2, n_kv_heads=1, head_dim=32, vocab=5000, dtype="f32")
+    w = W.make_weights(sh, seed=1)
+    B = 5
+    sess = Session(sh, w, max_batch=B, max_prefix=8, max_canvas=1024)
+    try:
+        r = np.random.default_rng(C * 31 + len(mode))
+        S = 10
+        kw = dict(canvas=C, steps=S, threshold=0.6, quota=3, seed=99)
+        if mode == "thr0":
+            kw.update(threshold=0.0)
+        if mode == "thr_big_q1":
+            kw.update(threshold=1.5, quota=1)
+        if mode == "eb":
+            kw.update(entropy_bound=2.0, corruption="uniform")
+        if mode == "uniform":
+            kw.update(corruption="uniform")
+        p_lib = sampler_params(**kw)
+        p_or = O.SamplerParams(**kw)
+        tokens = r.integers(0, sh.vocab, size=(B, C)).astype(np.int64)
+        committed = r.random((B, C)) < 0.3
+        step = r.integers(0, S - 1, size=B)
+        if mode == "forced":
+            step[:] = S - 1
+        done = np.zeros(B, bool)
+        done[4] = True
+        tokens[1, C // 2] = sh.eos_id          # a committed EOS mid-canvas
+        committed[1, C // 2] = True
+        cand = r.integers(0, sh.vocab, size=(B, C)).astype(np.int32)
+        cand[2, : max(1, C // 5)] = sh.eos_id  # sampler may commit an EOS
+        conf = r.random((B, C)).astype(np.float32)
+        conf[:, ::3] = conf[:, :1]             # ties -> lower index first
+        conf[3, :] = np.float32(0.6)           # exactly the threshold
+        ent = (r.random((B, C)) * 0.5).astype(np.float32)
+        ent[:, ::4] = np.float32(0.0)
+        cv = sess.new_canvas(B, C)
+        cv.load(tokens, committed, step, done, np.full(B, -1))
+        dev = lambda a: torch.as_tensor(a).cuda()
+        sess.commit(cv, p_lib, dev(cand), dev(conf), dev(ent))
+        sess.check()
+        got = cv.numpy()
+        st = O.CanvasState(tokens.copy(), committed.copy(), step.copy(), done.copy(),
+                           np.full(B, -1))
+        stats = [O.CanvasStats() for _ in range(B)]
+        for b in range(B):
+            O.select_canvas(st, b, cand[b], conf[b], ent[b], p_or, vocab=sh.vocab,
+                            mask_id=sh.mask_id, eos_id=sh.eos_id, stats=stats[b])
+        assert np.array_equal(got["tokens"], st.tokens)
+        assert np.array_equal(got["committed"], st.committed)
+        assert np.array_equal(got["step"], st.step)
+        assert np.array_equal(got["done"], st.done)
+        assert np.array_equal(got["eos_pos"][:4], st.eos_pos[:4])
+        for b in range(B):
+            assert list(got["stats"][b]) == [stats[b].steps_used, stats[b].committed_by_sampler,
+                                             stats[b].forced_at_budget, stats[b].eos_autofill]
+    finally:
+        sess.close()
+
+
+def test_canvas_init_uniform_bit_exact():
+    from masked_block_diffusion_denoise_b200.session import Session, sampler_params
+    sh = W.ModelShape(d_model=64, n_heads=2, n_kv_heads=1, head_dim=32, vocab=262144, dtype="f32")
+    sess = Session(sh, W.make_weights(sh, seed=2), max_batch=3, max_prefix=8, max_canvas=256)
+    try:
+        p = sampler_params(canvas=256, steps=48, corruption="uniform", seed=0xDEADBEEF12345)
+        cv = sess.new_canvas(3, 256)
+        sess.init(cv, p)
+        ref = O.init_canvas(3, O.SamplerParams(canvas=256, steps=48, corruption="uniform",
+                                               seed=0xDEADBEEF12345), 100, 262144)
+        assert np.array_equal(cv.numpy()["tokens"], ref.tokens)
+    finally:
+        sess.close()
+
+
+def test_kv_append_tokens_bf16():
+    wl = W.small_workload("kv_tokens", prefix_kind="tokens", prefix_len=(150, 333), batch=2)
+    sess, om, _ = make_pair(wl)
+    try:
+        Lcap = sess.max_prefix + sess.max_canvas
+        sh = wl.shape
+        kc = sess.buffer(DLM_BUF_K_CACHE, (2, sh.n_kv_heads, Lcap, sh.head_dim), torch.bfloat16)
+        vc = sess.buffer(DLM_BUF_V_CACHE, (2, sh.n_kv_heads, Lcap, sh.head_dim), torch.bfloat16)
+        lens, toks, _, _ = W.make_prefix(wl)
+        for b in range(2):
+            L = om.kv_len(b)
+            xe = om.embed(toks[b])
+            half = sh.head_dim // 2
+            tk = abs_terms(xe, om.w_k).reshape(L, sh.n_kv_heads, sh.head_dim).transpose(1, 0, 2)
+            tk = np.concatenate([tk[..., :half] + tk[..., half:]] * 2, axis=-1)
+            tv = abs_terms(xe, om.w_v).reshape(L, sh.n_kv_heads, sh.head_dim).transpose(1, 0, 2)
+            assert_storage_close(to64(kc[b, :, :L]), om.k_cache[b], "bf16", what="K", terms=tk)
+            assert_storage_close(to64(vc[b, :, :L]), om.v_cache[b], "bf16", what="V", terms=tv)
+    finally:
+        sess.close()
+
+
+# ---------------------------------------------------------------------------
+# full-size shapes: one step, sampled outputs
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["8b_b1", "encdec"])
+def test_full_size_step_sampled(name):
+    wl = W.WORKLOADS[name]
+    sess, om, _ = make_pair(wl)
+    try:
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        sess.init(cv, p_lib)
+        rows = np.array([0, 5, wl.canvas - 1])
+        check_one_step(sess, om, wl, cv, p_lib, p_or, rows_sample=rows, full_logits=False)
+    finally:
+        sess.close()
