@@ -226,6 +226,35 @@ enum { DLM_STAGE_EMBED = 0, DLM_STAGE_QKV = 1, DLM_STAGE_ATTENTION = 2, DLM_STAG
  * use.  DLM_EINVAL for a bad stage or n_pairs < 0. */
 int dlm_set_stage_events(dlm_ctx *ctx, int stage, void *const *events, int n_pairs);
 
+/* Canvas attention that allocates nothing.  The pages have no counterpart to
+ * this call: it exists for callers that cannot allocate device memory, such
+ * as a serving engine that reserves all device memory for its own pool at
+ * start-up, or code issued while a stream is being captured into a CUDA graph
+ * (where cudaMalloc would synchronise the device or is not allowed).  It runs
+ * the same split-KV attention kernels as dlm_denoise_step, but the split
+ * partials live in a fixed array compiled into the library (8 MiB of
+ * partial outputs plus 128 KiB of (max, sum) pairs: 16384 row slots, each
+ * GPU that loads the library holds it until the process exits).
+ *   q        device bf16 [batch*canvas][n_heads][head_dim], row b*canvas + i
+ *   k_cache, v_cache  device bf16 [kv_batch][n_kv_heads][kv_capacity][head_dim];
+ *            sequence b's keys are slots [0, lens[b] + canvas) (prefix
+ *            followed by the canvas's own K/V)
+ *   lens     device int32 [batch]; max_len (host) must be >= every lens[b]
+ *   o        device bf16 [batch*canvas][n_heads*head_dim], written
+ * head_dim must be 128, n_heads a multiple of n_kv_heads, batch <= kv_batch,
+ * max_len + canvas <= kv_capacity.  If the split plan needs more than the
+ * 16384 slots (batch * n_kv_heads * splits * query-rows-per-KV-head) the call
+ * fails with DLM_EINVAL and dlm_last_error(NULL) says how many it needed.
+ * The first call on a device looks up the array's device address; make that
+ * first call before any stream capture.  Every call shares the array, so
+ * calls that overlap on the GPU (different streams, or other threads) race;
+ * serialise them.  Launch errors are returned; a device-side wait that gives
+ * up is recorded in a device word that each call clears first. */
+int dlm_attention_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *lens, int max_len, void *o, int batch, int canvas,
+                          int n_heads, int n_kv_heads, int head_dim, int kv_batch,
+                          int kv_capacity, void *stream);
+
 /* Synchronise `stream` and return the device error word (DLM_OK, or
  * DLM_ETIMEOUT / DLM_EBOUNDS set by a kernel); clears it. */
 int dlm_check(dlm_ctx *ctx, void *stream);

@@ -24,7 +24,7 @@ __all__ = [
     "dlm_debug_logits", "dlm_check", "dlm_launches_per_step", "dlm_last_error",
     "EXPORTED_SYMBOLS", "dlm_set_stage_events", "DLM_STAGE_EMBED", "DLM_STAGE_QKV",
     "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_REDUCE",
-    "DLM_STAGE_COMMIT", "DLM_NUM_STAGES",
+    "DLM_STAGE_COMMIT", "DLM_NUM_STAGES", "dlm_attention_noalloc",
 ]
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, DLM_ESTATE = \
@@ -103,6 +103,7 @@ _SIGS = {
     "dlm_debug_buffer": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
     "dlm_debug_logits": (_I, [_P, _I, _I, _P, _P]),
     "dlm_set_stage_events": (_I, [_P, _I, ctypes.POINTER(_P), _I]),
+    "dlm_attention_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "dlm_check": (_I, [_P, _P]),
     "dlm_launches_per_step": (_I, [_P]),
     "dlm_last_error": (ctypes.c_char_p, [_P]),
@@ -234,6 +235,18 @@ def dlm_set_stage_events(ctx, stage: int, events) -> int:
     n = len(events)
     arr = (ctypes.c_void_p * max(n, 1))(*events)
     return _check(ctx, lib().dlm_set_stage_events(ctx, stage, arr if n else None, n // 2))
+
+
+def dlm_attention_noalloc(q, k_cache, v_cache, lens, max_len: int, o, batch: int, canvas: int,
+                          n_heads: int, n_kv_heads: int, head_dim: int, kv_batch: int,
+                          kv_capacity: int, stream=None) -> int:
+    """Canvas attention with no device allocation (see include/dlm.h)."""
+    rc = lib().dlm_attention_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(lens), max_len,
+                                     _ptr(o), batch, canvas, n_heads, n_kv_heads, head_dim,
+                                     kv_batch, kv_capacity, _stream(stream))
+    if rc != DLM_OK:
+        raise DlmError(rc, lib().dlm_last_error(None).decode())
+    return rc
 
 
 def dlm_check(ctx, stream=None) -> int:

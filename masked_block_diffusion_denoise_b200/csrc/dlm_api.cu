@@ -850,3 +850,95 @@ const char* dlm_last_error(const dlm_ctx* ctx) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attention without allocation: split partials in a fixed device array
+// ---------------------------------------------------------------------------
+
+// Row slots of split partials (one slot = one query row of one split of one
+// (sequence, KV head)): 16384 slots = 8 MiB of partial outputs (128 floats
+// each) + 128 KiB of (max, sum) pairs, plus one device error word.
+constexpr int kNoAllocSlots = 16384;
+constexpr int kNoAllocDh = 128;
+static __device__ __align__(256) float g_noalloc_opart[(size_t)kNoAllocSlots * kNoAllocDh];
+static __device__ __align__(256) float2 g_noalloc_ml[kNoAllocSlots];
+static __device__ __align__(256) int g_noalloc_err[1];
+
+namespace {
+
+struct NoAllocScratch {
+  bool ready = false;
+  float* opart = nullptr;
+  float2* ml = nullptr;
+  int* err = nullptr;
+};
+constexpr int kMaxDevices = 64;
+NoAllocScratch g_noalloc[kMaxDevices];
+
+}  // namespace
+
+extern "C" {
+
+int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* lens, int max_len, void* o, int batch, int canvas,
+                          int n_heads, int n_kv_heads, int head_dim, int kv_batch,
+                          int kv_capacity, void* stream) {
+  g_create_error.clear();
+  if (!q || !k_cache || !v_cache || !lens || !o)
+    return fail(nullptr, DLM_EINVAL, "attention_noalloc: NULL pointer argument");
+  if (head_dim != kNoAllocDh || n_heads <= 0 || n_kv_heads <= 0 || n_heads % n_kv_heads != 0)
+    return fail(nullptr, DLM_EINVAL,
+                "attention_noalloc: needs head_dim 128 and n_heads a multiple of n_kv_heads");
+  if (batch < 1 || canvas < 1 || batch > kv_batch || max_len < 0 ||
+      (long)max_len + canvas > kv_capacity)
+    return fail(nullptr, DLM_EINVAL,
+                "attention_noalloc: need 1 <= batch <= kv_batch and max_len + canvas <= "
+                "kv_capacity");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(nullptr, "cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(nullptr, DLM_EINVAL, "attention_noalloc: device index out of range");
+  NoAllocScratch& sc = g_noalloc[dev];
+  if (!sc.ready) {
+    // host code must not pass the arrays' names to a kernel: those are host
+    // stand-ins; the device addresses come from the runtime, once per device
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_opart)) != cudaSuccess)
+      return cuda_fail(nullptr, "cudaGetSymbolAddress(partials)", e);
+    sc.opart = static_cast<float*>(p);
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_ml)) != cudaSuccess)
+      return cuda_fail(nullptr, "cudaGetSymbolAddress(max/sum)", e);
+    sc.ml = static_cast<float2*>(p);
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_err)) != cudaSuccess)
+      return cuda_fail(nullptr, "cudaGetSymbolAddress(error word)", e);
+    sc.err = static_cast<int*>(p);
+    sc.ready = true;
+  }
+  // the split plan of dlm_denoise_step for these sizes
+  dlm_ctx plan_ctx;
+  plan_ctx.md = ModelDims{0, n_heads, n_kv_heads, head_dim, 0, -1, -1, kv_capacity, 2};
+  cudaDeviceGetAttribute(&plan_ctx.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, max_len + canvas);
+  const long slots = (long)batch * n_kv_heads * ap.nsplit * ap.R;
+  if (ap.nsplit > 1 && slots > kNoAllocSlots) {
+    g_create_error = "attention_noalloc: the split plan needs " + std::to_string(slots) +
+                     " partial row slots; the static array holds " +
+                     std::to_string(kNoAllocSlots);
+    return DLM_EINVAL;
+  }
+  CUtensorMap tmK, tmV;
+  const uint64_t planes = (uint64_t)kv_batch * n_kv_heads;
+  if (!map_kv(&tmK, const_cast<void*>(k_cache), planes, kv_capacity, head_dim) ||
+      !map_kv(&tmV, const_cast<void*>(v_cache), planes, kv_capacity, head_dim))
+    return fail(nullptr, DLM_ECUDA, "attention_noalloc: cuTensorMapEncodeTiled failed");
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((e = cudaMemsetAsync(sc.err, 0, sizeof(int), st)) != cudaSuccess)
+    return cuda_fail(nullptr, "cudaMemsetAsync(error word)", e);
+  e = attention_bf16(plan_ctx.md, ap, tmK, tmV, q, o, sc.opart, sc.ml, lens, nullptr, nullptr,
+                     sc.err, st);
+  if (e != cudaSuccess) return cuda_fail(nullptr, "attention_noalloc launch", e);
+  return DLM_OK;
+}
+
+}  // extern "C"
