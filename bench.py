@@ -272,7 +272,7 @@ def run_ours(a):
     stream.synchronize()
     lm_ms = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(S)]
     stages = {}
-    names = ["embed", "qkv", "attention", "wo", "lm_head", "reduce", "commit"]
+    names = ["embed", "qkv", "attention", "wo", "lm_head", "reduce+commit"]
     for st, name in enumerate(names):
         dlm.dlm_set_stage_events(sess.ctx, st, [e.cuda_event for e in evs])
         run_steps(2 * S, cv)

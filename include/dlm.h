@@ -211,9 +211,10 @@ int dlm_debug_buffer(dlm_ctx *ctx, int which, void **ptr, size_t *bytes);
  * the fused reduction (the store epilogue instead of the reduction). */
 int dlm_debug_logits(dlm_ctx *ctx, int batch, int canvas, float *logits, void *stream);
 
-/* Stages of a step, for dlm_set_stage_events. */
+/* Stages of a step, for dlm_set_stage_events.  DLM_STAGE_COMMIT is the one
+ * launch that combines the LM head's partials and commits / re-noises. */
 enum { DLM_STAGE_EMBED = 0, DLM_STAGE_QKV = 1, DLM_STAGE_ATTENTION = 2, DLM_STAGE_WO = 3,
-       DLM_STAGE_LM_HEAD = 4, DLM_STAGE_REDUCE = 5, DLM_STAGE_COMMIT = 6, DLM_NUM_STAGES = 7 };
+       DLM_STAGE_LM_HEAD = 4, DLM_STAGE_COMMIT = 5, DLM_NUM_STAGES = 6 };
 
 /* Measurement hook: record caller-created CUDA events (cudaEvent_t passed as
  * void*, created with timing enabled, owned by the caller) on the launch

@@ -23,8 +23,7 @@ __all__ = [
     "dlm_decode_block", "dlm_decode_block_host", "dlm_commit", "dlm_debug_buffer",
     "dlm_debug_logits", "dlm_check", "dlm_launches_per_step", "dlm_last_error",
     "EXPORTED_SYMBOLS", "dlm_set_stage_events", "DLM_STAGE_EMBED", "DLM_STAGE_QKV",
-    "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_REDUCE",
-    "DLM_STAGE_COMMIT", "DLM_NUM_STAGES", "dlm_attention_noalloc",
+    "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT", "DLM_NUM_STAGES", "dlm_attention_noalloc",
 ]
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, DLM_ESTATE = \
@@ -35,7 +34,7 @@ DLM_MASK, DLM_UNIFORM = 0, 1
  DLM_BUF_K_CACHE, DLM_BUF_V_CACHE) = range(9)
 
 (DLM_STAGE_EMBED, DLM_STAGE_QKV, DLM_STAGE_ATTENTION, DLM_STAGE_WO, DLM_STAGE_LM_HEAD,
- DLM_STAGE_REDUCE, DLM_STAGE_COMMIT, DLM_NUM_STAGES) = range(8)
+ DLM_STAGE_COMMIT, DLM_NUM_STAGES) = range(7)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 

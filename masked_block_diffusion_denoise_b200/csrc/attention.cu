@@ -48,6 +48,7 @@ struct AttnParams {
 __global__ void __launch_bounds__(32 * (kWarps + 1), 1)
     attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const AttnParams p) {
+  pdl_wait_then_release();
   if (p.n_active != nullptr && *p.n_active == 0) return;
   const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
@@ -272,11 +273,15 @@ __global__ void __launch_bounds__(32 * (kWarps + 1), 1)
   }
 }
 
-// log-sum-exp combination of the splits of one (sequence, KV head)
+// log-sum-exp combination of the splits of one (sequence, KV head); one warp
+// per query row, lane = 4 head-dim columns.  The split weights are computed
+// in parallel (lane s holds split s), then the partial rows are read in
+// batches of independent loads.
 __global__ void attn_combine_kernel(const float* __restrict__ opart, const float2* __restrict__ ml,
                                     __nv_bfloat16* __restrict__ o, const int32_t* __restrict__ lens,
                                     const uint8_t* __restrict__ done, const int* n_active, int H,
                                     int Hkv, int G, int C, int R, int chunk, int nsplit) {
+  pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   const int bg = blockIdx.x;
   const int b = bg / Hkv, g = bg - b * Hkv;
@@ -285,21 +290,48 @@ __global__ void attn_combine_kernel(const float* __restrict__ opart, const float
   const int r = blockIdx.y * (blockDim.x >> 5) + warp;
   if (r >= R) return;
   const int n_keys = lens[b] + C;
-  const int nvalid = min(nsplit, (n_keys + chunk - 1) / chunk);
-  float M = -CUDART_INF_F;
-  for (int s = 0; s < nvalid; ++s) M = fmaxf(M, ml[((size_t)bg * nsplit + s) * R + r].x);
+  const int nvalid = min(nsplit, (n_keys + chunk - 1) / chunk);   // <= 64
+  const size_t base = (size_t)bg * nsplit * R + r;                  // slot of split s: base + s*R
+  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+  if (lane < nvalid) {
+    const float2 v = ml[base + (size_t)lane * R];
+    m0 = v.x;
+    l0 = v.y;
+  }
+  if (lane + 32 < nvalid) {
+    const float2 v = ml[base + (size_t)(lane + 32) * R];
+    m1 = v.x;
+    l1 = v.y;
+  }
+  float M = fmaxf(m0, m1);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  const float w0 = lane < nvalid ? fast_exp2(m0 - M) : 0.f;
+  const float w1 = lane + 32 < nvalid ? fast_exp2(m1 - M) : 0.f;
+  float L = w0 * l0 + w1 * l1;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float L = 0.f;
-  for (int s = 0; s < nvalid; ++s) {
-    const size_t slot = ((size_t)bg * nsplit + s) * R + r;
-    const float2 v = ml[slot];
-    const float w = fast_exp2(v.x - M);
-    L += w * v.y;
-    const float4 x = *reinterpret_cast<const float4*>(opart + slot * kDh + lane * 4);
-    acc[0] += w * x.x;
-    acc[1] += w * x.y;
-    acc[2] += w * x.z;
-    acc[3] += w * x.w;
+  constexpr int kB = 8;
+  for (int s0 = 0; s0 < nvalid; s0 += kB) {
+    float4 x[kB];
+    float w[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int sidx = s0 + u;
+      const float wsel = sidx < 32 ? w0 : w1;
+      w[u] = __shfl_sync(0xffffffffu, wsel, sidx & 31);
+      x[u] = sidx < nvalid
+                 ? *reinterpret_cast<const float4*>(opart + (base + (size_t)sidx * R) * kDh + lane * 4)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      acc[0] += w[u] * x[u].x;
+      acc[1] += w[u] * x[u].y;
+      acc[2] += w[u] * x[u].z;
+      acc[3] += w[u] * x[u].w;
+    }
   }
   const float inv = 1.f / L;
   const int i = r / G, hh = r - i * G;
@@ -318,6 +350,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(int H, int Hkv, int C, in
                                                        const int32_t* __restrict__ lens,
                                                        const uint8_t* __restrict__ done,
                                                        const int* n_active, float scale) {
+  pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   constexpr int KT = 32;
   __shared__ float ks[KT][DH];
@@ -406,15 +439,14 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.nsplit = ap.nsplit;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
-  attn_bf16_kernel<<<grid, 32 * (kWarps + 1), kAttnSmem, st>>>(tmK, tmV, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(attn_bf16_kernel, grid, dim3(32 * (kWarps + 1)), kAttnSmem, st, tmK,
+                             tmV, p);
   if (e != cudaSuccess || ap.nsplit == 1) return e;
   const int rows_per_block = 8;
   dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);
-  attn_combine_kernel<<<g2, 32 * rows_per_block, 0, st>>>(opart, ml, (__nv_bfloat16*)o, lens,
-                                                          done, n_active, md.H, md.Hkv, ap.G,
-                                                          ap.C, ap.R, ap.chunk, ap.nsplit);
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, g2, dim3(32 * rows_per_block), 0, st,
+                    (const float*)opart, (const float2*)ml, (__nv_bfloat16*)o, lens, done,
+                    n_active, md.H, md.Hkv, ap.G, ap.C, ap.R, ap.chunk, ap.nsplit);
 }
 
 cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,
@@ -422,18 +454,19 @@ cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, con
                           const uint8_t* done, const int* n_active, cudaStream_t st) {
   const float scale = (float)(1.0 / sqrt((double)md.Dh));
   const int threads = 128;
+  cudaError_t e;
   if (md.Dh == 64)
-    attn_f32_kernel<64><<<B * md.H, threads, 0, st>>>(md.H, md.Hkv, C, md.Lcap, q, kcache, vcache,
-                                                      o, lens, done, n_active, scale);
+    e = launch_pdl(attn_f32_kernel<64>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
   else if (md.Dh == 128)
-    attn_f32_kernel<128><<<B * md.H, threads, 0, st>>>(md.H, md.Hkv, C, md.Lcap, q, kcache,
-                                                       vcache, o, lens, done, n_active, scale);
+    e = launch_pdl(attn_f32_kernel<128>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
   else if (md.Dh == 32)
-    attn_f32_kernel<32><<<B * md.H, threads, 0, st>>>(md.H, md.Hkv, C, md.Lcap, q, kcache, vcache,
-                                                      o, lens, done, n_active, scale);
+    e = launch_pdl(attn_f32_kernel<32>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
   else
     return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace dlm

@@ -431,17 +431,12 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     if (int rc = run_gemm(ctx, ctx->y, ctx->w_lm, md.V, pl, io, st)) return rc;
   }
   STAGE(DLM_STAGE_LM_HEAD, true);
-  // a6: cross-tile reduction
-  STAGE(DLM_STAGE_REDUCE, false);
-  e = lm_reduce(ctx->lmpart, rows, cdiv(md.V, pl.BN), C, c->done, ctx->n_active, ctx->cand,
-                ctx->conf, ctx->ent, st);
-  if (e != cudaSuccess) return cuda_fail(ctx, "lm reduce", e);
-  ++ctx->launches;
-  STAGE(DLM_STAGE_REDUCE, true);
-  // a7: commit / re-noise
+  // a6 + a7: cross-tile reduction, then commit / re-noise, one launch
+  const int n_part = ctx->bf16 ? gemm_tc_lm_partials(pl, ctx->num_sms) : cdiv(md.V, pl.BN);
   STAGE(DLM_STAGE_COMMIT, false);
   e = commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
-                  c->eos_pos, ctx->cand, ctx->conf, ctx->ent, stats, ctx->n_active, ctx->err, st);
+                  c->eos_pos, ctx->lmpart, n_part, ctx->cand, ctx->conf, ctx->ent, stats,
+                  ctx->n_active, ctx->err, st);
   if (e != cudaSuccess) return cuda_fail(ctx, "commit", e);
   ++ctx->launches;
   STAGE(DLM_STAGE_COMMIT, true);
@@ -778,8 +773,8 @@ int dlm_commit(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_p
   if (int rc = check_canvas(ctx, c)) return rc;
   if (!cand || !conf || !entropy) return fail(ctx, DLM_EINVAL, "cand/conf/entropy NULL");
   CK(commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
-                 c->eos_pos, cand, conf, entropy, stats, nullptr, ctx->err,
-                 (cudaStream_t)stream));
+                 c->eos_pos, nullptr, 0, const_cast<int32_t*>(cand), const_cast<float*>(conf),
+                 const_cast<float*>(entropy), stats, nullptr, ctx->err, (cudaStream_t)stream));
   return DLM_OK;
 }
 

@@ -23,6 +23,7 @@ template <int EPI>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A,
                                                        const float* __restrict__ B,
                                                        const SimtParams p) {
+  pdl_wait_then_release();
   if (p.n_active != nullptr && *p.n_active == 0) return;
   __shared__ float As[kTK][kT + 4];
   __shared__ float Bs[kTK][kT + 4];
@@ -117,11 +118,8 @@ cudaError_t gemm_f32(const float* A, const float* B, const GemmPlan& plan, const
   p.done = io.done;
   p.n_active = io.n_active;
   dim3 grid(p.n_tiles, (plan.M + kT - 1) / kT, plan.epi == EPI_LM ? 1 : plan.splits);
-  if (plan.epi == EPI_LM)
-    gemm_f32_kernel<EPI_LM><<<grid, 256, 0, st>>>(A, B, p);
-  else
-    gemm_f32_kernel<EPI_F32><<<grid, 256, 0, st>>>(A, B, p);
-  return cudaGetLastError();
+  if (plan.epi == EPI_LM) return launch_pdl(gemm_f32_kernel<EPI_LM>, grid, dim3(256), 0, st, A, B, p);
+  return launch_pdl(gemm_f32_kernel<EPI_F32>, grid, dim3(256), 0, st, A, B, p);
 }
 
 }  // namespace dlm

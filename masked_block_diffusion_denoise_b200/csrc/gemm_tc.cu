@@ -11,14 +11,17 @@
 //   warps 2..5  epilogue: tcgen05.ld the accumulator (one TMEM lane = one
 //               output row per thread) while the MMA warp fills the other
 //               accumulator.
-// Work units are (m tile, n tile, k split), m fastest, so that CTAs that run
-// at the same time share the same B (weight) slab through L2.
-//
 // Epilogues:
 //   EPI_F32  store f32 partial sums [split][M][N] (projections, split-K;
-//            full logits for inspection);
-//   EPI_LM   the LM head's fused vocabulary reduction: per (row, n tile) one
-//            LmPart; logits never leave the SM.
+//            full logits for inspection).  Work units (m tile, n tile,
+//            k split), m fastest, strided over the grid, so that CTAs that
+//            run at the same time share the same B (weight) slab through L2.
+//   EPI_LM   the LM head's fused vocabulary reduction.  CTA c keeps m tile
+//            c % m_tiles and walks vocabulary tiles c / m_tiles + k * slots;
+//            each epilogue thread folds every tile of its row into one row
+//            state and writes one LmPart per (row, CTA); logits never leave
+//            the SM.  CTAs with the same slot read the same weight slab at
+//            about the same time (L2 reuse across m tiles).
 #include <cstdio>
 
 #include "kernels.h"
@@ -61,13 +64,35 @@ __device__ __forceinline__ void unit_coords(const TcParams& p, int u, int& m, in
   kb1 = (int)(((long long)(split + 1) * p.kblocks) / p.splits);
 }
 
+// The k-th unit of this CTA.  EPI_F32: units strided over the grid.  EPI_LM:
+// the CTA keeps one m tile and walks the vocabulary tiles slot, slot+slots, ...
+// (slots = gridDim.x / m_tiles), so the epilogue can fold all of them into
+// one row state and write a single partial per (row, CTA).
+template <int EPI>
+__device__ __forceinline__ bool get_unit(const TcParams& p, int k, int& m, int& n, int& kb0,
+                                         int& kb1, int& split) {
+  if constexpr (EPI == EPI_LM) {
+    const int slots = gridDim.x / p.m_tiles;
+    m = blockIdx.x % p.m_tiles;
+    n = blockIdx.x / p.m_tiles + k * slots;
+    kb0 = 0;
+    kb1 = p.kblocks;
+    split = 0;
+    return n < p.n_tiles;
+  } else {
+    const int u = blockIdx.x + k * gridDim.x;
+    if (u >= p.units) return false;
+    unit_coords(p, u, m, n, kb0, kb1);
+    split = (u / p.m_tiles) / p.n_tiles;
+    return true;
+  }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
-  if (p.n_active != nullptr && *p.n_active == 0) return;
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -104,17 +129,21 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above touched only shared and tensor memory
+  pdl_wait_then_release();
+  const bool skip = p.n_active != nullptr && *p.n_active == 0;
 
-  if (warp == 0) {
+  if (skip) {
+    // nothing to do this step: fall through to the teardown
+  } else if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        int m, n, kb0, kb1;
-        unit_coords(p, u, m, n, kb0, kb1);
+      int m, n, kb0, kb1, split;
+      for (int it = 0; ok && get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -153,9 +182,8 @@ __global__ void __launch_bounds__(192, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        int m, n, kb0, kb1;
-        unit_coords(p, u, m, n, kb0, kb1);
+      int m, n, kb0, kb1, split;
+      for (int it = 0; ok && get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -192,9 +220,23 @@ __global__ void __launch_bounds__(192, 1)
     const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-      int m, n, kb0, kb1;
-      unit_coords(p, u, m, n, kb0, kb1);
+    int m = 0, n, kb0, kb1, split;
+    // EPI_LM: one row state for all vocabulary tiles of this CTA
+    RowState rs;
+    rs_init(rs);
+    int lm_row = -1, lm_canvas = 0, lm_pos = 0, lm_step = 0;
+    bool lm_live = false;
+    float lm_inv_t = 1.f;
+    if constexpr (EPI == EPI_LM) {
+      m = blockIdx.x % p.m_tiles;
+      lm_row = m * kBM + quad * 32 + lane;
+      lm_canvas = lm_row / p.epi.C;
+      lm_pos = lm_row - lm_canvas * p.epi.C;
+      lm_live = lm_row < p.M && (p.done == nullptr || p.done[lm_canvas] == 0);
+      lm_step = lm_live ? p.epi.step[lm_canvas] : 0;
+      lm_inv_t = lm_inv_temp(p.epi, lm_step);
+    }
+    for (int it = 0; get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int row0 = m * kBM + quad * 32;
@@ -202,7 +244,6 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
       if (row0 < p.M) {   // warp-uniform: tcgen05.ld is a warp-wide instruction
         if constexpr (EPI == EPI_F32) {
-          const int split = (u / p.m_tiles) / p.n_tiles;
           float* orow = p.out + ((size_t)split * p.M + row) * p.N;
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
@@ -222,20 +263,13 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         } else {
-          const int canvas = row / p.epi.C;
-          const int pos = row - canvas * p.epi.C;
-          const bool live = row < p.M && (p.done == nullptr || p.done[canvas] == 0);
-          const int step = live ? p.epi.step[canvas] : 0;
-          const float inv_t = lm_inv_temp(p.epi, step);
-          RowState rs;
-          rs_init(rs);
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
-            if (live) rs_update<32>(rs, v, n * BN + c, inv_t, p.epi, canvas, pos, step);
+            if (lm_live)
+              rs_update<32>(rs, v, n * BN + c, lm_inv_t, p.epi, lm_canvas, lm_pos, lm_step);
           }
-          if (live) rs_store(p.part + (size_t)row * p.epi.n_tiles + n, rs);
         }
       }
       tc_fence_before();
@@ -243,6 +277,10 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
+    }
+    if constexpr (EPI == EPI_LM) {
+      const int slots = gridDim.x / p.m_tiles;
+      if (lm_live) rs_store(p.part + (size_t)lm_row * slots + blockIdx.x / p.m_tiles, rs);
     }
   }
 
@@ -253,6 +291,18 @@ __global__ void __launch_bounds__(192, 1)
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
+}
+
+// EPI_LM: whole multiples of m_tiles CTAs (each keeps one m tile), at most
+// one CTA per SM per m tile slot; EPI_F32: one CTA per SM or per unit.
+int tc_grid(int units, int m_tiles, int n_tiles, int epi, int num_sms) {
+  if (epi == EPI_LM) {
+    int slots = num_sms / m_tiles;
+    if (slots < 1) slots = 1;
+    if (slots > n_tiles) slots = n_tiles;
+    return slots * m_tiles;
+  }
+  return units < num_sms ? units : num_sms;
 }
 
 template <int BN, int EPI>
@@ -266,9 +316,8 @@ cudaError_t launch_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const TcPa
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int grid = p.units < num_sms ? p.units : num_sms;
-  gemm_tc_kernel<BN, EPI><<<grid, 192, Cfg::kSmem, st>>>(tmA, tmB, p);
-  return cudaGetLastError();
+  const int grid = tc_grid(p.units, p.m_tiles, p.n_tiles, EPI, num_sms);
+  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(192), Cfg::kSmem, st, tmA, tmB, p);
 }
 
 }  // namespace
@@ -300,5 +349,11 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
 }
 
 int gemm_tc_smem_bytes(int BN) { return BN == 128 ? TcCfg<128>::kSmem : TcCfg<256>::kSmem; }
+
+int gemm_tc_lm_partials(const GemmPlan& plan, int num_sms) {
+  const int m_tiles = (plan.M + kBM - 1) / kBM;
+  const int n_tiles = (plan.N + plan.BN - 1) / plan.BN;
+  return tc_grid(m_tiles * n_tiles, m_tiles, n_tiles, EPI_LM, num_sms) / m_tiles;
+}
 
 }  // namespace dlm

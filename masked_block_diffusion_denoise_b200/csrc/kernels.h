@@ -31,6 +31,8 @@ struct GemmIO {
 cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPlan& plan,
                     const GemmIO& io, int num_sms, cudaStream_t st);
 int gemm_tc_smem_bytes(int BN);
+// LM partials per row written by the EPI_LM launch of `plan` (one per CTA slot)
+int gemm_tc_lm_partials(const GemmPlan& plan, int num_sms);
 
 // ---- gemm_simt.cu: fp32 GEMM on the CUDA cores (fp32 model) ----------------
 cudaError_t gemm_f32(const float* A, const float* B, const GemmPlan& plan, const GemmIO& io,
@@ -93,11 +95,6 @@ cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, con
                           const uint8_t* done, const int* n_active, cudaStream_t st);
 
 // ---- select.cu ------------------------------------------------------------------
-// combine LM partials of each row into candidate, confidence and entropy
-cudaError_t lm_reduce(const LmPart* part, int rows, int n_tiles, int C, const uint8_t* done,
-                      const int* n_active, int32_t* cand, float* conf, float* ent,
-                      cudaStream_t st);
-
 struct SelectArgs {
   int B, C, S, V;
   int quota;             // effective quota (>= 1)
@@ -109,9 +106,13 @@ struct SelectArgs {
   uint32_t seed_lo, seed_hi;
 };
 
+// Kernel (c).  With `part` != null it first combines the LM partials of each
+// row of its canvas (n_part per row) into cand / conf / ent (written to those
+// buffers), then selects from them; with part == null it selects from the
+// given cand / conf / ent.
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
-                        uint8_t* done, int32_t* eos_pos, const int32_t* cand, const float* conf,
-                        const float* ent, dlm_canvas_stats* stats, const int* n_active,
-                        int* err, cudaStream_t st);
+                        uint8_t* done, int32_t* eos_pos, const LmPart* part, int n_part,
+                        int32_t* cand, float* conf, float* ent, dlm_canvas_stats* stats,
+                        const int* n_active, int* err, cudaStream_t st);
 
 }  // namespace dlm

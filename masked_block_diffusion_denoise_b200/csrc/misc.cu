@@ -22,6 +22,7 @@ template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ emb,
                              T* __restrict__ x, int rows, int C, int d, int V, int B,
                              const uint8_t* __restrict__ done, int* n_active, int* err) {
+  pdl_wait_then_release();
   if (blockIdx.x == 0 && n_active != nullptr) {
     __shared__ int cnt;
     if (threadIdx.x == 0) cnt = 0;
@@ -53,6 +54,7 @@ __global__ void qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part
                                     const float2* __restrict__ rope, T* __restrict__ q,
                                     T* __restrict__ kc, T* __restrict__ vc,
                                     const uint8_t* __restrict__ done, const int* n_active) {
+  pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.x;
   const int hh = blockIdx.y + head0;
@@ -99,6 +101,7 @@ template <typename T>
 __global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, int rows, int d,
                                    int C, const T* __restrict__ x, T* __restrict__ y,
                                    const uint8_t* __restrict__ done, const int* n_active) {
+  pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.y;
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
@@ -158,13 +161,11 @@ cudaError_t embed_rows(const ModelDims& md, const int32_t* tokens, const void* e
                        int rows, int C, int B, const uint8_t* done, int* n_active, int* err,
                        cudaStream_t st) {
   if (md.esize == 2)
-    embed_kernel<__nv_bfloat16><<<rows, 128, 0, st>>>(
-        tokens, (const __nv_bfloat16*)emb, (__nv_bfloat16*)x, rows, C, md.d, md.V, B, done,
-        n_active, err);
-  else
-    embed_kernel<float><<<rows, 128, 0, st>>>(tokens, (const float*)emb, (float*)x, rows, C,
-                                              md.d, md.V, B, done, n_active, err);
-  return cudaGetLastError();
+    return launch_pdl(embed_kernel<__nv_bfloat16>, dim3(rows), dim3(128), 0, st, tokens,
+                      (const __nv_bfloat16*)emb, (__nv_bfloat16*)x, rows, C, md.d, md.V, B, done,
+                      n_active, err);
+  return launch_pdl(embed_kernel<float>, dim3(rows), dim3(128), 0, st, tokens, (const float*)emb,
+                    (float*)x, rows, C, md.d, md.V, B, done, n_active, err);
 }
 
 cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
@@ -173,14 +174,12 @@ cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int
                          const int* n_active, cudaStream_t st) {
   dim3 grid(rows, md.H + 2 * md.Hkv - head0);
   if (md.esize == 2)
-    qkv_epilogue_kernel<__nv_bfloat16><<<grid, md.Dh / 2, 0, st>>>(
-        md, part, splits, rows, C, seq_fixed, head0, lens, rope, (__nv_bfloat16*)q,
-        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active);
-  else
-    qkv_epilogue_kernel<float><<<grid, md.Dh / 2, 0, st>>>(
-        md, part, splits, rows, C, seq_fixed, head0, lens, rope, (float*)q, (float*)kcache,
-        (float*)vcache, done, n_active);
-  return cudaGetLastError();
+    return launch_pdl(qkv_epilogue_kernel<__nv_bfloat16>, grid, dim3(md.Dh / 2), 0, st, md, part,
+                      splits, rows, C, seq_fixed, head0, lens, rope, (__nv_bfloat16*)q,
+                      (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active);
+  return launch_pdl(qkv_epilogue_kernel<float>, grid, dim3(md.Dh / 2), 0, st, md, part, splits,
+                    rows, C, seq_fixed, head0, lens, rope, (float*)q, (float*)kcache,
+                    (float*)vcache, done, n_active);
 }
 
 cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
@@ -188,12 +187,10 @@ cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int 
                         cudaStream_t st) {
   dim3 grid((md.d + 255) / 256, rows);
   if (md.esize == 2)
-    wo_epilogue_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        part, splits, rows, md.d, C, (const __nv_bfloat16*)x, (__nv_bfloat16*)y, done, n_active);
-  else
-    wo_epilogue_kernel<float><<<grid, 256, 0, st>>>(part, splits, rows, md.d, C,
-                                                    (const float*)x, (float*)y, done, n_active);
-  return cudaGetLastError();
+    return launch_pdl(wo_epilogue_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, part, splits,
+                      rows, md.d, C, (const __nv_bfloat16*)x, (__nv_bfloat16*)y, done, n_active);
+  return launch_pdl(wo_epilogue_kernel<float>, grid, dim3(256), 0, st, part, splits, rows, md.d,
+                    C, (const float*)x, (float*)y, done, n_active);
 }
 
 cudaError_t kv_copy_in(const ModelDims& md, int seq, int n, const void* k, const void* v,

@@ -1,11 +1,10 @@
-// Selection half of the step:
-//   lm_reduce    combines the LM head's per-tile partials of every row into
-//                the candidate token, its confidence and the entropy;
-//   commit_step  kernel (c): one CTA per canvas ranks the uncommitted
-//                positions (bitonic sort in shared memory), applies the
-//                threshold + quota rule or the entropy bound, forces
-//                completion on the last step of the budget, handles EOS,
-//                re-noises the rest and advances step / done.
+// Selection half of the step, one CTA per canvas (kernel (c)):
+//   1. combines the LM head's partials of each row (one per LM-head CTA)
+//      into the candidate token, its confidence and the entropy;
+//   2. ranks the uncommitted positions (bitonic sort in shared memory),
+//      applies the threshold + quota rule or the entropy bound, forces
+//      completion on the last step of the budget, handles EOS, re-noises the
+//      rest and advances step / done.
 // The selection follows the DiffusionGemma page (BlockRefinementScheduler,
 // EntropyBoundScheduler), the course "Diffusion LLMs" section 12 (confidence
 // order, ties to the lower position) and the Nemotron guide, section 6 (the
@@ -15,22 +14,27 @@
 namespace dlm {
 namespace {
 
-__global__ void lm_reduce_kernel(const LmPart* __restrict__ part, int rows, int n_tiles, int C,
-                                 const uint8_t* __restrict__ done, const int* n_active,
-                                 int32_t* __restrict__ cand, float* __restrict__ conf,
-                                 float* __restrict__ ent) {
-  if (n_active != nullptr && *n_active == 0) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= rows) return;
-  if (done != nullptr && done[row / C]) return;
+// combine the n_part partials of one row (a warp) into cand / conf / entropy
+__device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, int32_t* cand,
+                           float* conf, float* ent) {
   RowState acc;
   rs_init(acc);
-  const LmPart* pr = part + (size_t)row * n_tiles;
-  for (int j = lane; j < n_tiles; j += 32) {
-    const LmPart q = pr[j];
-    RowState x{q.m, q.s, q.t, q.g, q.zw, q.idx};
-    acc = rs_combine(acc, x);
+  // issue all loads of a batch before combining (independent L2 reads)
+  constexpr int kU = 8;
+  for (int j0 = 0; j0 < n_part; j0 += 32 * kU) {
+    LmPart q[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int j = j0 + lane + 32 * u;
+      if (j < n_part) q[u] = pr[j];
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (j0 + lane + 32 * u < n_part) {
+        RowState x{q[u].m, q[u].s, q[u].t, q[u].g, q[u].zw, q[u].idx};
+        acc = rs_combine(acc, x);
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -45,13 +49,13 @@ __global__ void lm_reduce_kernel(const LmPart* __restrict__ part, int rows, int 
   }
   if (lane == 0) {
     if (acc.idx == 0x7fffffff || !(acc.s > 0.f)) {
-      cand[row] = 0;
-      conf[row] = 0.f;
-      ent[row] = 0.f;
+      *cand = 0;
+      *conf = 0.f;
+      *ent = 0.f;
     } else {
-      cand[row] = acc.idx;
-      conf[row] = expf(acc.zw - acc.m) / acc.s;
-      ent[row] = logf(acc.s) - acc.t / acc.s;
+      *cand = acc.idx;
+      *conf = expf(acc.zw - acc.m) / acc.s;
+      *ent = logf(acc.s) - acc.t / acc.s;
     }
   }
 }
@@ -86,22 +90,34 @@ __device__ int eos_fill(int32_t* tok, uint8_t* com, int C, int eos_id, int* e_s,
   return e < C ? e : -1;
 }
 
-__global__ void commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
+__global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
                               uint8_t* __restrict__ committed, int32_t* __restrict__ step,
                               uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
-                              const int32_t* __restrict__ cand, const float* __restrict__ conf,
-                              const float* __restrict__ ent, dlm_canvas_stats* stats,
+                              const LmPart* __restrict__ part, int n_part,
+                              int32_t* __restrict__ cand, float* __restrict__ conf,
+                              float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
+  pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   const int b = blockIdx.x;
   if (done[b]) return;
+  if (part != nullptr) {
+    // a6: the cross-tile reduction of this canvas's rows, one warp per row
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int i = warp; i < a.C; i += nw) {
+      const size_t row = (size_t)b * a.C + i;
+      reduce_row(part + row * n_part, n_part, lane, cand + row, conf + row, ent + row);
+    }
+    __syncthreads();
+  }
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
   __shared__ uint8_t com[kMaxC];
   __shared__ int e_s, k_s, krule_s;
   const int i = threadIdx.x;
-  const int P = blockDim.x;
   const int C = a.C;
+  int P = 32;               // keys sorted: the next power of two >= C
+  while (P < C) P <<= 1;
   const size_t base = (size_t)b * C;
   const int s = step[b];
   if (i < C) {
@@ -119,14 +135,14 @@ __global__ void commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
     const uint32_t hi = a.eb ? ordered_bits(ent[base + i]) : ~ordered_bits(conf[base + i]);
     key = ((unsigned long long)hi << 32) | (unsigned)i;
   }
-  keys[i] = key;
+  if (i < P) keys[i] = key;
   const int nU = __syncthreads_count(open);
   const int nthr = __syncthreads_count(open && !a.eb && conf[base + i] >= a.threshold);
 
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       const int ixj = i ^ j;
-      if (ixj > i) {
+      if (i < P && ixj > i) {
         const unsigned long long x = keys[i], y = keys[ixj];
         const bool up = (i & k) == 0;
         if ((x > y) == up) {
@@ -202,25 +218,16 @@ __global__ void commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
 
 }  // namespace
 
-cudaError_t lm_reduce(const LmPart* part, int rows, int n_tiles, int C, const uint8_t* done,
-                      const int* n_active, int32_t* cand, float* conf, float* ent,
-                      cudaStream_t st) {
-  const int rows_per_block = 8;
-  lm_reduce_kernel<<<(rows + rows_per_block - 1) / rows_per_block, 32 * rows_per_block, 0, st>>>(
-      part, rows, n_tiles, C, done, n_active, cand, conf, ent);
-  return cudaGetLastError();
-}
-
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
-                        uint8_t* done, int32_t* eos_pos, const int32_t* cand, const float* conf,
-                        const float* ent, dlm_canvas_stats* stats, const int* n_active,
-                        int* err, cudaStream_t st) {
+                        uint8_t* done, int32_t* eos_pos, const LmPart* part, int n_part,
+                        int32_t* cand, float* conf, float* ent, dlm_canvas_stats* stats,
+                        const int* n_active, int* err, cudaStream_t st) {
   int P = 32;
   while (P < a.C) P <<= 1;
   if (P > kMaxC) return cudaErrorInvalidValue;
-  commit_kernel<<<a.B, P, 0, st>>>(a, tokens, committed, step, done, eos_pos, cand, conf, ent,
-                                   stats, n_active, err);
-  return cudaGetLastError();
+  if (part != nullptr && P < 512) P = 512;   // enough warps for the row reductions
+  return launch_pdl(commit_kernel, dim3(a.B), dim3(P), 0, st, a, tokens, committed, step, done,
+                    eos_pos, part, n_part, cand, conf, ent, stats, n_active, err);
 }
 
 }  // namespace dlm
