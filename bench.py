@@ -121,7 +121,9 @@ class Clocks:
 # distributed plumbing
 # ---------------------------------------------------------------------------
 
-def dist_init(n_gpus):
+def dist_init(n_gpus, backend="nccl"):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE from the launcher);
+    returns (world, rank, local_rank, torch.distributed or None)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -132,18 +134,21 @@ def dist_init(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
         pg = dist
     return world, rank, local, pg
 
 
 def barrier(pg, device):
+    """All ranks meet, then the device drains (the same collective on every rank)."""
     import torch
     if pg is not None:
         t = torch.zeros(1, device=device)
         pg.all_reduce(t)
-    torch.cuda.synchronize(device)
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
 
 
 def max_over_ranks(pg, value, device):
@@ -153,6 +158,11 @@ def max_over_ranks(pg, value, device):
     t = torch.tensor([value], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(world, units_per_rank, ms_max):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -336,7 +346,7 @@ def run_ours(a):
             roof["traffic"] = traffic
         step_s = ms_max / 1e3 / K
         line = {
-            "metric": "denoise steps/s", "value": round(world * K / (ms_max / 1e3), 2),
+            "metric": "denoise steps/s", "value": round(aggregate_rate(world, K, ms_max), 2),
             "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": max(Wm, S),
             "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if sh.dtype == "bf16" else "f32",
@@ -370,11 +380,17 @@ def run_ours(a):
 
 def _ncu_traffic(workload):
     """DRAM bytes per LM-head launch from the committed ncu summary, if it
-    describes this workload and the current kernel."""
+    describes this workload and the kernel sources have not changed since."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "lm_head_%s.json" % workload)
     try:
         with open(path) as f:
-            return json.load(f).get("dram_bytes_per_launch")
+            d = json.load(f)
+        h = hashlib.sha256()
+        for src in d["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return d["dram_bytes_per_launch"] if h.hexdigest() == d["source_sha256"] else None
     except Exception:
         return None
 

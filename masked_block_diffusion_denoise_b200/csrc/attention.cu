@@ -6,14 +6,12 @@
 // epilogue into cache slots len..len+C-1, so the keys of sequence b are cache
 // slots [0, len_b + C).
 //
-// bf16 kernel: one CTA per (key split, 128-query-row tile, sequence x KV
-// head).  The query rows of a CTA are the G = H/Hkv query heads that share
-// the KV head times the C canvas positions (GQA grouping), so each K/V tile
-// is read once for all of them.  A producer warp streams 64-key K and V
-// tiles from HBM with TMA (128-byte swizzle) through a 4-stage ring; eight
-// consumer warps own 16 query rows each and run QK^T and PV with
-// mma.sync m16n8k16 (fp32 accumulate), keeping the online-softmax state
-// (running max, sum) in registers with quad shuffles.  Splits write
+// bf16 kernel (tcgen05): one CTA per (key split, 128-query-row tile,
+// sequence x KV head).  The query rows of a CTA are the G = H/Hkv query heads
+// that share the KV head times the C canvas positions (GQA grouping), so each
+// K/V tile is read once for all of them.  K and V stream from HBM with TMA;
+// S = Q K^T and O += P V run on the tensor cores with S and O in tensor
+// memory; the online softmax keeps one query row per thread.  Splits write
 // unnormalised partials that a second kernel combines (log-sum-exp).
 #include <math_constants.h>
 
@@ -23,14 +21,16 @@ namespace dlm {
 namespace {
 
 constexpr int kDh = 128;
-constexpr int kKT = 64;          // keys per tile
-constexpr int kStages = 4;
-constexpr int kWarps = 8;        // consumer warps
-constexpr int kRowsCta = 16 * kWarps;
-constexpr int kQBytes = kRowsCta * kDh * 2;       // 32 KB
-constexpr int kTileBytes = kKT * kDh * 2;         // 16 KB (K or V)
-constexpr int kStageBytes = 2 * kTileBytes;       // K + V
-constexpr int kAttnSmem = kQBytes + kStages * kStageBytes + 1024 + 128;
+constexpr int kKeys = 128;                    // keys per tile (the N of S = Q K^T)
+constexpr int kRowsCta = 128;                 // query rows per CTA (the M of both MMAs)
+constexpr int kStages = 2;
+constexpr int kHalf = kRowsCta * 128;         // one 64-column half of a 128-row tile: 16 KB
+constexpr int kQBytes = 2 * kHalf;            // Q tile, 32 KB
+constexpr int kPBytes = 2 * kHalf;            // P tile, 32 KB
+constexpr int kStageBytes = 4 * kHalf;        // K and V tiles, two halves each: 64 KB
+constexpr int kAttnSmem = kQBytes + kPBytes + kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 512;           // S double buffer (2 x 128) + O (128)
+constexpr uint32_t kColO = 256;
 
 struct AttnParams {
   const __nv_bfloat16* q;
@@ -45,9 +45,18 @@ struct AttnParams {
   float scale_log2;
 };
 
-__global__ void __launch_bounds__(32 * (kWarps + 1), 1)
-    attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const AttnParams p) {
+// One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
+//   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
+//              128-byte swizzle) into a 2-stage ring;
+//   warp 1     MMA issuer: S(t) = Q K(t)^T into one of two TMEM S buffers
+//              (issued one tile ahead), then O += P(t) V(t) with V as an
+//              MN-major operand;
+//   warps 2-5  softmax: thread = query row = TMEM lane; reads S(t), keeps the
+//              running max and sum (base 2), writes P(t) in bf16 to shared
+//              memory (128-byte swizzle) and rescales O in TMEM.
+__global__ void __launch_bounds__(192, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const AttnParams p) {
   pdl_wait_then_release();
   if (p.n_active != nullptr && *p.n_active == 0) return;
   const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
@@ -57,26 +66,41 @@ __global__ void __launch_bounds__(32 * (kWarps + 1), 1)
   const int k_begin = split * p.chunk;
   if (k_begin >= n_keys) return;
   const int k_end = min(k_begin + p.chunk, n_keys);
-  const int n_tiles = (k_end - k_begin + kKT - 1) / kKT;
+  const int n_tiles = (k_end - k_begin + kKeys - 1) / kKeys;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qs = smem;
-  uint8_t* ring = smem + kQBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  uint8_t* ps = smem + kQBytes;
+  uint8_t* ring = ps + kPBytes;
+  uint64_t* kv_full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
+  uint64_t* kv_empty = kv_full + kStages;
+  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint64_t* mma_done = pv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kWarps);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   // query tile -> shared memory, two 64-column halves, 128-byte swizzle
   for (int idx = tid; idx < kRowsCta * 16; idx += blockDim.x) {
     const int lr = idx >> 4, ch = idx & 15;
@@ -84,193 +108,215 @@ __global__ void __launch_bounds__(32 * (kWarps + 1), 1)
     uint4 val = make_uint4(0, 0, 0, 0);
     if (r < p.R) {
       const int i = r / p.G, hh = r - i * p.G;
-      const __nv_bfloat16* src =
-          p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8;
-      val = *reinterpret_cast<const uint4*>(src);
+      val = *reinterpret_cast<const uint4*>(
+          p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8);
     }
-    *reinterpret_cast<uint4*>(qs + (ch >> 3) * (kRowsCta * 128) + sw128_off(lr, ch & 7)) = val;
+    *reinterpret_cast<uint4*>(qs + (ch >> 3) * kHalf + sw128_off(lr, ch & 7)) = val;
   }
+  fence_proxy_async_smem();
+  tc_fence_before();
   __syncthreads();
-
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
   const int plane = b * p.Hkv + g;
-  if (warp == kWarps) {
+
+  if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
       int issued = 0;
-      bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
-        const int stage = t % kStages;
-        const uint32_t phase = (uint32_t)((t / kStages) & 1);
-        if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+        const int st = t & 1;
+        if (!mbar_wait_bounded(&kv_empty[st], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag)) break;
+        uint8_t* base = ring + st * kStageBytes;
+        const int key0 = k_begin + t * kKeys;
+        mbar_arrive_expect_tx(&kv_full[st], kStageBytes);
+        tma_load_3d(base, &tmK, &kv_full[st], 0, key0, plane);
+        tma_load_3d(base + kHalf, &tmK, &kv_full[st], 64, key0, plane);
+        tma_load_3d(base + 2 * kHalf, &tmV, &kv_full[st], 0, key0, plane);
+        tma_load_3d(base + 3 * kHalf, &tmV, &kv_full[st], 64, key0, plane);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA exits
+        for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
+          mbar_wait_bounded(&kv_full[t & 1], (uint32_t)((t >> 1) & 1), nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsCta, kKeys);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsCta, kDh, true);
+      const uint32_t qaddr = smem_u32(qs), paddr = smem_u32(ps);
+      auto issue_s = [&](int t) {
+        const uint32_t kaddr = smem_u32(ring + (t & 1) * kStageBytes);
+        const uint32_t d = tmem_base + (uint32_t)((t & 1) * kKeys);
+#pragma unroll
+        for (int k = 0; k < kDh / 16; ++k) {
+          const uint32_t off = (uint32_t)((k >> 2) * kHalf + (k & 3) * 32);
+          umma_bf16(d, sw128_desc(qaddr + off), sw128_desc(kaddr + off), idesc_s, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[t & 1]);
+      };
+      bool ok = mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        if (t + 1 < n_tiles) {
+          const int u = (t + 1) >> 1;   // use index of the S buffer
+          if (!mbar_wait_bounded(&kv_full[(t + 1) & 1], (uint32_t)(u & 1), abort_flag) ||
+              (u >= 1 &&
+               !mbar_wait_bounded(&s_free[(t + 1) & 1], (uint32_t)((u - 1) & 1), abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(t + 1);
+        }
+        if (!mbar_wait_bounded(p_full, (uint32_t)(t & 1), abort_flag)) {
           ok = false;
           break;
         }
-        uint8_t* ks = ring + stage * kStageBytes;
-        uint8_t* vs = ks + kTileBytes;
-        const int key0 = k_begin + t * kKT;
-        mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        tma_load_3d(ks, &tmK, &full[stage], 0, key0, plane);
-        tma_load_3d(ks + kTileBytes / 2, &tmK, &full[stage], 64, key0, plane);
-        tma_load_3d(vs, &tmV, &full[stage], 0, key0, plane);
-        tma_load_3d(vs + kTileBytes / 2, &tmV, &full[stage], 64, key0, plane);
-        ++issued;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(ring + (t & 1) * kStageBytes + 2 * kHalf);
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k) {
+          const uint64_t adesc =
+              sw128_desc(paddr + (uint32_t)((k >> 2) * kHalf + (k & 3) * 32));
+          const uint64_t bdesc = sw128_desc_mn(vaddr + (uint32_t)(k * 2048), kHalf);
+          umma_bf16(tmem_base + kColO, adesc, bdesc, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done);
+        umma_commit(&kv_empty[t & 1]);
       }
-      if (!ok) {
-        for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
-          mbar_wait_bounded(&full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
-        raise_error(p.err, DLM_ETIMEOUT);
+      umma_commit(mma_done);
+      mbar_wait_bounded(mma_done, 0, nullptr);
+    }
+  } else {
+    // ---------------- softmax warps ----------------
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;                 // query row within the tile = TMEM lane
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int buf = t & 1;
+      if (!mbar_wait_bounded(&s_full[buf], (uint32_t)((t >> 1) & 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) {
+        float v[32];
+        tmem_ld32(lane_addr + (uint32_t)(buf * kKeys + c * 32), v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[c * 32 + j] = v[j];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[buf]);
+      const int key_base = k_begin + t * kKeys;
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int j = 0; j < kKeys; ++j) {
+        const float v = (key_base + j < k_end) ? sv[j] * p.scale_log2 : -CUDART_INF_F;
+        sv[j] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const float alpha = fast_exp2(m_run - m_new);
+      float rsum = 0.f;
+#pragma unroll
+      for (int j = 0; j < kKeys; ++j) {
+        const float e = fast_exp2(sv[j] - m_new);
+        sv[j] = e;
+        rsum += e;
+      }
+      l_run = l_run * alpha + rsum;
+      m_run = m_new;
+      if (t > 0) {
+        // the previous P V has finished: P may be overwritten, O is stable
+        if (!mbar_wait_bounded(pv_done, (uint32_t)((t - 1) & 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < kKeys / 8; ++c) {
+        uint4 w;
+        w.x = pack_bf16(sv[8 * c + 0], sv[8 * c + 1]);
+        w.y = pack_bf16(sv[8 * c + 2], sv[8 * c + 3]);
+        w.z = pack_bf16(sv[8 * c + 4], sv[8 * c + 5]);
+        w.w = pack_bf16(sv[8 * c + 6], sv[8 * c + 7]);
+        *reinterpret_cast<uint4*>(ps + (c >> 3) * kHalf + sw128_off(row, c & 7)) = w;
+      }
+      if (t > 0) {
+#pragma unroll
+        for (int c = 0; c < kDh / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + kColO + (uint32_t)(c * 32), o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] *= alpha;
+          tmem_st32(lane_addr + kColO + (uint32_t)(c * 32), o);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait_bounded(pv_done, (uint32_t)((n_tiles - 1) & 1), abort_flag)) {
+      tc_fence_after();
+      const int r = rt * kRowsCta + row;
+      float ov[kDh];
+#pragma unroll
+      for (int c = 0; c < kDh / 32; ++c) {
+        float v[32];
+        tmem_ld32(lane_addr + kColO + (uint32_t)(c * 32), v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ov[c * 32 + j] = v[j];
+      }
+      if (r < p.R) {
+        if (p.nsplit == 1) {
+          const int i = r / p.G, hh = r - i * p.G;
+          __nv_bfloat16* dst = p.o + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh;
+          const float inv = 1.f / l_run;
+#pragma unroll
+          for (int c = 0; c < kDh / 8; ++c) {
+            uint4 w;
+            w.x = pack_bf16(ov[8 * c + 0] * inv, ov[8 * c + 1] * inv);
+            w.y = pack_bf16(ov[8 * c + 2] * inv, ov[8 * c + 3] * inv);
+            w.z = pack_bf16(ov[8 * c + 4] * inv, ov[8 * c + 5] * inv);
+            w.w = pack_bf16(ov[8 * c + 6] * inv, ov[8 * c + 7] * inv);
+            reinterpret_cast<uint4*>(dst)[c] = w;
+          }
+        } else {
+          const size_t slot = ((size_t)bg * p.nsplit + split) * p.R + r;
+          float4* dst = reinterpret_cast<float4*>(p.opart + slot * kDh);
+#pragma unroll
+          for (int c = 0; c < kDh / 4; ++c)
+            dst[c] = make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3]);
+          p.ml[slot] = make_float2(m_run, l_run);
+        }
       }
     }
-    return;
   }
 
-  // ---------------- consumers: 16 query rows per warp ----------------
-  uint32_t qf[8][4];
-  {
-    const int mi = lane >> 3;
-    const int row = warp * 16 + (lane & 7) + (mi & 1) * 8;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int ch = 2 * ks + (mi >> 1);
-      ldsm_x4(smem_u32(qs + (ch >> 3) * (kRowsCta * 128) + sw128_off(row, ch & 7)), qf[ks][0],
-              qf[ks][1], qf[ks][2], qf[ks][3]);
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
   }
-  float oacc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};
-  float l_run[2] = {0.f, 0.f};
-
-  bool ok = true;
-  for (int t = 0; t < n_tiles; ++t) {
-    const int stage = t % kStages;
-    const uint32_t phase = (uint32_t)((t / kStages) & 1);
-    if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
-      ok = false;
-      break;
-    }
-    const uint8_t* ks = ring + stage * kStageBytes;
-    const uint8_t* vs = ks + kTileBytes;
-
-    // S = Q K^T over 64 keys
-    float sc[8][4];
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
-      const int key = nb * 8 + (lane & 7);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int ch = 4 * j + (lane >> 3);
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4(smem_u32(ks + (ch >> 3) * (kTileBytes / 2) + sw128_off(key, ch & 7)), r0, r1, r2,
-                r3);
-        mma_bf16_16816(sc[nb], qf[2 * j], r0, r1);
-        mma_bf16_16816(sc[nb], qf[2 * j + 1], r2, r3);
-      }
-    }
-    // scale to base 2, mask keys past the end, online softmax
-    const int key_base = k_begin + t * kKT;
-    float mx[2] = {-CUDART_INF_F, -CUDART_INF_F};
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key_base + nb * 8 + 2 * (lane & 3) + (e & 1);
-        const float v = (key < k_end) ? sc[nb][e] * p.scale_log2 : -CUDART_INF_F;
-        sc[nb][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-    float alpha[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-      const float m_new = fmaxf(m_run[h], mx[h]);
-      alpha[h] = fast_exp2(m_run[h] - m_new);
-      m_run[h] = m_new;
-    }
-    float rsum[2] = {0.f, 0.f};
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float pv = fast_exp2(sc[nb][e] - m_run[e >> 1]);
-        sc[nb][e] = pv;
-        rsum[e >> 1] += pv;
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) l_run[h] = l_run[h] * alpha[h] + rsum[h];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      oacc[i][0] *= alpha[0];
-      oacc[i][1] *= alpha[0];
-      oacc[i][2] *= alpha[1];
-      oacc[i][3] *= alpha[1];
-    }
-    // O += P V
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pf[4];
-      pf[0] = pack_bf16(sc[2 * kk][0], sc[2 * kk][1]);
-      pf[1] = pack_bf16(sc[2 * kk][2], sc[2 * kk][3]);
-      pf[2] = pack_bf16(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-      pf[3] = pack_bf16(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-      const int mi = lane >> 3;
-      const int key = kk * 16 + (lane & 7) + (mi & 1) * 8;
-#pragma unroll
-      for (int nbp = 0; nbp < 8; ++nbp) {
-        const int blk = 2 * nbp + (mi >> 1);
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4_t(smem_u32(vs + (blk >> 3) * (kTileBytes / 2) + sw128_off(key, blk & 7)), r0, r1,
-                  r2, r3);
-        mma_bf16_16816(oacc[2 * nbp], pf, r0, r1);
-        mma_bf16_16816(oacc[2 * nbp + 1], pf, r2, r3);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
-  }
-  if (!ok) {
-    if (lane == 0) raise_error(p.err, DLM_ETIMEOUT);
-    return;
-  }
-
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
-    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
-  }
-  const int rbase = rt * kRowsCta + warp * 16 + (lane >> 2);
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int r = rbase + h * 8;
-    if (r >= p.R) continue;
-    if (p.nsplit == 1) {
-      const int i = r / p.G, hh = r - i * p.G;
-      __nv_bfloat16* dst = p.o + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh;
-      const float inv = 1.f / l_run[h];
-#pragma unroll
-      for (int nb = 0; nb < 16; ++nb) {
-        const int dh = nb * 8 + 2 * (lane & 3);
-        *reinterpret_cast<__nv_bfloat162*>(dst + dh) =
-            __floats2bfloat162_rn(oacc[nb][2 * h] * inv, oacc[nb][2 * h + 1] * inv);
-      }
-    } else {
-      const size_t slot = ((size_t)bg * p.nsplit + split) * p.R + r;
-      float* dst = p.opart + slot * kDh;
-#pragma unroll
-      for (int nb = 0; nb < 16; ++nb) {
-        const int dh = nb * 8 + 2 * (lane & 3);
-        *reinterpret_cast<float2*>(dst + dh) = make_float2(oacc[nb][2 * h], oacc[nb][2 * h + 1]);
-      }
-      if ((lane & 3) == 0) p.ml[slot] = make_float2(m_run[h], l_run[h]);
-    }
-  }
+  if (tid == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
 }
 
 // log-sum-exp combination of the splits of one (sequence, KV head); one warp
@@ -416,7 +462,7 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
                            const int* n_active, int* err, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -439,8 +485,7 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.nsplit = ap.nsplit;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
-  cudaError_t e = launch_pdl(attn_bf16_kernel, grid, dim3(32 * (kWarps + 1)), kAttnSmem, st, tmK,
-                             tmV, p);
+  cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kAttnSmem, st, tmK, tmV, p);
   if (e != cudaSuccess || ap.nsplit == 1) return e;
   const int rows_per_block = 8;
   dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);

@@ -146,7 +146,7 @@ bool map_kv(CUtensorMap* m, void* base, uint64_t planes, uint64_t Lcap, uint64_t
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {Dh, Lcap, planes};
   cuuint64_t strides[2] = {Dh * 2, Lcap * Dh * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, 128, 1};   // 64 head-dim columns x 128 keys (one attention tile half)
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -213,7 +213,7 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, int max_keys) {
   const int nbg = B * ctx->md.Hkv * a.rtiles;
   long best_cost = -1;
   for (int ns = 1; ns <= 64; ++ns) {
-    const int chunk = cdiv(cdiv(max_keys, ns), 64) * 64;
+    const int chunk = cdiv(cdiv(max_keys, ns), 128) * 128;   // whole 128-key attention tiles
     const int nse = cdiv(max_keys, chunk);
     if (nse != ns) continue;
     const long waves = cdiv(nbg * nse, ctx->num_sms);

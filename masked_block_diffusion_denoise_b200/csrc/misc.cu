@@ -47,18 +47,16 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
   for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
 }
 
+// block (row, group of heads): one rotary pair (j, j + Dh/2) per thread
 template <typename T>
-__global__ void qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part, int splits,
-                                    int rows, int C, int seq_fixed, int head0,
-                                    const int32_t* __restrict__ lens,
-                                    const float2* __restrict__ rope, T* __restrict__ q,
-                                    T* __restrict__ kc, T* __restrict__ vc,
-                                    const uint8_t* __restrict__ done, const int* n_active) {
+__global__ void __launch_bounds__(256)
+    qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part, int splits, int rows, int C,
+                        int seq_fixed, int head0, const int32_t* __restrict__ lens,
+                        const float2* __restrict__ rope, T* __restrict__ q, T* __restrict__ kc,
+                        T* __restrict__ vc, const uint8_t* __restrict__ done, const int* n_active) {
   pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.x;
-  const int hh = blockIdx.y + head0;
-  const int j = threadIdx.x;
   const int half = md.Dh / 2;
   int seq, p_in;
   if (seq_fixed >= 0) {
@@ -70,31 +68,39 @@ __global__ void qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part
     if (done != nullptr && done[seq]) return;
   }
   const int pos = lens[seq] + p_in;
-  const int ncols = (md.H + 2 * md.Hkv - head0) * md.Dh;
-  const int cb = (hh - head0) * md.Dh;
-  float a = 0.f, b = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* pr = part + ((size_t)s * rows + r) * ncols + cb;
-    a += pr[j];
-    b += pr[j + half];
+  const int nheads = md.H + 2 * md.Hkv - head0;
+  const int ncols = nheads * md.Dh;
+  const int per_block = blockDim.x / half;
+  {
+    const int item = blockIdx.y * per_block * half + threadIdx.x;
+    if (item >= nheads * half) return;
+    const int hl = item / half, j = item - hl * half;
+    const int hh = hl + head0;
+    const int cb = hl * md.Dh;
+    float a = 0.f, b = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float* pr = part + ((size_t)s * rows + r) * ncols + cb;
+      a += pr[j];
+      b += pr[j + half];
+    }
+    if (rope != nullptr && hh < md.H + md.Hkv) {
+      const float2 cs = rope[(size_t)pos * half + j];
+      const float a2 = a * cs.x - b * cs.y;
+      const float b2 = b * cs.x + a * cs.y;
+      a = a2;
+      b = b2;
+    }
+    T* dst;
+    if (hh < md.H) {
+      dst = q + ((size_t)r * md.H + hh) * md.Dh;
+    } else if (hh < md.H + md.Hkv) {
+      dst = kc + (((size_t)seq * md.Hkv + (hh - md.H)) * md.Lcap + pos) * md.Dh;
+    } else {
+      dst = vc + (((size_t)seq * md.Hkv + (hh - md.H - md.Hkv)) * md.Lcap + pos) * md.Dh;
+    }
+    dst[j] = from_f32<T>(a);
+    dst[j + half] = from_f32<T>(b);
   }
-  if (rope != nullptr && hh < md.H + md.Hkv) {
-    const float2 cs = rope[(size_t)pos * half + j];
-    const float a2 = a * cs.x - b * cs.y;
-    const float b2 = b * cs.x + a * cs.y;
-    a = a2;
-    b = b2;
-  }
-  T* dst;
-  if (hh < md.H) {
-    dst = q + ((size_t)r * md.H + hh) * md.Dh;
-  } else if (hh < md.H + md.Hkv) {
-    dst = kc + (((size_t)seq * md.Hkv + (hh - md.H)) * md.Lcap + pos) * md.Dh;
-  } else {
-    dst = vc + (((size_t)seq * md.Hkv + (hh - md.H - md.Hkv)) * md.Lcap + pos) * md.Dh;
-  }
-  dst[j] = from_f32<T>(a);
-  dst[j + half] = from_f32<T>(b);
 }
 
 template <typename T>
@@ -172,12 +178,14 @@ cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int
                          int seq_fixed, int head0, const int32_t* lens, const float2* rope,
                          void* q, void* kcache, void* vcache, const uint8_t* done,
                          const int* n_active, cudaStream_t st) {
-  dim3 grid(rows, md.H + 2 * md.Hkv - head0);
+  const int half = md.Dh / 2;
+  const int per_block = 256 / half;   // heads per block
+  dim3 grid(rows, (md.H + 2 * md.Hkv - head0 + per_block - 1) / per_block);
   if (md.esize == 2)
-    return launch_pdl(qkv_epilogue_kernel<__nv_bfloat16>, grid, dim3(md.Dh / 2), 0, st, md, part,
+    return launch_pdl(qkv_epilogue_kernel<__nv_bfloat16>, grid, dim3(per_block * half), 0, st, md, part,
                       splits, rows, C, seq_fixed, head0, lens, rope, (__nv_bfloat16*)q,
                       (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active);
-  return launch_pdl(qkv_epilogue_kernel<float>, grid, dim3(md.Dh / 2), 0, st, md, part, splits,
+  return launch_pdl(qkv_epilogue_kernel<float>, grid, dim3(per_block * half), 0, st, md, part, splits,
                     rows, C, seq_fixed, head0, lens, rope, (float*)q, (float*)kcache,
                     (float*)vcache, done, n_active);
 }
