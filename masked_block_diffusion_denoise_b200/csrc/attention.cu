@@ -23,13 +23,12 @@ namespace {
 constexpr int kDh = 128;
 constexpr int kKeys = 128;                    // keys per tile (the N of S = Q K^T)
 constexpr int kRowsCta = 128;                 // query rows per CTA (the M of both MMAs)
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kHalf = kRowsCta * 128;         // one 64-column half of a 128-row tile: 16 KB
 constexpr int kQBytes = 2 * kHalf;            // Q tile, 32 KB
-constexpr int kPBytes = 2 * kHalf;            // P tile, 32 KB
 constexpr int kStageBytes = 4 * kHalf;        // K and V tiles, two halves each: 64 KB
-constexpr int kAttnSmem = kQBytes + kPBytes + kStages * kStageBytes + 1024 + 256;
-constexpr uint32_t kTmemCols = 512;           // S double buffer (2 x 128) + O (128)
+constexpr int kAttnSmem = kQBytes + kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 512;           // S/P double buffer (2 x 128) + O (128)
 constexpr uint32_t kColO = 256;
 
 struct AttnParams {
@@ -47,13 +46,15 @@ struct AttnParams {
 
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
 //   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
-//              128-byte swizzle) into a 2-stage ring;
-//   warp 1     MMA issuer: S(t) = Q K(t)^T into one of two TMEM S buffers
-//              (issued one tile ahead), then O += P(t) V(t) with V as an
-//              MN-major operand;
+//              128-byte swizzle) into a 3-stage ring;
+//   warp 1     MMA issuer: S(t) = Q K(t)^T into TMEM buffer t % 2, issued one
+//              tile ahead; then O += P(t) V(t), P read from TMEM (bf16 pairs
+//              written over S(t)), V as an MN-major shared-memory operand;
 //   warps 2-5  softmax: thread = query row = TMEM lane; reads S(t), keeps the
-//              running max and sum (base 2), writes P(t) in bf16 to shared
-//              memory (128-byte swizzle) and rescales O in TMEM.
+//              running max and sum (base 2), writes P(t) to TMEM and, only
+//              when a row's maximum moved, rescales O in TMEM.
+// tcgen05 operations of the issuing thread run in order, so S(t+2) cannot
+// overwrite P(t) before P(t) V(t) has read it.
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const AttnParams p) {
@@ -72,13 +73,11 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* qs = smem;
-  uint8_t* ps = smem + kQBytes;
-  uint8_t* ring = ps + kPBytes;
+  uint8_t* ring = smem + kQBytes;
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
+  uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 1;
   uint64_t* mma_done = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -90,10 +89,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
@@ -127,8 +123,9 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch(&tmV);
       int issued = 0;
       for (int t = 0; t < n_tiles; ++t) {
-        const int st = t & 1;
-        if (!mbar_wait_bounded(&kv_empty[st], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag)) break;
+        const int st = t % kStages;
+        if (!mbar_wait_bounded(&kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag))
+          break;
         uint8_t* base = ring + st * kStageBytes;
         const int key0 = k_begin + t * kKeys;
         mbar_arrive_expect_tx(&kv_full[st], kStageBytes);
@@ -141,7 +138,7 @@ __global__ void __launch_bounds__(192, 1)
       if (*abort_flag) {
         // let the copies already in flight land before the CTA exits
         for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
-          mbar_wait_bounded(&kv_full[t & 1], (uint32_t)((t >> 1) & 1), nullptr);
+          mbar_wait_bounded(&kv_full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
       }
     }
   } else if (warp == 1) {
@@ -149,9 +146,9 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsCta, kKeys);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsCta, kDh, true);
-      const uint32_t qaddr = smem_u32(qs), paddr = smem_u32(ps);
+      const uint32_t qaddr = smem_u32(qs);
       auto issue_s = [&](int t) {
-        const uint32_t kaddr = smem_u32(ring + (t & 1) * kStageBytes);
+        const uint32_t kaddr = smem_u32(ring + (t % kStages) * kStageBytes);
         const uint32_t d = tmem_base + (uint32_t)((t & 1) * kKeys);
 #pragma unroll
         for (int k = 0; k < kDh / 16; ++k) {
@@ -167,31 +164,30 @@ __global__ void __launch_bounds__(192, 1)
       }
       for (int t = 0; ok && t < n_tiles; ++t) {
         if (t + 1 < n_tiles) {
-          const int u = (t + 1) >> 1;   // use index of the S buffer
-          if (!mbar_wait_bounded(&kv_full[(t + 1) & 1], (uint32_t)(u & 1), abort_flag) ||
-              (u >= 1 &&
-               !mbar_wait_bounded(&s_free[(t + 1) & 1], (uint32_t)((u - 1) & 1), abort_flag))) {
+          const int t1 = t + 1;
+          if (!mbar_wait_bounded(&kv_full[t1 % kStages], (uint32_t)((t1 / kStages) & 1),
+                                 abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_s(t + 1);
+          issue_s(t1);
         }
         if (!mbar_wait_bounded(p_full, (uint32_t)(t & 1), abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t vaddr = smem_u32(ring + (t & 1) * kStageBytes + 2 * kHalf);
+        const uint32_t vaddr = smem_u32(ring + (t % kStages) * kStageBytes + 2 * kHalf);
+        const uint32_t pcol = tmem_base + (uint32_t)((t & 1) * kKeys);
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k) {
-          const uint64_t adesc =
-              sw128_desc(paddr + (uint32_t)((k >> 2) * kHalf + (k & 3) * 32));
           const uint64_t bdesc = sw128_desc_mn(vaddr + (uint32_t)(k * 2048), kHalf);
-          umma_bf16(tmem_base + kColO, adesc, bdesc, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem_base + kColO, pcol + (uint32_t)(k * 8), bdesc, idesc_o,
+                           (t > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(pv_done);
-        umma_commit(&kv_empty[t & 1]);
+        umma_commit(&kv_empty[t % kStages]);
       }
       umma_commit(mma_done);
       mbar_wait_bounded(mma_done, 0, nullptr);
@@ -211,53 +207,54 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       float sv[kKeys];
+      {
+        uint32_t raw[kKeys / 32][32];
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        float v[32];
-        tmem_ld32(lane_addr + (uint32_t)(buf * kKeys + c * 32), v);
+        for (int c = 0; c < kKeys / 32; ++c)
+          tmem_ld32_nowait(lane_addr + (uint32_t)(buf * kKeys + c * 32), raw[c]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sv[c * 32 + j] = v[j];
+        for (int c = 0; c < kKeys / 32; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(raw[c][j]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[buf]);
       const int key_base = k_begin + t * kKeys;
+      if (key_base + kKeys > k_end) {   // ragged last tile (warp-uniform): mask past the end
+#pragma unroll
+        for (int j = 0; j < kKeys; ++j)
+          if (key_base + j >= k_end) sv[j] = -CUDART_INF_F;
+      }
+      // maximum on the raw scores (the scale is positive), then one FFMA per score
       float mx = -CUDART_INF_F;
 #pragma unroll
-      for (int j = 0; j < kKeys; ++j) {
-        const float v = (key_base + j < k_end) ? sv[j] * p.scale_log2 : -CUDART_INF_F;
-        sv[j] = v;
-        mx = fmaxf(mx, v);
-      }
-      const float m_new = fmaxf(m_run, mx);
+      for (int j = 0; j < kKeys; ++j) mx = fmaxf(mx, sv[j]);
+      const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const float alpha = fast_exp2(m_run - m_new);
       float rsum = 0.f;
 #pragma unroll
       for (int j = 0; j < kKeys; ++j) {
-        const float e = fast_exp2(sv[j] - m_new);
+        const float e = fast_exp2(fmaf(sv[j], p.scale_log2, -m_new));
         sv[j] = e;
         rsum += e;
       }
       l_run = l_run * alpha + rsum;
       m_run = m_new;
-      if (t > 0) {
-        // the previous P V has finished: P may be overwritten, O is stable
+      // P(t) in bf16, two keys per 32-bit TMEM column, over the S(t) columns
+#pragma unroll
+      for (int c = 0; c < kKeys / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = pack_bf16(sv[64 * c + 2 * j], sv[64 * c + 2 * j + 1]);
+        tmem_st32_u(lane_addr + (uint32_t)(buf * kKeys + c * 32), w);
+      }
+      // rescale O only when some row of the warp saw a new maximum; O must
+      // first hold every earlier P V
+      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!mbar_wait_bounded(pv_done, (uint32_t)((t - 1) & 1), abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-#pragma unroll
-      for (int c = 0; c < kKeys / 8; ++c) {
-        uint4 w;
-        w.x = pack_bf16(sv[8 * c + 0], sv[8 * c + 1]);
-        w.y = pack_bf16(sv[8 * c + 2], sv[8 * c + 3]);
-        w.z = pack_bf16(sv[8 * c + 4], sv[8 * c + 5]);
-        w.w = pack_bf16(sv[8 * c + 6], sv[8 * c + 7]);
-        *reinterpret_cast<uint4*>(ps + (c >> 3) * kHalf + sw128_off(row, c & 7)) = w;
-      }
-      if (t > 0) {
 #pragma unroll
         for (int c = 0; c < kDh / 32; ++c) {
           float o[32];
@@ -266,9 +263,8 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < 32; ++j) o[j] *= alpha;
           tmem_st32(lane_addr + kColO + (uint32_t)(c * 32), o);
         }
-        tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
@@ -277,12 +273,16 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int r = rt * kRowsCta + row;
       float ov[kDh];
+      {
+        uint32_t raw[kDh / 32][32];
 #pragma unroll
-      for (int c = 0; c < kDh / 32; ++c) {
-        float v[32];
-        tmem_ld32(lane_addr + kColO + (uint32_t)(c * 32), v);
+        for (int c = 0; c < kDh / 32; ++c)
+          tmem_ld32_nowait(lane_addr + kColO + (uint32_t)(c * 32), raw[c]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ov[c * 32 + j] = v[j];
+        for (int c = 0; c < kDh / 32; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[c * 32 + j] = __uint_as_float(raw[c][j]);
       }
       if (r < p.R) {
         if (p.nsplit == 1) {

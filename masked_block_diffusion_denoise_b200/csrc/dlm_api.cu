@@ -203,25 +203,50 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
   return p;
 }
 
-AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, int max_keys) {
+// Split plan of the attention: every chunk size (whole 128-key tiles) is
+// costed by list-scheduling the CTAs in launch order (split fastest, one CTA
+// per SM) with a per-tile time, a per-CTA fixed time and the combine's cost
+// per partial; ragged prefixes (lens, host) are taken as they are.
+AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int max_len_all) {
   AttnPlan a{};
   a.B = B;
   a.C = C;
   a.G = ctx->md.H / ctx->md.Hkv;
   a.R = a.G * C;
   a.rtiles = cdiv(a.R, 128);
-  const int nbg = B * ctx->md.Hkv * a.rtiles;
-  long best_cost = -1;
-  for (int ns = 1; ns <= 64; ++ns) {
-    const int chunk = cdiv(cdiv(max_keys, ns), 128) * 128;   // whole 128-key attention tiles
-    const int nse = cdiv(max_keys, chunk);
-    if (nse != ns) continue;
-    const long waves = cdiv(nbg * nse, ctx->num_sms);
-    const long cost = waves * chunk + 16L * nse;
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
+  const int Hkv = ctx->md.Hkv;
+  const int sms = std::min(std::max(ctx->num_sms, 1), 1024);
+  const int max_keys = max_len_all + C;
+  const int max_tiles = cdiv(max_keys, 128);
+  const double t_tile = 2.0, t_cta = 2.0, t_comb = 3.0, t_part = 0.02;   // microseconds
+  double best = -1.0;
+  double sm_free[1024];   // no heap: this also runs inside dlm_attention_noalloc
+  for (int ct = 1; ct <= max_tiles; ++ct) {
+    const int chunk = ct * 128;
+    const int nsplit = cdiv(max_keys, chunk);
+    if (nsplit > 64) continue;
+    std::fill(sm_free, sm_free + sms, 0.0);
+    long partials = 0;
+    double makespan = 0.0;
+    for (int bg = 0; bg < B * Hkv; ++bg) {
+      const int keys = (lens ? lens[bg / Hkv] : max_len_all) + C;
+      for (int rt = 0; rt < a.rtiles; ++rt) {
+        for (int sp = 0; sp < nsplit; ++sp) {
+          const int k0 = sp * chunk;
+          if (k0 >= keys) continue;   // exits at once
+          const int tiles = cdiv(std::min(chunk, keys - k0), 128);
+          double* it = std::min_element(sm_free, sm_free + sms);
+          *it += t_cta + tiles * t_tile;
+          makespan = std::max(makespan, *it);
+          ++partials;
+        }
+      }
+    }
+    const double cost = makespan + (nsplit > 1 ? t_comb + t_part * partials : 0.0);
+    if (best < 0.0 || cost < best - 1e-9) {
+      best = cost;
       a.chunk = chunk;
-      a.nsplit = nse;
+      a.nsplit = nsplit;
     }
   }
   return a;
@@ -663,7 +688,7 @@ int dlm_denoise_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
   if (int rc = check_canvas(ctx, c)) return rc;
-  AttnPlan ap = plan_attention(ctx, batch, p->canvas, max_len(ctx, batch) + p->canvas);
+  AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
   ctx->launches = 0;
@@ -676,7 +701,7 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
   if (int rc = check_canvas(ctx, c)) return rc;
-  AttnPlan ap = plan_attention(ctx, batch, p->canvas, max_len(ctx, batch) + p->canvas);
+  AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
   // the graph bakes in pointers, sizes, parameters and the attention plan
@@ -914,7 +939,7 @@ int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cach
   dlm_ctx plan_ctx;
   plan_ctx.md = ModelDims{0, n_heads, n_kv_heads, head_dim, 0, -1, -1, kv_capacity, 2};
   cudaDeviceGetAttribute(&plan_ctx.num_sms, cudaDevAttrMultiProcessorCount, dev);
-  const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, max_len + canvas);
+  const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, nullptr, max_len);
   const long slots = (long)batch * n_kv_heads * ap.nsplit * ap.R;
   if (ap.nsplit > 1 && slots > kNoAllocSlots) {
     g_create_error = "attention_noalloc: the split plan needs " + std::to_string(slots) +

@@ -93,40 +93,40 @@ __device__ __forceinline__ void rs_update(RowState& r, const float (&v)[N], int 
     }
     r.m = cmax;
   }
+  // branch-free: masked columns contribute exactly zero (selects, not branches,
+  // so independent work of the chunk can interleave)
 #pragma unroll
   for (int j = 0; j < N; ++j) {
-    if (z[j] != -CUDART_INF_F) {
-      const float d = z[j] - r.m;
-      const float ex = __expf(d);
-      r.s += ex;
-      r.t = fmaf(ex, d, r.t);
-    }
+    const bool valid = z[j] != -CUDART_INF_F;
+    const float d = valid ? z[j] - r.m : 0.f;
+    const float ex = valid ? __expf(d) : 0.f;
+    r.s += ex;
+    r.t = fmaf(ex, d, r.t);
   }
   if (e.mode == LM_GREEDY) {
     // columns arrive in increasing order: on equal values the earlier wins
-    if (cmax > r.g) {
-      r.g = cmax;
-      r.zw = cmax;
-      r.idx = col0 + carg;
-    }
+    const bool better = cmax > r.g;
+    r.g = better ? cmax : r.g;
+    r.zw = better ? cmax : r.zw;
+    r.idx = better ? col0 + carg : r.idx;
   } else {
+    U32x4 w[N / 4];
 #pragma unroll
-    for (int j4 = 0; j4 < N; j4 += 4) {
-      const int col = col0 + j4;
-      const U32x4 w = philox10(U32x4{(uint32_t)canvas, (uint32_t)step, (uint32_t)pos,
-                                     (uint32_t)(col >> 2)},
-                               e.seed_lo, e.seed_hi);
-      const uint32_t ws[4] = {w.a, w.b, w.c, w.d};
+    for (int j4 = 0; j4 < N / 4; ++j4)
+      w[j4] = philox10(U32x4{(uint32_t)canvas, (uint32_t)step, (uint32_t)pos,
+                             (uint32_t)((col0 >> 2) + j4)},
+                       e.seed_lo, e.seed_hi);
+#pragma unroll
+    for (int j4 = 0; j4 < N / 4; ++j4) {
+      const uint32_t ws[4] = {w[j4].a, w[j4].b, w[j4].c, w[j4].d};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float zj = z[j4 + q];
-        if (zj == -CUDART_INF_F) continue;
-        const float gj = zj + gumbel_from_bits(ws[q]);
-        if (gj > r.g) {
-          r.g = gj;
-          r.zw = zj;
-          r.idx = col + q;
-        }
+        const float zj = z[4 * j4 + q];
+        const float gj = zj + gumbel_from_bits(ws[q]);   // -inf stays -inf
+        const bool better = gj > r.g;                     // ties keep the lower index
+        r.g = better ? gj : r.g;
+        r.zw = better ? zj : r.zw;
+        r.idx = better ? col0 + 4 * j4 + q : r.idx;
       }
     }
   }
