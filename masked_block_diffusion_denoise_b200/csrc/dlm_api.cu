@@ -198,8 +198,14 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
     p.BN = mt > 1 ? 256 : 128;
     return p;
   }
-  p.BN = (mt > 1 && mt * cdiv(N, 128) >= 4 * ctx->num_sms) ? 256 : 128;
-  if (mt == 1) p.splits = pick_splits(cdiv(N, p.BN), cdiv(K, 64), ctx->num_sms, 16);
+  if (mt > 1) {
+    // tensor-bound: 256-wide tiles (less L2 traffic per flop), K not split,
+    // so the projection epilogues can be fused into the GEMM
+    p.BN = 256;
+    return p;
+  }
+  p.BN = 128;
+  p.splits = pick_splits(cdiv(N, p.BN), cdiv(K, 64), ctx->num_sms, 16);
   return p;
 }
 
@@ -385,6 +391,24 @@ int stage_event(dlm_ctx* ctx, int stage, bool end, cudaStream_t st) {
     if (int rc_ = stage_event(ctx, (s), (end), st)) return rc_;         \
   } while (0)
 
+// destinations of the fused projection epilogues
+ProjEpi proj_epi(const dlm_ctx* ctx, int C) {
+  ProjEpi pe;
+  pe.H = ctx->md.H;
+  pe.Hkv = ctx->md.Hkv;
+  pe.Dh = ctx->md.Dh;
+  pe.Lcap = ctx->Lcap;
+  pe.C = C;
+  pe.lens = ctx->lens_d;
+  pe.rope = ctx->d.rope_theta > 0.0f ? ctx->rope : nullptr;
+  pe.q = ctx->q;
+  pe.kcache = ctx->kc;
+  pe.vcache = ctx->vc;
+  pe.x = ctx->x;
+  pe.y = ctx->y;
+  return pe;
+}
+
 // the kernel sequence of one denoising step
 int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
                  dlm_canvas_stats* stats, const AttnPlan& ap, cudaStream_t st) {
@@ -407,11 +431,19 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.out = ctx->part;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
+    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+    if (fused) {
+      pl.epi = EPI_QKV;
+      io.done = c->done;
+      io.proj = proj_epi(ctx, C);
+    }
     if (int rc = run_gemm(ctx, ctx->x, ctx->w_qkv, ctx->Nqkv, pl, io, st)) return rc;
-    e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
-                     ctx->kc, ctx->vc, c->done, ctx->n_active, st);
-    if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue", e);
-    ++ctx->launches;
+    if (!fused) {
+      e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
+                       ctx->kc, ctx->vc, c->done, ctx->n_active, st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue", e);
+      ++ctx->launches;
+    }
   }
   STAGE(DLM_STAGE_QKV, true);
   // a3: attention over [prefix ; canvas]
@@ -436,11 +468,19 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.out = ctx->part;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
+    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+    if (fused) {
+      pl.epi = EPI_RESID;
+      io.done = c->done;
+      io.proj = proj_epi(ctx, C);
+    }
     if (int rc = run_gemm(ctx, ctx->o, ctx->w_o, md.d, pl, io, st)) return rc;
-    e = wo_epilogue(md, ctx->part, pl.splits, rows, C, ctx->x, ctx->y, c->done, ctx->n_active,
-                    st);
-    if (e != cudaSuccess) return cuda_fail(ctx, "wo epilogue", e);
-    ++ctx->launches;
+    if (!fused) {
+      e = wo_epilogue(md, ctx->part, pl.splits, rows, C, ctx->x, ctx->y, c->done, ctx->n_active,
+                      st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "wo epilogue", e);
+      ++ctx->launches;
+    }
   }
   STAGE(DLM_STAGE_WO, true);
   // a5: LM head with the fused vocabulary reduction

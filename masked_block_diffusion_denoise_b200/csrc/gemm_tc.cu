@@ -16,6 +16,9 @@
 //            full logits for inspection).  Work units (m tile, n tile,
 //            k split), m fastest, strided over the grid, so that CTAs that
 //            run at the same time share the same B (weight) slab through L2.
+//   EPI_QKV  (BN 256, K not split) the QKV projection: RoPE on q and k,
+//            bf16 stores of q and of the canvas K / V into their cache slots.
+//   EPI_RESID (BN 256, K not split) the output projection plus residual.
 //   EPI_LM   the LM head's fused vocabulary reduction.  CTA c keeps m tile
 //            c % m_tiles and walks vocabulary tiles c / m_tiles + k * slots;
 //            each epilogue thread folds every tile of its row into one row
@@ -49,6 +52,7 @@ struct TcParams {
   float* out;
   LmPart* part;
   LmEpi epi;
+  ProjEpi proj;
   const uint8_t* done;   // [B] canvases that are finished (LM rows skipped)
   const int* n_active;   // whole launch skipped when *n_active == 0
   int* err;
@@ -262,13 +266,95 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
           }
-        } else {
+        } else if constexpr (EPI == EPI_LM) {
 #pragma unroll 1
           for (int c = 0; c < BN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
             if (lm_live)
               rs_update<32>(rs, v, n * BN + c, lm_inv_t, p.epi, lm_canvas, lm_pos, lm_step);
+          }
+        } else if constexpr (EPI == EPI_QKV) {
+          // one 128-column head at a time: rotate pairs (j, j+64) of q and k,
+          // store q rows and the canvas K / V into the cache slots
+          const ProjEpi& pe = p.proj;
+          const int seq = row / pe.C, p_in = row - seq * pe.C;
+          const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
+#pragma unroll 1
+          for (int hc = 0; hc < BN / 128; ++hc) {
+            float v[128];
+            {
+              uint32_t raw[4][32];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) tmem_ld32_nowait(taddr + hc * 128 + c * 32, raw[c]);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(raw[c][j]);
+            }
+            const int head = (n * BN) / 128 + hc;
+            if (live && head < pe.H + 2 * pe.Hkv) {
+              const int pos = pe.lens[seq] + p_in;
+              if (pe.rope != nullptr && head < pe.H + pe.Hkv) {
+                const float2* cs = pe.rope + (size_t)pos * 64;
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                  const float2 r = cs[j];
+                  const float a = v[j], b = v[j + 64];
+                  v[j] = a * r.x - b * r.y;
+                  v[j + 64] = b * r.x + a * r.y;
+                }
+              }
+              __nv_bfloat16* dst;
+              if (head < pe.H) {
+                dst = (__nv_bfloat16*)pe.q + ((size_t)row * pe.H + head) * 128;
+              } else if (head < pe.H + pe.Hkv) {
+                dst = (__nv_bfloat16*)pe.kcache +
+                      (((size_t)seq * pe.Hkv + (head - pe.H)) * pe.Lcap + pos) * 128;
+              } else {
+                dst = (__nv_bfloat16*)pe.vcache +
+                      (((size_t)seq * pe.Hkv + (head - pe.H - pe.Hkv)) * pe.Lcap + pos) * 128;
+              }
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                uint4 w;
+                w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
+                w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+                w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+                w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
+                reinterpret_cast<uint4*>(dst)[c] = w;
+              }
+            }
+          }
+        } else {
+          // EPI_RESID: y = x + acc
+          const ProjEpi& pe = p.proj;
+          const int seq = row / pe.C;
+          const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            tmem_ld32(taddr + c, v);
+            const int col0 = n * BN + c;
+            if (live && col0 < p.N) {
+              const uint4* xs =
+                  reinterpret_cast<const uint4*>((const __nv_bfloat16*)pe.x + (size_t)row * p.N + col0);
+              uint4* ys = reinterpret_cast<uint4*>((__nv_bfloat16*)pe.y + (size_t)row * p.N + col0);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const uint4 xv = xs[q4];
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                uint32_t yw[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&xw[u]);
+                  const float2 xf = __bfloat1622float2(x2);
+                  yw[u] = pack_bf16(xf.x + v[8 * q4 + 2 * u], xf.y + v[8 * q4 + 2 * u + 1]);
+                }
+                ys[q4] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+              }
+            }
           }
         }
       }
@@ -337,6 +423,7 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.part = io.part;
   p.epi = io.epi;
   p.epi.n_tiles = p.n_tiles;
+  p.proj = io.proj;
   p.done = io.done;
   p.n_active = io.n_active;
   p.err = io.err;
@@ -344,8 +431,12 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
     return plan.epi == EPI_LM ? launch_tc<128, EPI_LM>(tmA, tmB, p, num_sms, st)
                               : launch_tc<128, EPI_F32>(tmA, tmB, p, num_sms, st);
   }
-  return plan.epi == EPI_LM ? launch_tc<256, EPI_LM>(tmA, tmB, p, num_sms, st)
-                            : launch_tc<256, EPI_F32>(tmA, tmB, p, num_sms, st);
+  switch (plan.epi) {
+    case EPI_LM: return launch_tc<256, EPI_LM>(tmA, tmB, p, num_sms, st);
+    case EPI_QKV: return launch_tc<256, EPI_QKV>(tmA, tmB, p, num_sms, st);
+    case EPI_RESID: return launch_tc<256, EPI_RESID>(tmA, tmB, p, num_sms, st);
+    default: return launch_tc<256, EPI_F32>(tmA, tmB, p, num_sms, st);
+  }
 }
 
 int gemm_tc_smem_bytes(int BN) { return BN == 128 ? TcCfg<128>::kSmem : TcCfg<256>::kSmem; }

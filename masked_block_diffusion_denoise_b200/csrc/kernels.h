@@ -9,7 +9,10 @@
 
 namespace dlm {
 
-enum { EPI_F32 = 0, EPI_LM = 1 };
+// GEMM epilogues: f32 (split-K) partials; the LM head's vocabulary
+// reduction; the QKV projection with RoPE and q / KV-cache stores; the output
+// projection with the residual add.  The last two run when K is not split.
+enum { EPI_F32 = 0, EPI_LM = 1, EPI_QKV = 2, EPI_RESID = 3 };
 
 struct GemmPlan {
   int M, N, K;
@@ -18,10 +21,25 @@ struct GemmPlan {
   int epi;      // EPI_F32 / EPI_LM
 };
 
+struct ModelDims;
+
+// destinations of the fused projection epilogues (bf16 model)
+struct ProjEpi {
+  int H = 0, Hkv = 0, Dh = 0, Lcap = 0, C = 1;
+  const int32_t* lens = nullptr;     // [B] prefix lengths (canvas slots follow)
+  const float2* rope = nullptr;      // [Lcap][Dh/2] cos/sin, or null
+  void* q = nullptr;                 // EPI_QKV: [M][H][Dh]
+  void* kcache = nullptr;            // EPI_QKV: [B][Hkv][Lcap][Dh]
+  void* vcache = nullptr;
+  const void* x = nullptr;           // EPI_RESID: residual [M][N]
+  void* y = nullptr;                 // EPI_RESID: [M][N]
+};
+
 struct GemmIO {
   float* out = nullptr;        // EPI_F32: [splits][M][N]
   LmPart* part = nullptr;      // EPI_LM:  [M][n_tiles]
   LmEpi epi{};
+  ProjEpi proj{};
   const uint8_t* done = nullptr;
   const int* n_active = nullptr;
   int* err = nullptr;
