@@ -8,9 +8,9 @@
 //   warp 1      MMA issuer: one thread issues tcgen05.mma 128xBNx16 into one
 //               of two TMEM accumulators and frees ring slots with
 //               tcgen05.commit;
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (one TMEM lane = one
-//               output row per thread) while the MMA warp fills the other
-//               accumulator.
+//   warps 2..9  epilogue: tcgen05.ld the accumulator (one TMEM lane = one
+//               output row per thread; two warpgroups, one column half each)
+//               while the MMA warp fills the other accumulator.
 // Epilogues:
 //   EPI_F32  store f32 partial sums [split][M][N] (projections, split-K;
 //            full logits for inspection).  Work units (m tile, n tile,
@@ -43,7 +43,8 @@ struct TcCfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kSmem =
+      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + 128 * 32 /*row states*/;
 };
 
 struct TcParams {
@@ -92,8 +93,10 @@ __device__ __forceinline__ bool get_unit(const TcParams& p, int k, int& m, int& 
   }
 }
 
+constexpr int kGemmThreads = 320;   // producer, MMA, 8 epilogue warps
+
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -220,8 +223,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait_bounded(mma_done, 0, nullptr);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
+    // two warpgroups; warp w reads TMEM lanes 32*(w%4).. and warpgroup
+    // (w-2)/4 takes one half of the columns of every accumulator tile
     const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
+    const int wg = (warp - 2) >> 2;
+    constexpr int kHalfN = BN / 2;
+    const int cb = wg * kHalfN;           // first column of this warpgroup
     int acc = 0;
     uint32_t acc_phase = 0;
     int m = 0, n, kb0, kb1, split;
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
         if constexpr (EPI == EPI_F32) {
           float* orow = p.out + ((size_t)split * p.M + row) * p.N;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = cb; c < cb + kHalfN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
             const int col0 = n * BN + c;
@@ -268,7 +276,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         } else if constexpr (EPI == EPI_LM) {
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = cb; c < cb + kHalfN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
             if (lm_live)
@@ -281,32 +289,12 @@ __global__ void __launch_bounds__(192, 1)
           const int seq = row / pe.C, p_in = row - seq * pe.C;
           const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
 #pragma unroll 1
-          for (int hc = 0; hc < BN / 128; ++hc) {
-            float v[128];
-            {
-              uint32_t raw[4][32];
-#pragma unroll
-              for (int c = 0; c < 4; ++c) tmem_ld32_nowait(taddr + hc * 128 + c * 32, raw[c]);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(raw[c][j]);
-            }
+          for (int hc = cb / 128; hc < (cb + kHalfN) / 128; ++hc) {
             const int head = (n * BN) / 128 + hc;
-            if (live && head < pe.H + 2 * pe.Hkv) {
-              const int pos = pe.lens[seq] + p_in;
-              if (pe.rope != nullptr && head < pe.H + pe.Hkv) {
-                const float2* cs = pe.rope + (size_t)pos * 64;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                  const float2 r = cs[j];
-                  const float a = v[j], b = v[j + 64];
-                  v[j] = a * r.x - b * r.y;
-                  v[j + 64] = b * r.x + a * r.y;
-                }
-              }
-              __nv_bfloat16* dst;
+            const bool store = live && head < pe.H + 2 * pe.Hkv;
+            const int pos = store ? pe.lens[seq] + p_in : 0;
+            __nv_bfloat16* dst = nullptr;
+            if (store) {
               if (head < pe.H) {
                 dst = (__nv_bfloat16*)pe.q + ((size_t)row * pe.H + head) * 128;
               } else if (head < pe.H + pe.Hkv) {
@@ -316,14 +304,46 @@ __global__ void __launch_bounds__(192, 1)
                 dst = (__nv_bfloat16*)pe.vcache +
                       (((size_t)seq * pe.Hkv + (head - pe.H - pe.Hkv)) * pe.Lcap + pos) * 128;
               }
+            }
+            const bool rotate = pe.rope != nullptr && head < pe.H + pe.Hkv;
+            // rotary pairs (j, j + 64) in two chunks of 32 pairs
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t lo_raw[32], hi_raw[32];
+              tmem_ld32_nowait(taddr + hc * 128 + c * 32, lo_raw);
+              tmem_ld32_nowait(taddr + hc * 128 + 64 + c * 32, hi_raw);
+              tmem_wait_ld();
+              if (store) {
+                float lo[32], hi[32];
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                uint4 w;
-                w.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
-                w.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
-                w.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
-                w.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
-                reinterpret_cast<uint4*>(dst)[c] = w;
+                for (int j = 0; j < 32; ++j) {
+                  lo[j] = __uint_as_float(lo_raw[j]);
+                  hi[j] = __uint_as_float(hi_raw[j]);
+                }
+                if (rotate) {
+                  const float2* cs = pe.rope + (size_t)pos * 64 + c * 32;
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) {
+                    const float2 r = cs[j];
+                    const float a = lo[j], b2 = hi[j];
+                    lo[j] = a * r.x - b2 * r.y;
+                    hi[j] = b2 * r.x + a * r.y;
+                  }
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  uint4 w, u;
+                  w.x = pack_bf16(lo[8 * q4 + 0], lo[8 * q4 + 1]);
+                  w.y = pack_bf16(lo[8 * q4 + 2], lo[8 * q4 + 3]);
+                  w.z = pack_bf16(lo[8 * q4 + 4], lo[8 * q4 + 5]);
+                  w.w = pack_bf16(lo[8 * q4 + 6], lo[8 * q4 + 7]);
+                  u.x = pack_bf16(hi[8 * q4 + 0], hi[8 * q4 + 1]);
+                  u.y = pack_bf16(hi[8 * q4 + 2], hi[8 * q4 + 3]);
+                  u.z = pack_bf16(hi[8 * q4 + 4], hi[8 * q4 + 5]);
+                  u.w = pack_bf16(hi[8 * q4 + 6], hi[8 * q4 + 7]);
+                  reinterpret_cast<uint4*>(dst + c * 32)[q4] = w;
+                  reinterpret_cast<uint4*>(dst + 64 + c * 32)[q4] = u;
+                }
               }
             }
           }
@@ -333,7 +353,7 @@ __global__ void __launch_bounds__(192, 1)
           const int seq = row / pe.C;
           const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = cb; c < cb + kHalfN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
             const int col0 = n * BN + c;
@@ -365,8 +385,17 @@ __global__ void __launch_bounds__(192, 1)
       if (acc == 0) acc_phase ^= 1u;
     }
     if constexpr (EPI == EPI_LM) {
-      const int slots = gridDim.x / p.m_tiles;
-      if (lm_live) rs_store(p.part + (size_t)lm_row * slots + blockIdx.x / p.m_tiles, rs);
+      // the two warpgroups' states of a row: warpgroup 1 hands its state over
+      // through shared memory, warpgroup 0 combines (fixed order) and stores
+      RowState* xch = reinterpret_cast<RowState*>(reinterpret_cast<uint8_t*>(full) + 256);
+      const int lr = quad * 32 + lane;
+      if (wg == 1) xch[lr] = rs;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (wg == 0) {
+        const RowState both = rs_combine(rs, xch[lr]);
+        const int slots = gridDim.x / p.m_tiles;
+        if (lm_live) rs_store(p.part + (size_t)lm_row * slots + blockIdx.x / p.m_tiles, both);
+      }
     }
   }
 
@@ -403,7 +432,8 @@ cudaError_t launch_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const TcPa
     attr_set = true;
   }
   const int grid = tc_grid(p.units, p.m_tiles, p.n_tiles, EPI, num_sms);
-  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(192), Cfg::kSmem, st, tmA, tmB, p);
+  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kGemmThreads), Cfg::kSmem, st, tmA,
+                    tmB, p);
 }
 
 }  // namespace
