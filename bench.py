@@ -296,7 +296,7 @@ def run_ours(a):
     if not a.no_e2e:
         host = {k: getattr(tmpl, k).cpu().pin_memory() for k in
                 ("tokens", "committed", "step", "done", "eos_pos")}
-        hstats = torch.zeros((wl.batch, 4), dtype=torch.int32).pin_memory()
+        hstats = torch.zeros((wl.batch, 6), dtype=torch.int32).pin_memory()
         work = {k: v.clone().pin_memory() for k, v in host.items()}
         n_blocks = max(1, K // S)
         h2d = sum(v.numel() * v.element_size() for v in host.values()) + hstats.numel() * 4

@@ -93,7 +93,8 @@ typedef struct { const void *emb, *w_q, *w_k, *w_v, *w_o, *w_lm; } dlm_weights;
  *   corruption  DLM_MASK: uncommitted slots hold mask_id (which is excluded
  *               from the argmax, softmax and entropy); DLM_UNIFORM: they are
  *               re-noised with uniform random ids after every step
- *   editing     must be 0 (re-editing committed tokens is not supported)
+ *   editing     0: committed tokens are final; 1: token editing (see
+ *               editing_threshold below)
  *   entropy_bound  >= 0 selects the entropy-bound rule (temperature annealed
  *               linearly from t_max at step 0 to t_min at step S-1, Gumbel
  *               sampling); < 0 selects threshold + quota
@@ -109,11 +110,30 @@ typedef struct {
   float entropy_bound;
   float temperature, t_max, t_min;
   unsigned long long seed;
+  /* adaptive stopping (DiffusionGemma page, "adaptive stopping" and the
+   * stability_threshold / confidence_threshold arguments): a canvas is
+   * frozen -- every uncommitted position commits its current candidate and
+   * the canvas is done -- once its argmax over all positions has been the
+   * same for `stability_steps` consecutive steps and the mean entropy of its
+   * positions is below `stop_entropy` (nats).  stop_entropy <= 0 turns it
+   * off (then prev_cand / stable in dlm_canvas may be NULL). */
+  int stability_steps;
+  float stop_entropy;
+  /* token editing (DiffusionGemma page, editing_threshold: committed tokens
+   * may be re-edited; course "Diffusion LLMs", section 14: LLaDA2.1
+   * token-to-token editing).  With editing = 1, at the start of every step a
+   * position committed earlier and lying before the first committed EOS
+   * takes the step's candidate when the candidate differs from its token
+   * and its confidence is >= editing_threshold; it stays committed.  A
+   * canvas is done once every position is committed, as without editing. */
+  float editing_threshold;
 } dlm_sampler_params;
 
 /* Canvas state of `batch` sequences, device, caller-owned, updated in place:
  *   tokens [B][C] int32, committed [B][C] uint8 (0/1), step [B] int32 (steps
- *   taken), done [B] uint8, eos_pos [B] int32 (first committed EOS or -1).
+ *   taken), done [B] uint8, eos_pos [B] int32 (first committed EOS or -1),
+ *   and for adaptive stopping prev_cand / stable (may be NULL when it is
+ *   off; dlm_canvas_init sets prev_cand to -1 and stable to 0).
  * Canvas b attends to KV sequence b. */
 typedef struct {
   int32_t *tokens;
@@ -121,18 +141,24 @@ typedef struct {
   int32_t *step;
   uint8_t *done;
   int32_t *eos_pos;
+  int32_t *prev_cand;   /* [B][C] last step's candidates (adaptive stopping)     */
+  int32_t *stable;      /* [B] consecutive steps with unchanged candidates       */
 } dlm_canvas;
 
 /* Per-canvas counters, device, caller-owned and caller-zeroed; every step
  * adds to them.  committed_by_sampler counts positions the selection chose
  * (forced ones included); forced_at_budget those committed only because the
  * budget ran out; eos_autofill the uncommitted positions filled with EOS
- * after the first committed EOS. */
+ * after the first committed EOS; frozen those committed when adaptive
+ * stopping froze the canvas (not counted in committed_by_sampler); edited
+ * the committed tokens replaced by token editing. */
 typedef struct {
   int32_t steps_used;
   int32_t committed_by_sampler;
   int32_t forced_at_budget;
   int32_t eos_autofill;
+  int32_t frozen;       /* positions committed by adaptive stopping */
+  int32_t edited;       /* committed tokens replaced by token editing */
 } dlm_canvas_stats;
 
 /* Create a context: validates the descriptor, allocates the KV cache
@@ -188,6 +214,27 @@ int dlm_decode_block_host(dlm_ctx *ctx, int32_t *tokens, uint8_t *committed, int
                           uint8_t *done, int32_t *eos_pos, int batch,
                           const dlm_sampler_params *params, dlm_canvas_stats *stats,
                           void *stream);
+
+/* Multi-block generation (Nemotron guide, section 6: blocks follow one
+ * another until gen_length or EOS; DiffusionGemma page: the outer loop over
+ * canvases, each finished canvas joins the cache, eos_early_stop; course
+ * "Diffusion LLMs", section 14: the finished block is cached through a clean
+ * pass).  For block k = 0, 1, ..., n_blocks-1: initialise the canvases with
+ * seed + k, decode the block (the steps of dlm_decode_block, launched
+ * directly on `stream` rather than through a graph), copy its tokens to
+ * out_tokens[b][k*C .. k*C+C-1], then append it to every sequence's KV cache:
+ * K/V recomputed from the block's final tokens at absolute positions
+ * len_b .. len_b+C-1 (the lengths grow by C).  With eos_early_stop != 0 the
+ * loop ends after a block in which every sequence has a committed EOS.
+ * out_tokens: device int32 [batch][n_blocks*C]; blocks not generated are
+ * left as they were.  *blocks_done (host, may be NULL) receives the number
+ * of blocks run.  With eos_early_stop the call synchronises `stream` after
+ * every block to read the EOS positions; without it, it returns with the
+ * work queued.  Canvas stats accumulate over the blocks.
+ * DLM_ECAP before any work if a prefix plus n_blocks*C exceeds max_prefix. */
+int dlm_generate(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+                 const dlm_sampler_params *params, int n_blocks, int eos_early_stop,
+                 int32_t *out_tokens, dlm_canvas_stats *stats, int *blocks_done, void *stream);
 
 /* Kernel (c) alone: the sampler update of dlm_denoise_step applied to given
  * per-position candidates (device int32 [B][C]), confidences and entropies

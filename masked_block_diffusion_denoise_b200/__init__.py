@@ -20,7 +20,7 @@ __all__ = [
     "dlm_model_desc", "dlm_weights", "dlm_sampler_params", "dlm_canvas", "dlm_canvas_stats",
     "DlmError", "lib", "library_path", "dlm_create", "dlm_destroy", "dlm_kv_append",
     "dlm_reset_kv", "dlm_kv_length", "dlm_canvas_init", "dlm_denoise_step",
-    "dlm_decode_block", "dlm_decode_block_host", "dlm_commit", "dlm_debug_buffer",
+    "dlm_decode_block", "dlm_decode_block_host", "dlm_commit", "dlm_generate", "dlm_debug_buffer",
     "dlm_debug_logits", "dlm_check", "dlm_launches_per_step", "dlm_last_error",
     "EXPORTED_SYMBOLS", "dlm_set_stage_events", "DLM_STAGE_EMBED", "DLM_STAGE_QKV",
     "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT", "DLM_NUM_STAGES", "dlm_attention_noalloc",
@@ -62,16 +62,19 @@ class dlm_sampler_params(ctypes.Structure):
                 ("corruption", ctypes.c_int), ("editing", ctypes.c_int),
                 ("entropy_bound", ctypes.c_float), ("temperature", ctypes.c_float),
                 ("t_max", ctypes.c_float), ("t_min", ctypes.c_float),
-                ("seed", ctypes.c_ulonglong)]
+                ("seed", ctypes.c_ulonglong), ("stability_steps", ctypes.c_int),
+                ("stop_entropy", ctypes.c_float), ("editing_threshold", ctypes.c_float)]
 
 
 class dlm_canvas(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("tokens", "committed", "step", "done", "eos_pos")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("tokens", "committed", "step", "done", "eos_pos",
+                                                  "prev_cand", "stable")]
 
 
 class dlm_canvas_stats(ctypes.Structure):
     _fields_ = [("steps_used", ctypes.c_int32), ("committed_by_sampler", ctypes.c_int32),
-                ("forced_at_budget", ctypes.c_int32), ("eos_autofill", ctypes.c_int32)]
+                ("forced_at_budget", ctypes.c_int32), ("eos_autofill", ctypes.c_int32),
+                ("frozen", ctypes.c_int32), ("edited", ctypes.c_int32)]
 
 
 class DlmError(RuntimeError):
@@ -99,6 +102,8 @@ _SIGS = {
                                    ctypes.POINTER(dlm_sampler_params), _P, _P]),
     "dlm_commit": (_I, [_P, ctypes.POINTER(dlm_canvas), _I, ctypes.POINTER(dlm_sampler_params),
                         _P, _P, _P, _P, _P]),
+    "dlm_generate": (_I, [_P, ctypes.POINTER(dlm_canvas), _I, ctypes.POINTER(dlm_sampler_params),
+                          _I, _I, _P, _P, ctypes.POINTER(_I), _P]),
     "dlm_debug_buffer": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]),
     "dlm_debug_logits": (_I, [_P, _I, _I, _P, _P]),
     "dlm_set_stage_events": (_I, [_P, _I, ctypes.POINTER(_P), _I]),
@@ -214,6 +219,17 @@ def dlm_commit(ctx, canvas: dlm_canvas, batch: int, params: dlm_sampler_params, 
     return _check(ctx, lib().dlm_commit(ctx, ctypes.byref(canvas), batch, ctypes.byref(params),
                                         _ptr(cand), _ptr(conf), _ptr(entropy), _ptr(stats),
                                         _stream(stream)))
+
+
+def dlm_generate(ctx, canvas: dlm_canvas, batch: int, params: dlm_sampler_params,
+                 n_blocks: int, out_tokens, eos_early_stop: bool = True, stats=None,
+                 stream=None) -> int:
+    """Decodes up to n_blocks blocks; returns how many were decoded."""
+    n = ctypes.c_int(0)
+    _check(ctx, lib().dlm_generate(ctx, ctypes.byref(canvas), batch, ctypes.byref(params),
+                                   n_blocks, 1 if eos_early_stop else 0, _ptr(out_tokens),
+                                   _ptr(stats), ctypes.byref(n), _stream(stream)))
+    return n.value
 
 
 def dlm_debug_buffer(ctx, which: int):

@@ -72,7 +72,8 @@ struct dlm_ctx {
   int* n_active = nullptr;
   int* err = nullptr;
   // device copies of a canvas for the host-buffer entry point
-  int32_t *h_tok = nullptr, *h_step = nullptr, *h_eos = nullptr;
+  int32_t *h_tok = nullptr, *h_step = nullptr, *h_eos = nullptr, *h_prev = nullptr,
+          *h_stable = nullptr;
   uint8_t *h_com = nullptr, *h_done = nullptr;
   dlm_canvas_stats* h_stats = nullptr;
   std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> maps;
@@ -302,18 +303,24 @@ int check_params(dlm_ctx* ctx, const dlm_sampler_params* p, int batch) {
   if (!(p->threshold >= 0.0f)) return fail(ctx, DLM_EINVAL, "threshold must be >= 0");
   if (p->corruption != DLM_MASK && p->corruption != DLM_UNIFORM)
     return fail(ctx, DLM_EINVAL, "corruption must be DLM_MASK or DLM_UNIFORM");
-  if (p->editing != 0) return fail(ctx, DLM_EINVAL, "editing mode is not supported");
+  if (p->editing != 0 && p->editing != 1) return fail(ctx, DLM_EINVAL, "editing must be 0 or 1");
+  if (p->editing && !(p->editing_threshold == p->editing_threshold))
+    return fail(ctx, DLM_EINVAL, "editing_threshold must be a number");
   if (p->corruption == DLM_MASK && (ctx->d.mask_id < 0 || ctx->d.mask_id >= ctx->d.vocab))
     return fail(ctx, DLM_EINVAL, "mask corruption needs mask_id in [0, vocab)");
   if (!(p->temperature >= 0.0f)) return fail(ctx, DLM_EINVAL, "temperature must be >= 0");
   if (p->entropy_bound >= 0.0f && !(p->t_min > 0.0f && p->t_max >= p->t_min))
     return fail(ctx, DLM_EINVAL, "entropy bound needs 0 < t_min <= t_max");
+  if (p->stop_entropy > 0.0f && p->stability_steps < 0)
+    return fail(ctx, DLM_EINVAL, "adaptive stopping needs stability_steps >= 0");
   return DLM_OK;
 }
 
-int check_canvas(dlm_ctx* ctx, const dlm_canvas* c) {
+int check_canvas(dlm_ctx* ctx, const dlm_canvas* c, const dlm_sampler_params* p) {
   if (c == nullptr || !c->tokens || !c->committed || !c->step || !c->done || !c->eos_pos)
     return fail(ctx, DLM_EINVAL, "canvas buffers must all be non-NULL");
+  if (p != nullptr && p->stop_entropy > 0.0f && (!c->prev_cand || !c->stable))
+    return fail(ctx, DLM_EINVAL, "adaptive stopping needs canvas prev_cand and stable");
   return DLM_OK;
 }
 
@@ -354,6 +361,10 @@ SelectArgs make_select(const dlm_ctx* ctx, const dlm_sampler_params* p, int batc
   a.eos_id = ctx->d.eos_id;
   a.seed_lo = (uint32_t)(p->seed & 0xFFFFFFFFull);
   a.seed_hi = (uint32_t)(p->seed >> 32);
+  a.stability_steps = p->stability_steps;
+  a.stop_entropy = p->stop_entropy;
+  a.editing = p->editing;
+  a.edit_thr = p->editing_threshold;
   return a;
 }
 
@@ -500,12 +511,41 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
   const int n_part = ctx->bf16 ? gemm_tc_lm_partials(pl, ctx->num_sms) : cdiv(md.V, pl.BN);
   STAGE(DLM_STAGE_COMMIT, false);
   e = commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
-                  c->eos_pos, ctx->lmpart, n_part, ctx->cand, ctx->conf, ctx->ent, stats,
-                  ctx->n_active, ctx->err, st);
+                  c->eos_pos, c->prev_cand, c->stable, ctx->lmpart, n_part, ctx->cand, ctx->conf,
+                  ctx->ent, stats, ctx->n_active, ctx->err, st);
   if (e != cudaSuccess) return cuda_fail(ctx, "commit", e);
   ++ctx->launches;
   STAGE(DLM_STAGE_COMMIT, true);
   ++ctx->ev_step;
+  return DLM_OK;
+}
+
+// The clean pass over finished tokens of every sequence of the batch: K/V
+// at positions len_b .. len_b+C-1 from the tokens themselves, then len_b += C.
+int enqueue_clean_pass(dlm_ctx* ctx, const int32_t* tokens, int batch, int C, cudaStream_t st) {
+  const ModelDims& md = ctx->md;
+  const int rows = batch * C;
+  cudaError_t e = embed_rows(md, tokens, ctx->emb, ctx->x, rows, C, batch, nullptr, nullptr,
+                             ctx->err, st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "embed (clean pass)", e);
+  GemmPlan pl = plan_gemm(ctx, rows, ctx->Nqkv, md.d, EPI_F32);
+  GemmIO io;
+  io.out = ctx->part;
+  io.err = ctx->err;
+  const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+  if (fused) {
+    pl.epi = EPI_QKV;
+    io.proj = proj_epi(ctx, C);
+  }
+  if (int rc = run_gemm(ctx, ctx->x, ctx->w_qkv, ctx->Nqkv, pl, io, st)) return rc;
+  if (!fused) {
+    e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
+                     ctx->kc, ctx->vc, nullptr, nullptr, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue (clean pass)", e);
+  }
+  e = add_len_all(ctx->lens_d, batch, C, st);
+  if (e != cudaSuccess) return cuda_fail(ctx, "add_len_all", e);
+  for (int b = 0; b < batch; ++b) ctx->lens_h[b] += C;
   return DLM_OK;
 }
 
@@ -613,6 +653,8 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if ((rc = dalloc(ctx, &ctx->h_done, d.max_batch))) return bail(rc);
   if ((rc = dalloc(ctx, &ctx->h_eos, d.max_batch * sizeof(int32_t)))) return bail(rc);
   if ((rc = dalloc(ctx, &ctx->h_stats, d.max_batch * sizeof(dlm_canvas_stats)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_prev, ctx->Mmax * sizeof(int32_t)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->h_stable, d.max_batch * sizeof(int32_t)))) return bail(rc);
   ctx->part_floats = part_floats_needed(ctx);
   if ((rc = dalloc(ctx, &ctx->part, ctx->part_floats * sizeof(float)))) return bail(rc);
 
@@ -716,9 +758,9 @@ int dlm_canvas_init(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_samp
   if (ctx == nullptr) return DLM_EINVAL;
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
-  if (int rc = check_canvas(ctx, c)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
   CK(canvas_init(ctx->md, batch, p->canvas, p->corruption, p->seed, c->tokens, c->committed,
-                 c->step, c->done, c->eos_pos, (cudaStream_t)stream));
+                 c->step, c->done, c->eos_pos, c->prev_cand, c->stable, (cudaStream_t)stream));
   return DLM_OK;
 }
 
@@ -727,7 +769,7 @@ int dlm_denoise_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   if (ctx == nullptr) return DLM_EINVAL;
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
-  if (int rc = check_canvas(ctx, c)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
   AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
@@ -740,7 +782,7 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   if (ctx == nullptr) return DLM_EINVAL;
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
-  if (int rc = check_canvas(ctx, c)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
   AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
@@ -813,8 +855,11 @@ int dlm_decode_block_host(dlm_ctx* ctx, int32_t* tokens, uint8_t* committed, int
   if (stats)
     CK(cudaMemcpyAsync(ctx->h_stats, stats, batch * sizeof(dlm_canvas_stats),
                        cudaMemcpyHostToDevice, st));
-  dlm_canvas c{ctx->h_tok, ctx->h_com, ctx->h_step, ctx->h_done, ctx->h_eos};
-  const std::string keep = ctx->msg;
+  // adaptive-stopping state starts fresh for every call
+  CK(cudaMemsetAsync(ctx->h_prev, 0xFF, n * sizeof(int32_t), st));
+  CK(cudaMemsetAsync(ctx->h_stable, 0, batch * sizeof(int32_t), st));
+  dlm_canvas c{ctx->h_tok, ctx->h_com, ctx->h_step, ctx->h_done, ctx->h_eos, ctx->h_prev,
+               ctx->h_stable};
   if (int rc = dlm_decode_block(ctx, &c, batch, p, stats ? ctx->h_stats : nullptr, stream))
     return rc;
   CK(cudaMemcpyAsync(tokens, ctx->h_tok, n * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
@@ -829,17 +874,62 @@ int dlm_decode_block_host(dlm_ctx* ctx, int32_t* tokens, uint8_t* committed, int
   return DLM_OK;
 }
 
+int dlm_generate(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                 int n_blocks, int eos_early_stop, int32_t* out_tokens, dlm_canvas_stats* stats,
+                 int* blocks_done, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (blocks_done) *blocks_done = 0;
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
+  if (n_blocks < 1 || out_tokens == nullptr)
+    return fail(ctx, DLM_EINVAL, "generate needs n_blocks >= 1 and out_tokens");
+  const int C = p->canvas;
+  for (int b = 0; b < batch; ++b)
+    if ((long)ctx->lens_h[b] + (long)n_blocks * C > ctx->d.max_prefix)
+      return fail(ctx, DLM_ECAP, "prefix + n_blocks * canvas exceeds max_prefix");
+  cudaStream_t st = (cudaStream_t)stream;
+  std::vector<int32_t> eos(batch);
+  for (int k = 0; k < n_blocks; ++k) {
+    dlm_sampler_params pk = *p;
+    pk.seed = p->seed + (unsigned long long)k;   // block k's random streams
+    CK(canvas_init(ctx->md, batch, C, pk.corruption, pk.seed, c->tokens, c->committed, c->step,
+                   c->done, c->eos_pos, c->prev_cand, c->stable, st));
+    AttnPlan ap = plan_attention(ctx, batch, C, ctx->lens_h.data(), max_len(ctx, batch));
+    if (ctx->bf16)
+      if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
+    ctx->launches = 0;
+    for (int s = 0; s < pk.steps; ++s)
+      if (int rc = enqueue_step(ctx, c, batch, &pk, stats, ap, st)) return rc;
+    CK(cudaMemcpy2DAsync(out_tokens + (size_t)k * C, (size_t)n_blocks * C * sizeof(int32_t),
+                         c->tokens, (size_t)C * sizeof(int32_t), (size_t)C * sizeof(int32_t),
+                         batch, cudaMemcpyDeviceToDevice, st));
+    if (int rc = enqueue_clean_pass(ctx, c->tokens, batch, C, st)) return rc;
+    if (blocks_done) *blocks_done = k + 1;
+    if (eos_early_stop) {
+      CK(cudaMemcpyAsync(eos.data(), c->eos_pos, batch * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                         st));
+      CK(cudaStreamSynchronize(st));
+      bool all = true;
+      for (int b = 0; b < batch; ++b) all = all && eos[b] >= 0;
+      if (all) break;
+    }
+  }
+  return DLM_OK;
+}
+
 int dlm_commit(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
                const int32_t* cand, const float* conf, const float* entropy,
                dlm_canvas_stats* stats, void* stream) {
   if (ctx == nullptr) return DLM_EINVAL;
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
-  if (int rc = check_canvas(ctx, c)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
   if (!cand || !conf || !entropy) return fail(ctx, DLM_EINVAL, "cand/conf/entropy NULL");
   CK(commit_step(make_select(ctx, p, batch), c->tokens, c->committed, c->step, c->done,
-                 c->eos_pos, nullptr, 0, const_cast<int32_t*>(cand), const_cast<float*>(conf),
-                 const_cast<float*>(entropy), stats, nullptr, ctx->err, (cudaStream_t)stream));
+                 c->eos_pos, c->prev_cand, c->stable, nullptr, 0, const_cast<int32_t*>(cand),
+                 const_cast<float*>(conf), const_cast<float*>(entropy), stats, nullptr, ctx->err,
+                 (cudaStream_t)stream));
   return DLM_OK;
 }
 

@@ -94,7 +94,10 @@ cudaError_t add_len(int32_t* lens, int seq, int n, cudaStream_t st);
 
 cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint64_t seed,
                         int32_t* tokens, uint8_t* committed, int32_t* step, uint8_t* done,
-                        int32_t* eos_pos, cudaStream_t st);
+                        int32_t* eos_pos, int32_t* prev_cand, int32_t* stable, cudaStream_t st);
+
+// lens[b] += n for b < B
+cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st);
 
 // ---- attention.cu ------------------------------------------------------------
 struct AttnPlan {
@@ -122,6 +125,10 @@ struct SelectArgs {
   int uniform;           // re-noise with uniform ids
   int mask_id, eos_id;
   uint32_t seed_lo, seed_hi;
+  int stability_steps;   // adaptive stopping (stop_entropy > 0)
+  float stop_entropy;
+  int editing;           // token editing of committed positions
+  float edit_thr;
 };
 
 // Kernel (c).  With `part` != null it first combines the LM partials of each
@@ -129,8 +136,8 @@ struct SelectArgs {
 // buffers), then selects from them; with part == null it selects from the
 // given cand / conf / ent.
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
-                        uint8_t* done, int32_t* eos_pos, const LmPart* part, int n_part,
-                        int32_t* cand, float* conf, float* ent, dlm_canvas_stats* stats,
-                        const int* n_active, int* err, cudaStream_t st);
+                        uint8_t* done, int32_t* eos_pos, int32_t* prev_cand, int32_t* stable,
+                        const LmPart* part, int n_part, int32_t* cand, float* conf, float* ent,
+                        dlm_canvas_stats* stats, const int* n_active, int* err, cudaStream_t st);
 
 }  // namespace dlm

@@ -135,11 +135,18 @@ __global__ void kv_copy_kernel(int Hkv, int Lcap, int Dh, int seq, int n,
 
 __global__ void add_len_kernel(int32_t* lens, int seq, int n) { lens[seq] += n; }
 
+__global__ void add_len_all_kernel(int32_t* lens, int B, int n) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) lens[b] += n;
+}
+
 __global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint32_t s0,
                                    uint32_t s1, int32_t* tokens, uint8_t* committed,
-                                   int32_t* step, uint8_t* done, int32_t* eos_pos) {
+                                   int32_t* step, uint8_t* done, int32_t* eos_pos,
+                                   int32_t* prev_cand, int32_t* stable) {
   const int b = blockIdx.x;
   for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    if (prev_cand != nullptr) prev_cand[(size_t)b * C + i] = -1;
     int32_t t = mask_id;
     if (uniform) {
       const U32x4 w = philox10(U32x4{(uint32_t)b, 0u, (uint32_t)i, kRenoiseWord}, s0, s1);
@@ -152,6 +159,7 @@ __global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint3
     step[b] = 0;
     done[b] = 0;
     eos_pos[b] = -1;
+    if (stable != nullptr) stable[b] = 0;
   }
 }
 
@@ -223,12 +231,17 @@ cudaError_t add_len(int32_t* lens, int seq, int n, cudaStream_t st) {
 
 cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint64_t seed,
                         int32_t* tokens, uint8_t* committed, int32_t* step, uint8_t* done,
-                        int32_t* eos_pos, cudaStream_t st) {
+                        int32_t* eos_pos, int32_t* prev_cand, int32_t* stable, cudaStream_t st) {
   const int threads = C < 1024 ? ((C + 31) / 32) * 32 : 1024;
   canvas_init_kernel<<<B, threads, 0, st>>>(C, md.V, md.mask_id, corruption == DLM_UNIFORM,
                                             (uint32_t)(seed & 0xFFFFFFFFull),
                                             (uint32_t)(seed >> 32), tokens, committed, step,
-                                            done, eos_pos);
+                                            done, eos_pos, prev_cand, stable);
+  return cudaGetLastError();
+}
+
+cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st) {
+  add_len_all_kernel<<<(B + 127) / 128, 128, 0, st>>>(lens, B, n);
   return cudaGetLastError();
 }
 

@@ -93,6 +93,7 @@ __device__ int eos_fill(int32_t* tok, uint8_t* com, int C, int eos_id, int* e_s,
 __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
                               uint8_t* __restrict__ committed, int32_t* __restrict__ step,
                               uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
+                              int32_t* __restrict__ prev_cand, int32_t* __restrict__ stable,
                               const LmPart* __restrict__ part, int n_part,
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
@@ -127,7 +128,79 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   __syncthreads();
 
   int fill0 = 0, fill1 = 0;
-  eos_fill(tok, com, C, a.eos_id, &e_s, &fill0);
+  const int e0 = eos_fill(tok, com, C, a.eos_id, &e_s, &fill0);
+
+  int nedit = 0;
+  if (a.editing) {
+    // token editing: a position committed before this step and before the
+    // first committed EOS takes its candidate when that differs from the
+    // token with confidence >= edit_thr (float32, -0 folded onto +0)
+    const int lim = e0 < 0 ? C : e0;
+    bool ed = false;
+    if (i < lim && com[i]) {
+      int c = cand[base + i];
+      if (c != tok[i] && conf[base + i] + 0.0f >= a.edit_thr) {
+        if (c < 0 || c >= a.V) {
+          raise_error(err, DLM_EBOUNDS);
+          c = 0;
+        }
+        tok[i] = c;
+        ed = true;
+      }
+    }
+    nedit = __syncthreads_count(ed);
+  }
+
+  if (a.stop_entropy > 0.f) {
+    // adaptive stopping: the argmax of every position unchanged since the
+    // previous step counts one stable step; with enough stable steps and a
+    // mean entropy (float32, summed in position order) below the bound the
+    // canvas freezes: every open position commits its candidate
+    __shared__ int freeze_s;
+    const bool same = (i >= C) || (cand[base + i] == prev_cand[base + i]);
+    const int all_same = __syncthreads_and(same);
+    if (i < C) prev_cand[base + i] = cand[base + i];
+    if (i == 0) {
+      float total = 0.f;
+      for (int j = 0; j < C; ++j) total = __fadd_rn(total, ent[base + j] + 0.0f);
+      const float mean = __fdiv_rn(total, (float)C);
+      const int st = all_same ? stable[b] + 1 : 0;
+      stable[b] = st;
+      freeze_s = (st >= a.stability_steps && mean < a.stop_entropy) ? 1 : 0;
+    }
+    __syncthreads();
+    if (freeze_s) {
+      const bool opened = i < C && !com[i];
+      if (opened) {
+        int c = cand[base + i];
+        if (c < 0 || c >= a.V) {
+          raise_error(err, DLM_EBOUNDS);
+          c = 0;
+        }
+        tok[i] = c;
+        com[i] = 1;
+      }
+      const int nfrozen = __syncthreads_count(opened);
+      const int e = eos_fill(tok, com, C, a.eos_id, &e_s, &fill1);
+      if (i < C) {
+        tokens[base + i] = tok[i];
+        committed[base + i] = com[i];
+      }
+      const int all = __syncthreads_and(i >= C || com[i]);
+      if (i == 0) {
+        done[b] = all ? 1 : 0;
+        step[b] = s + 1;
+        eos_pos[b] = e;
+        if (stats != nullptr) {
+          stats[b].steps_used += 1;
+          stats[b].frozen += nfrozen;
+          stats[b].eos_autofill += fill0 + fill1;
+          stats[b].edited += nedit;
+        }
+      }
+      return;
+    }
+  }
 
   const bool open = (i < C) && !com[i];
   unsigned long long key = ~0ull;
@@ -212,6 +285,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
       stats[b].committed_by_sampler += k;
       stats[b].forced_at_budget += k - krule_s;
       stats[b].eos_autofill += fill0 + fill1;
+      stats[b].edited += nedit;
     }
   }
 }
@@ -219,15 +293,15 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
 }  // namespace
 
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
-                        uint8_t* done, int32_t* eos_pos, const LmPart* part, int n_part,
-                        int32_t* cand, float* conf, float* ent, dlm_canvas_stats* stats,
-                        const int* n_active, int* err, cudaStream_t st) {
+                        uint8_t* done, int32_t* eos_pos, int32_t* prev_cand, int32_t* stable,
+                        const LmPart* part, int n_part, int32_t* cand, float* conf, float* ent,
+                        dlm_canvas_stats* stats, const int* n_active, int* err, cudaStream_t st) {
   int P = 32;
   while (P < a.C) P <<= 1;
   if (P > kMaxC) return cudaErrorInvalidValue;
   if (part != nullptr && P < 512) P = 512;   // enough warps for the row reductions
   return launch_pdl(commit_kernel, dim3(a.B), dim3(P), 0, st, a, tokens, committed, step, done,
-                    eos_pos, part, n_part, cand, conf, ent, stats, n_active, err);
+                    eos_pos, prev_cand, stable, part, n_part, cand, conf, ent, stats, n_active, err);
 }
 
 }  // namespace dlm

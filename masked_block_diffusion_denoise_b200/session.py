@@ -14,7 +14,7 @@ import torch
 
 from . import (DLM_BF16, DLM_F32, DLM_MASK, DLM_UNIFORM, dlm_canvas, dlm_canvas_init,
                dlm_canvas_stats, dlm_check, dlm_commit, dlm_create, dlm_debug_buffer,
-               dlm_debug_logits, dlm_decode_block, dlm_decode_block_host, dlm_denoise_step,
+               dlm_debug_logits, dlm_decode_block, dlm_decode_block_host, dlm_denoise_step, dlm_generate,
                dlm_destroy, dlm_kv_append, dlm_model_desc, dlm_sampler_params, dlm_weights)
 
 _TORCH = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -46,12 +46,15 @@ class Canvas:
     step: torch.Tensor
     done: torch.Tensor
     eos_pos: torch.Tensor
-    stats: torch.Tensor   # int32 [B][4]
+    stats: torch.Tensor      # int32 [B][6]
+    prev_cand: torch.Tensor  # int32 [B][C], adaptive stopping
+    stable: torch.Tensor     # int32 [B], adaptive stopping
 
     @property
     def c(self) -> dlm_canvas:
         return dlm_canvas(self.tokens.data_ptr(), self.committed.data_ptr(),
-                          self.step.data_ptr(), self.done.data_ptr(), self.eos_pos.data_ptr())
+                          self.step.data_ptr(), self.done.data_ptr(), self.eos_pos.data_ptr(),
+                          self.prev_cand.data_ptr(), self.stable.data_ptr())
 
     def numpy(self) -> Dict[str, np.ndarray]:
         return {"tokens": self.tokens.cpu().numpy().astype(np.int64),
@@ -59,23 +62,35 @@ class Canvas:
                 "step": self.step.cpu().numpy().astype(np.int64),
                 "done": self.done.cpu().numpy().astype(bool),
                 "eos_pos": self.eos_pos.cpu().numpy().astype(np.int64),
+                "prev_cand": self.prev_cand.cpu().numpy().astype(np.int64),
+                "stable": self.stable.cpu().numpy().astype(np.int64),
                 "stats": self.stats.cpu().numpy()}
 
-    def load(self, tokens, committed, step, done, eos_pos) -> None:
+    def load(self, tokens, committed, step, done, eos_pos, prev_cand=None, stable=None) -> None:
         self.tokens.copy_(torch.as_tensor(np.asarray(tokens, dtype=np.int32)))
         self.committed.copy_(torch.as_tensor(np.asarray(committed, dtype=np.uint8)))
         self.step.copy_(torch.as_tensor(np.asarray(step, dtype=np.int32)))
         self.done.copy_(torch.as_tensor(np.asarray(done, dtype=np.uint8)))
         self.eos_pos.copy_(torch.as_tensor(np.asarray(eos_pos, dtype=np.int32)))
+        if prev_cand is None:
+            self.prev_cand.fill_(-1)
+        else:
+            self.prev_cand.copy_(torch.as_tensor(np.asarray(prev_cand, dtype=np.int32)))
+        if stable is None:
+            self.stable.zero_()
+        else:
+            self.stable.copy_(torch.as_tensor(np.asarray(stable, dtype=np.int32)))
 
 
 def sampler_params(canvas: int, steps: int, threshold: float = 0.9, quota: int = 0,
                    corruption: str = "mask", entropy_bound: float = -1.0,
                    temperature: float = 0.0, t_max: float = 0.8, t_min: float = 0.4,
-                   seed: int = 0) -> dlm_sampler_params:
+                   seed: int = 0, stability_steps: int = 1, stop_entropy: float = -1.0,
+                   editing: int = 0, editing_threshold: float = 0.9) -> dlm_sampler_params:
     return dlm_sampler_params(canvas, steps, threshold, quota,
-                              DLM_UNIFORM if corruption == "uniform" else DLM_MASK, 0,
-                              entropy_bound, temperature, t_max, t_min, seed)
+                              DLM_UNIFORM if corruption == "uniform" else DLM_MASK, editing,
+                              entropy_bound, temperature, t_max, t_min, seed, stability_steps,
+                              stop_entropy, editing_threshold)
 
 
 class Session:
@@ -132,7 +147,9 @@ class Session:
                       torch.zeros(batch, dtype=torch.int32, device=dev),
                       torch.zeros(batch, dtype=torch.uint8, device=dev),
                       torch.full((batch,), -1, dtype=torch.int32, device=dev),
-                      torch.zeros((batch, 4), dtype=torch.int32, device=dev))
+                      torch.zeros((batch, 6), dtype=torch.int32, device=dev),
+                      torch.full((batch, C), -1, dtype=torch.int32, device=dev),
+                      torch.zeros(batch, dtype=torch.int32, device=dev))
 
     def init(self, cv: Canvas, p: dlm_sampler_params, stream=None) -> None:
         dlm_canvas_init(self.ctx, cv.c, cv.tokens.shape[0], p, stream=stream)
@@ -146,6 +163,15 @@ class Session:
     def commit(self, cv: Canvas, p: dlm_sampler_params, cand, conf, ent, stream=None) -> None:
         dlm_commit(self.ctx, cv.c, cv.tokens.shape[0], p, cand, conf, ent, stats=cv.stats,
                    stream=stream)
+
+    def generate(self, cv: Canvas, p: dlm_sampler_params, n_blocks: int,
+                 eos_early_stop: bool = True, stream=None) -> tuple:
+        """(tokens [B][n_blocks*C] int32 on the device, blocks decoded)."""
+        B, C = cv.tokens.shape
+        out = torch.zeros((B, n_blocks * C), dtype=torch.int32, device=self.device)
+        n = dlm_generate(self.ctx, cv.c, B, p, n_blocks, out, eos_early_stop=eos_early_stop,
+                         stats=cv.stats, stream=stream)
+        return out, n
 
     def check(self, stream=None) -> None:
         dlm_check(self.ctx, stream)

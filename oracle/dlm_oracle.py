@@ -421,6 +421,12 @@ class SamplerParams:
     t_max: float = 0.8
     t_min: float = 0.4
     seed: int = 0
+    # adaptive stopping (DiffusionGemma page): off when stop_entropy <= 0
+    stability_steps: int = 1
+    stop_entropy: float = -1.0
+    # token editing (DiffusionGemma page editing_threshold): off when editing == 0
+    editing: int = 0
+    editing_threshold: float = 0.9
     # oracle-only readings, for pins and for the readings table
     quota_rule: str = "union"      # "union": max(n_thr, q); "additive": n_thr + q
     schedule: str = "quota"        # "quota" | "course" (m_s = ceil(N(S-s)/S))
@@ -437,10 +443,19 @@ class CanvasState:
     step: np.ndarray        # int64 [B]
     done: np.ndarray        # bool  [B]
     eos_pos: np.ndarray     # int64 [B]
+    prev_cand: Optional[np.ndarray] = None   # int64 [B][C], -1 before the first step
+    stable: Optional[np.ndarray] = None      # int64 [B]
+
+    def __post_init__(self):
+        if self.prev_cand is None:
+            self.prev_cand = np.full(self.tokens.shape, -1, dtype=np.int64)
+        if self.stable is None:
+            self.stable = np.zeros(self.tokens.shape[0], dtype=np.int64)
 
     def copy(self) -> "CanvasState":
         return CanvasState(self.tokens.copy(), self.committed.copy(), self.step.copy(),
-                           self.done.copy(), self.eos_pos.copy())
+                           self.done.copy(), self.eos_pos.copy(), self.prev_cand.copy(),
+                           self.stable.copy())
 
 
 @dataclass
@@ -449,14 +464,18 @@ class CanvasStats:
     committed_by_sampler: int = 0
     forced_at_budget: int = 0
     eos_autofill: int = 0
+    frozen: int = 0
+    edited: int = 0
 
 
-def init_canvas(batch: int, p: SamplerParams, mask_id: int, vocab: int) -> CanvasState:
+def init_canvas(batch: int, p: SamplerParams, mask_id: int, vocab: int,
+                seed: Optional[int] = None) -> CanvasState:
     """All-mask canvas (Nemotron guide, section 6) or, in uniform mode, uniform
     random ids from the step-0 re-noise stream."""
     C = p.canvas
+    seed = p.seed if seed is None else seed
     if p.corruption == "uniform":
-        tok = np.stack([uniform_token_ids(p.seed, b, 0, np.arange(C), vocab) for b in range(batch)])
+        tok = np.stack([uniform_token_ids(seed, b, 0, np.arange(C), vocab) for b in range(batch)])
     else:
         tok = np.full((batch, C), mask_id, dtype=np.int64)
     return CanvasState(tok.astype(np.int64), np.zeros((batch, C), bool),
@@ -509,9 +528,48 @@ def select_canvas(state: CanvasState, b: int, cand, conf, H, p: SamplerParams, *
     tok, com = state.tokens[b], state.committed[b]
     s = int(state.step[b])
     e, fill0 = _eos_fill(tok, com, eos_id)
+    if p.editing:
+        # token editing (DiffusionGemma page: editing_threshold re-edits
+        # committed tokens; course section 14: LLaDA2.1 replaces an opened
+        # token that a later iteration finds weak).  READING: a position
+        # committed before this step and before the first committed EOS
+        # takes the model's current candidate when it differs from its token
+        # and its float32 confidence is >= editing_threshold; it stays
+        # committed.
+        tau_e = F32(p.editing_threshold)
+        for i in range(e if e >= 0 else C):
+            if com[i] and int(cand[i]) != int(tok[i]) and _canon(conf[i]) >= tau_e:
+                tok[i] = int(cand[i])
+                if stats is not None:
+                    stats.edited += 1
     U = [i for i in range(C) if not com[i]]
     conf32 = [_canon(conf[i]) for i in range(C)]
     H32 = [_canon(H[i]) for i in range(C)]
+    if p.stop_entropy > 0:
+        # adaptive stopping (DiffusionGemma page): READING -- the argmax of all
+        # C positions unchanged since the previous step counts one stable
+        # step; the mean entropy is the float32 sum over the positions in
+        # order, divided by C
+        same = all(int(cand[i]) == int(state.prev_cand[b][i]) for i in range(C))
+        state.stable[b] = state.stable[b] + 1 if same else 0
+        state.prev_cand[b][:] = [int(c) for c in cand[:C]]
+        total = F32(0.0)
+        for i in range(C):
+            total = F32(total + H32[i])
+        mean_h = F32(total / F32(C))
+        if state.stable[b] >= p.stability_steps and mean_h < F32(p.stop_entropy):
+            for i in U:
+                tok[i] = int(cand[i])
+                com[i] = True
+            e2, fill1 = _eos_fill(tok, com, eos_id)
+            state.done[b] = bool(com.all())
+            state.step[b] = s + 1
+            state.eos_pos[b] = e2
+            if stats is not None:
+                stats.steps_used += 1
+                stats.frozen += len(U)
+                stats.eos_autofill += fill0 + fill1
+            return
     if p.entropy_bound >= 0:
         order = sorted(U, key=lambda i: (H32[i], i))
         k, run = 0, F32(0.0)
@@ -611,6 +669,30 @@ def decode_block(model: OracleModel, state: CanvasState, p: SamplerParams,
         denoise_step(model, state, p, stats)
         calls += 1
     return calls
+
+
+def generate(model: OracleModel, p: SamplerParams, batch: int, n_blocks: int,
+             eos_early_stop: bool = True, stats: Optional[List[CanvasStats]] = None):
+    """Blocks one after another (Nemotron guide, section 6: until gen_length
+    or EOS; DiffusionGemma page: outer loop over canvases with eos_early_stop;
+    course section 14: the finished block joins the cache through a clean
+    pass).  READING: block k uses seed + k for its random streams.  Returns
+    (tokens int64 [batch][blocks*C], blocks run)."""
+    d = model.dims
+    C = p.canvas
+    out = []
+    blocks = 0
+    for k in range(n_blocks):
+        pk = SamplerParams(**{**p.__dict__, "seed": p.seed + k})
+        st = init_canvas(batch, pk, d.mask_id, d.vocab)
+        decode_block(model, st, pk, stats)
+        out.append(st.tokens.copy())
+        for b in range(batch):
+            model.kv_append_tokens(b, st.tokens[b])
+        blocks += 1
+        if eos_early_stop and (st.eos_pos >= 0).all():
+            break
+    return np.concatenate(out, axis=1), blocks
 
 
 # ---------------------------------------------------------------------------

@@ -135,7 +135,8 @@ def check_one_step(sess, om, wl, cv, p_lib, p_or, *, rows_sample=None, heads_sam
     dstats = post["stats"] - pre["stats"]
     for b in range(B):
         assert list(dstats[b]) == [stats[b].steps_used, stats[b].committed_by_sampler,
-                                   stats[b].forced_at_budget, stats[b].eos_autofill]
+                                   stats[b].forced_at_budget, stats[b].eos_autofill,
+                                   stats[b].frozen, stats[b].edited]
     if report is not None:
         report["near_ties"] = report.get("near_ties", 0) + near_ties
     return pre, post
@@ -285,7 +286,8 @@ def test_entropy_bound_sampling_stage():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("C", [1, 7, 32, 100, 256, 1024])
-@pytest.mark.parametrize("mode", ["greedy", "thr0", "thr_big_q1", "eb", "uniform", "forced"])
+@pytest.mark.parametrize("mode", ["greedy", "thr0", "thr_big_q1", "eb", "uniform", "forced",
+                                  "stop", "stop_high_h", "edit", "edit_all"])
 def test_commit_bit_exact(C, mode):
     from masked_block_diffusion_denoise_b200.session import Session, sampler_params
     sh = W.ModelShape(d_model=64, n_heads=2, n_kv_heads=1, head_dim=32, vocab=5000, dtype="f32")
@@ -304,6 +306,14 @@ def test_commit_bit_exact(C, mode):
             kw.update(entropy_bound=2.0, corruption="uniform")
         if mode == "uniform":
             kw.update(corruption="uniform")
+        if mode == "stop":
+            kw.update(stability_steps=2, stop_entropy=0.5)
+        if mode == "stop_high_h":
+            kw.update(stability_steps=1, stop_entropy=0.05)
+        if mode == "edit":
+            kw.update(editing=1, editing_threshold=0.6)
+        if mode == "edit_all":
+            kw.update(editing=1, editing_threshold=0.0, corruption="uniform")
         p_lib = sampler_params(**kw)
         p_or = O.SamplerParams(**kw)
         tokens = r.integers(0, sh.vocab, size=(B, C)).astype(np.int64)
@@ -322,14 +332,19 @@ def test_commit_bit_exact(C, mode):
         conf[3, :] = np.float32(0.6)           # exactly the threshold
         ent = (r.random((B, C)) * 0.5).astype(np.float32)
         ent[:, ::4] = np.float32(0.0)
+        # adaptive stopping state: canvases 0-2 repeat their argmax, canvas 3
+        # changes one position; canvas 0 and 1 reach two stable steps
+        prev_cand = cand.astype(np.int64).copy()
+        prev_cand[3, C - 1] += 1
+        stable = np.array([1, 2, 0, 5, 0], dtype=np.int64)
         cv = sess.new_canvas(B, C)
-        cv.load(tokens, committed, step, done, np.full(B, -1))
+        cv.load(tokens, committed, step, done, np.full(B, -1), prev_cand, stable)
         dev = lambda a: torch.as_tensor(a).cuda()
         sess.commit(cv, p_lib, dev(cand), dev(conf), dev(ent))
         sess.check()
         got = cv.numpy()
         st = O.CanvasState(tokens.copy(), committed.copy(), step.copy(), done.copy(),
-                           np.full(B, -1))
+                           np.full(B, -1), prev_cand.copy(), stable.copy())
         stats = [O.CanvasStats() for _ in range(B)]
         for b in range(B):
             O.select_canvas(st, b, cand[b], conf[b], ent[b], p_or, vocab=sh.vocab,
@@ -339,9 +354,17 @@ def test_commit_bit_exact(C, mode):
         assert np.array_equal(got["step"], st.step)
         assert np.array_equal(got["done"], st.done)
         assert np.array_equal(got["eos_pos"][:4], st.eos_pos[:4])
+        if mode.startswith("stop"):
+            assert np.array_equal(got["prev_cand"][:4], st.prev_cand[:4])
+            assert np.array_equal(got["stable"][:4], st.stable[:4])
+        if mode == "stop":
+            assert sum(x.frozen for x in stats) > 0
+        if mode.startswith("edit") and C > 1:
+            assert sum(x.edited for x in stats) > 0
         for b in range(B):
             assert list(got["stats"][b]) == [stats[b].steps_used, stats[b].committed_by_sampler,
-                                             stats[b].forced_at_budget, stats[b].eos_autofill]
+                                             stats[b].forced_at_budget, stats[b].eos_autofill,
+                                             stats[b].frozen, stats[b].edited]
     finally:
         sess.close()
 
