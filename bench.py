@@ -321,7 +321,9 @@ def run_ours(a):
         pk = peaks()
         shape = RL.StepShape(sh.d_model, sh.n_heads, sh.n_kv_heads, sh.head_dim, sh.vocab, 2,
                              wl.canvas, [int(x) for x in lens])
-        work_ = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256)
+        lm_fp8 = bool(getattr(sh, "lm_fp8", False))
+        work_ = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256,
+                             lm_elem_bytes=1 if lm_fp8 else 0)
         lm_avg_s = statistics.mean(lm_ms) / 1e3
         bound = "hbm" if work_["lm_head"]["flop"] / work_["lm_head"]["bytes"] < 250 else "tensor"
         if bound == "hbm":
@@ -332,7 +334,8 @@ def run_ours(a):
             ach = work_["lm_head"]["flop"] / lm_avg_s / 1e12
             peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
             unit = "TFLOP/s"
-        roof = {"kernel": "gemm_tc_kernel<EPI_LM> (LM head + fused vocab reduction)",
+        roof = {"kernel": "gemm_tc_kernel<EPI_LM%s> (LM head + fused vocab reduction)"
+                          % (", e4m3" if lm_fp8 else ""),
                 "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
                 "frac": round(ach / peak, 4), "traffic": None,
                 "peak_source": pk.get("source", "measured") + (" hbm_gbs" if bound == "hbm"
@@ -349,7 +352,8 @@ def run_ours(a):
             "metric": "denoise steps/s", "value": round(aggregate_rate(world, K, ms_max), 2),
             "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": max(Wm, S),
             "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if sh.dtype == "bf16" else "f32",
+            "vs_baseline": None,
+            "dtype": ("bf16, LM head e4m3" if lm_fp8 else "bf16") if sh.dtype == "bf16" else "f32",
             "data": "synthetic: seeded random-init weights N(0,0.02), embeddings and prefix "
                     "K/V N(0,1), all-mask canvas",
             "config": {"workload": a.workload, "batch": wl.batch, "canvas": wl.canvas,

@@ -75,6 +75,17 @@ typedef struct {
   int max_batch;    /* sequences (canvases) per call                       */
   int max_prefix;   /* KV capacity per sequence for the finished prefix    */
   int max_canvas;   /* largest canvas length, <= 1024                       */
+  /* 1: e4m3 LM head (bf16 models, d_model % 16 == 0).  Online FP8
+   * quantisation of the head's weights (NLD tutorial, section 8.6; course
+   * "Diffusion LLMs", section 15: low-bit weights are the Blackwell path):
+   * dlm_create quantises W_lm per vocabulary row into a context-owned copy,
+   * scale s_v = max|W_v| / 448 (1 for a zero row), q = e4m3(W / s_v), round
+   * to nearest even, saturating; W_lm is not read afterwards.  The tensor
+   * cores take both operands in 8 bits, so every step quantises the head's
+   * input rows y the same way (a_r = max|y_r| / 448) and the logits are
+   * (sum_k qy_rk qW_vk) * (a_r * s_v), the factor rounded to float32.
+   * 0: the head in the model's element type. */
+  int lm_fp8;
 } dlm_model_desc;
 
 /* Device pointers, caller-owned, valid for the life of the context; element
@@ -247,15 +258,21 @@ int dlm_commit(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
  * which: DLM_BUF_X [M][d], DLM_BUF_Q [M][H][Dh], DLM_BUF_O [M][H*Dh],
  * DLM_BUF_Y [M][d] (model element type; M = batch * C, row b*C + i),
  * DLM_BUF_CAND int32 [M], DLM_BUF_CONF float [M], DLM_BUF_ENTROPY float [M],
- * DLM_BUF_K_CACHE / DLM_BUF_V_CACHE [max_batch][Hkv][max_prefix+max_canvas][Dh].
+ * DLM_BUF_K_CACHE / DLM_BUF_V_CACHE [max_batch][Hkv][max_prefix+max_canvas][Dh];
+ * with lm_fp8 also DLM_BUF_LM_Q uint8 e4m3 [vocab][d] and DLM_BUF_LM_SCALE
+ * float [vocab rounded up to 256] (zero padding), DLM_BUF_Y_Q uint8 e4m3
+ * [M][d] and DLM_BUF_Y_SCALE float [M] (DLM_EINVAL without lm_fp8).
  * *ptr receives a device pointer owned by the context, *bytes its size. */
 enum { DLM_BUF_X = 0, DLM_BUF_Q = 1, DLM_BUF_O = 2, DLM_BUF_Y = 3, DLM_BUF_CAND = 4,
-       DLM_BUF_CONF = 5, DLM_BUF_ENTROPY = 6, DLM_BUF_K_CACHE = 7, DLM_BUF_V_CACHE = 8 };
+       DLM_BUF_CONF = 5, DLM_BUF_ENTROPY = 6, DLM_BUF_K_CACHE = 7, DLM_BUF_V_CACHE = 8,
+       DLM_BUF_LM_Q = 9, DLM_BUF_LM_SCALE = 10, DLM_BUF_Y_Q = 11, DLM_BUF_Y_SCALE = 12 };
 int dlm_debug_buffer(dlm_ctx *ctx, int which, void **ptr, size_t *bytes);
 
 /* Full float32 logits of the rows in DLM_BUF_Y: `logits` (device float
  * [batch*canvas][vocab]) receives y W_lm^T from the same GEMM main loop as
- * the fused reduction (the store epilogue instead of the reduction). */
+ * the fused reduction (the store epilogue instead of the reduction); with
+ * lm_fp8 the logits of the last step's quantised rows (DLM_BUF_Y_Q) with the
+ * same scale factor as the step. */
 int dlm_debug_logits(dlm_ctx *ctx, int batch, int canvas, float *logits, void *stream);
 
 /* Stages of a step, for dlm_set_stage_events.  DLM_STAGE_COMMIT is the one

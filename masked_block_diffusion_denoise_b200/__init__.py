@@ -16,7 +16,8 @@ __all__ = [
     "DLM_OK", "DLM_EINVAL", "DLM_ENOMEM", "DLM_ECUDA", "DLM_ECAP", "DLM_ETIMEOUT",
     "DLM_EBOUNDS", "DLM_ESTATE", "DLM_F32", "DLM_BF16", "DLM_MASK", "DLM_UNIFORM",
     "DLM_BUF_X", "DLM_BUF_Q", "DLM_BUF_O", "DLM_BUF_Y", "DLM_BUF_CAND", "DLM_BUF_CONF",
-    "DLM_BUF_ENTROPY", "DLM_BUF_K_CACHE", "DLM_BUF_V_CACHE",
+    "DLM_BUF_ENTROPY", "DLM_BUF_K_CACHE", "DLM_BUF_V_CACHE", "DLM_BUF_LM_Q", "DLM_BUF_LM_SCALE",
+    "DLM_BUF_Y_Q", "DLM_BUF_Y_SCALE",
     "dlm_model_desc", "dlm_weights", "dlm_sampler_params", "dlm_canvas", "dlm_canvas_stats",
     "DlmError", "lib", "library_path", "dlm_create", "dlm_destroy", "dlm_kv_append",
     "dlm_reset_kv", "dlm_kv_length", "dlm_canvas_init", "dlm_denoise_step",
@@ -31,7 +32,8 @@ DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, 
 DLM_F32, DLM_BF16 = 0, 1
 DLM_MASK, DLM_UNIFORM = 0, 1
 (DLM_BUF_X, DLM_BUF_Q, DLM_BUF_O, DLM_BUF_Y, DLM_BUF_CAND, DLM_BUF_CONF, DLM_BUF_ENTROPY,
- DLM_BUF_K_CACHE, DLM_BUF_V_CACHE) = range(9)
+ DLM_BUF_K_CACHE, DLM_BUF_V_CACHE, DLM_BUF_LM_Q, DLM_BUF_LM_SCALE, DLM_BUF_Y_Q,
+ DLM_BUF_Y_SCALE) = range(13)
 
 (DLM_STAGE_EMBED, DLM_STAGE_QKV, DLM_STAGE_ATTENTION, DLM_STAGE_WO, DLM_STAGE_LM_HEAD,
  DLM_STAGE_COMMIT, DLM_NUM_STAGES) = range(7)
@@ -49,7 +51,8 @@ class dlm_model_desc(ctypes.Structure):
                 ("vocab", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("rope_theta", ctypes.c_float), ("mask_id", ctypes.c_int),
                 ("eos_id", ctypes.c_int), ("max_batch", ctypes.c_int),
-                ("max_prefix", ctypes.c_int), ("max_canvas", ctypes.c_int)]
+                ("max_prefix", ctypes.c_int), ("max_canvas", ctypes.c_int),
+                ("lm_fp8", ctypes.c_int)]
 
 
 class dlm_weights(ctypes.Structure):

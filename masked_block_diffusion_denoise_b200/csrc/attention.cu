@@ -58,7 +58,11 @@ struct AttnParams {
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const AttnParams p) {
-  pdl_wait_then_release();
+  // Before the wait for the previous kernel this CTA reads only data of
+  // kernels that finished before that one started (cache lengths, done
+  // flags, the active count) and the cached prefix: barriers, tensor memory
+  // and the K/V tiles that lie wholly inside the prefix are set up early;
+  // the query tile and tiles that reach the canvas slots follow the wait.
   if (p.n_active != nullptr && *p.n_active == 0) return;
   const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
@@ -97,6 +101,29 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  __syncthreads();
+  const int plane = b * p.Hkv + g;
+  auto issue_kv = [&](int t) {
+    const int st = t % kStages;
+    uint8_t* base = ring + st * kStageBytes;
+    const int key0 = k_begin + t * kKeys;
+    mbar_arrive_expect_tx(&kv_full[st], kStageBytes);
+    tma_load_3d(base, &tmK, &kv_full[st], 0, key0, plane);
+    tma_load_3d(base + kHalf, &tmK, &kv_full[st], 64, key0, plane);
+    tma_load_3d(base + 2 * kHalf, &tmV, &kv_full[st], 0, key0, plane);
+    tma_load_3d(base + 3 * kHalf, &tmV, &kv_full[st], 64, key0, plane);
+  };
+  int pre = 0;   // tiles issued before the wait (prefix keys only)
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    const int n_prefix = p.lens[b];
+    while (pre < kStages && pre < n_tiles && k_begin + (pre + 1) * kKeys <= n_prefix) {
+      issue_kv(pre);
+      ++pre;
+    }
+  }
+  pdl_wait_then_release();
   // query tile -> shared memory, two 64-column halves, 128-byte swizzle
   for (int idx = tid; idx < kRowsCta * 16; idx += blockDim.x) {
     const int lr = idx >> 4, ch = idx & 15;
@@ -114,25 +141,16 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int plane = b * p.Hkv + g;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      tma_prefetch(&tmK);
-      tma_prefetch(&tmV);
-      int issued = 0;
-      for (int t = 0; t < n_tiles; ++t) {
+      int issued = pre;
+      for (int t = pre; t < n_tiles; ++t) {
         const int st = t % kStages;
         if (!mbar_wait_bounded(&kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag))
           break;
-        uint8_t* base = ring + st * kStageBytes;
-        const int key0 = k_begin + t * kKeys;
-        mbar_arrive_expect_tx(&kv_full[st], kStageBytes);
-        tma_load_3d(base, &tmK, &kv_full[st], 0, key0, plane);
-        tma_load_3d(base + kHalf, &tmK, &kv_full[st], 64, key0, plane);
-        tma_load_3d(base + 2 * kHalf, &tmV, &kv_full[st], 0, key0, plane);
-        tma_load_3d(base + 3 * kHalf, &tmV, &kv_full[st], 64, key0, plane);
+        issue_kv(t);
         ++issued;
       }
       if (*abort_flag) {

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
@@ -49,6 +50,11 @@ struct dlm_ctx {
   ModelDims md{};
   int dev = 0, num_sms = 148;
   bool bf16 = true;
+  // e4m3 LM head: quantised weights, their scales, the step's quantised rows
+  bool lm_f8 = false;
+  uint8_t *w_lm_q = nullptr, *yq = nullptr;
+  float *s_lm = nullptr, *s_y = nullptr;
+  size_t s_lm_count = 0;
   size_t es = 2;
   const void *emb = nullptr, *w_o = nullptr, *w_lm = nullptr;
   void* w_qkv = nullptr;
@@ -123,21 +129,24 @@ int dalloc(dlm_ctx* ctx, T** p, size_t bytes) {
   return DLM_OK;
 }
 
+// row-major [rows][cols] of bf16 (u8 = false) or one-byte e4m3 (u8 = true);
+// the box is 128 bytes of a row (the 128-byte swizzle span) x box_rows
 const CUtensorMap* map2d(dlm_ctx* ctx, const void* ptr, uint64_t rows, uint64_t cols,
-                         uint32_t box_rows) {
-  auto key = std::make_tuple(ptr, rows, cols, box_rows);
+                         uint32_t box_rows, bool u8 = false) {
+  auto key = std::make_tuple(ptr, rows, cols, box_rows | (u8 ? 0x10000u : 0u));
   auto it = ctx->maps.find(key);
   if (it != ctx->maps.end()) return &it->second;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return nullptr;
   CUtensorMap m;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {cols * (u8 ? 1 : 2)};
+  cuuint32_t box[2] = {u8 ? 128u : 64u, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(&m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return nullptr;
   return &(ctx->maps[key] = m);
 }
@@ -197,6 +206,7 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
   const int mt = cdiv(M, 128);
   if (epi == EPI_LM) {
     p.BN = mt > 1 ? 256 : 128;
+    p.f8 = ctx->lm_f8 ? 1 : 0;
     return p;
   }
   if (mt > 1) {
@@ -373,8 +383,10 @@ int run_gemm(dlm_ctx* ctx, const void* A, const void* B, int Brows, const GemmPl
              const GemmIO& io, cudaStream_t st) {
   cudaError_t e;
   if (ctx->bf16) {
-    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K, 128);
-    const CUtensorMap* tb = map2d(ctx, B, (uint64_t)Brows, (uint64_t)plan.K, (uint32_t)plan.BN);
+    const bool u8 = plan.f8 != 0;
+    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K, 128, u8);
+    const CUtensorMap* tb =
+        map2d(ctx, B, (uint64_t)Brows, (uint64_t)plan.K, (uint32_t)plan.BN, u8);
     if (ta == nullptr || tb == nullptr)
       return fail(ctx, DLM_ECUDA, "cuTensorMapEncodeTiled failed");
     e = gemm_tc(*ta, *tb, plan, io, ctx->num_sms, st);
@@ -504,7 +516,18 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.done = c->done;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
-    if (int rc = run_gemm(ctx, ctx->y, ctx->w_lm, md.V, pl, io, st)) return rc;
+    if (ctx->lm_f8) {
+      // e4m3 head: the rows are quantised first, the scales enter the epilogue
+      e = quantize_rows_e4m3(ctx->y, rows, md.d, ctx->yq, ctx->s_y, C, c->done, ctx->n_active,
+                             st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "quantize rows", e);
+      ++ctx->launches;
+      io.epi.row_scale = ctx->s_y;
+      io.epi.col_scale = ctx->s_lm;
+      if (int rc = run_gemm(ctx, ctx->yq, ctx->w_lm_q, md.V, pl, io, st)) return rc;
+    } else {
+      if (int rc = run_gemm(ctx, ctx->y, ctx->w_lm, md.V, pl, io, st)) return rc;
+    }
   }
   STAGE(DLM_STAGE_LM_HEAD, true);
   // a6 + a7: cross-tile reduction, then commit / re-noise, one launch
@@ -603,10 +626,14 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
     return fail(nullptr, DLM_EINVAL, "need max_batch >= 1, max_prefix >= 0, 1 <= max_canvas <= 1024");
   if (!w->emb || !w->w_q || !w->w_k || !w->w_v || !w->w_o || !w->w_lm)
     return fail(nullptr, DLM_EINVAL, "every weight pointer must be non-NULL");
+  if (d.lm_fp8 != 0 && d.lm_fp8 != 1) return fail(nullptr, DLM_EINVAL, "lm_fp8 must be 0 or 1");
+  if (d.lm_fp8 && (d.dtype != DLM_BF16 || d.d_model % 16 != 0))
+    return fail(nullptr, DLM_EINVAL, "lm_fp8 needs a bf16 model with d_model % 16 == 0");
 
   dlm_ctx* ctx = new dlm_ctx();
   ctx->d = d;
   ctx->bf16 = d.dtype == DLM_BF16;
+  ctx->lm_f8 = d.lm_fp8 == 1;
   ctx->es = ctx->bf16 ? 2 : 4;
   cudaGetDevice(&ctx->dev);
   cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->dev);
@@ -657,6 +684,13 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if ((rc = dalloc(ctx, &ctx->h_stable, d.max_batch * sizeof(int32_t)))) return bail(rc);
   ctx->part_floats = part_floats_needed(ctx);
   if ((rc = dalloc(ctx, &ctx->part, ctx->part_floats * sizeof(float)))) return bail(rc);
+  if (ctx->lm_f8) {
+    ctx->s_lm_count = (size_t)cdiv(d.vocab, 256) * 256;   // whole tiles of either width
+    if ((rc = dalloc(ctx, &ctx->w_lm_q, (size_t)d.vocab * dm))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->s_lm, ctx->s_lm_count * sizeof(float)))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->yq, ctx->Mmax * dm))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->s_y, ctx->Mmax * sizeof(float)))) return bail(rc);
+  }
 
   cudaError_t e = cudaSuccess;
   auto ck = [&](cudaError_t r, const char* what) {
@@ -681,6 +715,14 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if (d.rope_theta > 0.0f)
     ck(rope_table_init(ctx->rope, ctx->Lcap, d.head_dim, (double)d.rope_theta, nullptr),
        "rope table");
+  if (ctx->lm_f8) {
+    ck(cudaMemset(ctx->s_lm, 0, ctx->s_lm_count * sizeof(float)), "memset LM scales");
+    ck(cudaMemset(ctx->yq, 0, ctx->Mmax * dm), "memset quantised rows");
+    ck(cudaMemset(ctx->s_y, 0, ctx->Mmax * sizeof(float)), "memset row scales");
+    ck(quantize_rows_e4m3(w->w_lm, d.vocab, d.d_model, ctx->w_lm_q, ctx->s_lm, 1, nullptr,
+                          nullptr, nullptr),
+       "quantise LM head");
+  }
   ck(cudaStreamCreateWithFlags(&ctx->cap, cudaStreamNonBlocking), "capture stream");
   ck(cudaDeviceSynchronize(), "create sync");
   if (e != cudaSuccess) return bail(DLM_ECUDA);
@@ -948,6 +990,25 @@ int dlm_debug_buffer(dlm_ctx* ctx, int which, void** ptr, size_t* bytes) {
     case DLM_BUF_ENTROPY: *ptr = ctx->ent; *bytes = M * 4; break;
     case DLM_BUF_K_CACHE: *ptr = ctx->kc; *bytes = kv * es; break;
     case DLM_BUF_V_CACHE: *ptr = ctx->vc; *bytes = kv * es; break;
+    case DLM_BUF_LM_Q:
+    case DLM_BUF_LM_SCALE:
+    case DLM_BUF_Y_Q:
+    case DLM_BUF_Y_SCALE:
+      if (!ctx->lm_f8) return fail(ctx, DLM_EINVAL, "the context has no e4m3 LM head");
+      if (which == DLM_BUF_LM_Q) {
+        *ptr = ctx->w_lm_q;
+        *bytes = (size_t)ctx->d.vocab * dm;
+      } else if (which == DLM_BUF_LM_SCALE) {
+        *ptr = ctx->s_lm;
+        *bytes = ctx->s_lm_count * 4;
+      } else if (which == DLM_BUF_Y_Q) {
+        *ptr = ctx->yq;
+        *bytes = M * dm;
+      } else {
+        *ptr = ctx->s_y;
+        *bytes = M * 4;
+      }
+      break;
     default: return fail(ctx, DLM_EINVAL, "unknown buffer id");
   }
   return DLM_OK;
@@ -965,6 +1026,11 @@ int dlm_debug_logits(dlm_ctx* ctx, int batch, int canvas, float* logits, void* s
   GemmIO io;
   io.out = logits;
   io.err = ctx->err;
+  if (ctx->lm_f8) {
+    io.epi.row_scale = ctx->s_y;
+    io.epi.col_scale = ctx->s_lm;
+    return run_gemm(ctx, ctx->yq, ctx->w_lm_q, ctx->d.vocab, pl, io, (cudaStream_t)stream);
+  }
   return run_gemm(ctx, ctx->y, ctx->w_lm, ctx->d.vocab, pl, io, (cudaStream_t)stream);
 }
 

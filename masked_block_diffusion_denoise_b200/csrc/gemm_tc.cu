@@ -95,11 +95,29 @@ __device__ __forceinline__ bool get_unit(const TcParams& p, int k, int& m, int& 
 
 constexpr int kGemmThreads = 320;   // producer, MMA, 8 epilogue warps
 
-template <int BN, int EPI>
+// Scale 32 accumulator columns of one row to logits: v_j * (a * s_j), the
+// factor rounded to float32 first (e4m3 operands with per-row scales).
+__device__ __forceinline__ void scale_chunk(float (&v)[32], float a, const float* __restrict__ cs) {
+  const float4* c4 = reinterpret_cast<const float4*>(cs);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 sc = c4[j];
+    v[4 * j + 0] = __fmul_rn(v[4 * j + 0], __fmul_rn(a, sc.x));
+    v[4 * j + 1] = __fmul_rn(v[4 * j + 1], __fmul_rn(a, sc.y));
+    v[4 * j + 2] = __fmul_rn(v[4 * j + 2], __fmul_rn(a, sc.z));
+    v[4 * j + 3] = __fmul_rn(v[4 * j + 3], __fmul_rn(a, sc.w));
+  }
+}
+
+// F8: e4m3 operands (kind::f8f6f4); a k-block is then 128 elements, the same
+// 128 bytes per row as 64 bf16 elements, so ring, swizzle and descriptors
+// are shared.
+template <int BN, int EPI, bool F8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
+  constexpr int kBKe = F8 ? 2 * kBK : kBK;   // elements per k-block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -136,12 +154,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the prologue above touched only shared and tensor memory
+  // The weights (B) do not depend on the previous kernel: before waiting for
+  // it, the producer puts the B tiles of the first ring stages in flight
+  // (expected bytes raised, no arrival yet); the A tiles follow the wait.
+  // Weights are read once per launch: they stream through L2 with evict_first.
+  int pre = 0;
+  uint64_t pol_stream = 0;
+  if (warp == 0 && lane == 0) {
+    pol_stream = l2_evict_first_policy();
+    int m0, n0, kb0, kb1, sp0;
+    if (get_unit<EPI>(p, 0, m0, n0, kb0, kb1, sp0)) {
+      pre = min(Cfg::kStages, kb1 - kb0);
+      for (int s = 0; s < pre; ++s) {
+        const int kb = kb0 + s;
+        mbar_expect_tx(&full[s], Cfg::kBBytes);
+        tma_load_2d_hint(smem + s * Cfg::kStageBytes + Cfg::kABytes, &tmB, &full[s], kb * kBKe,
+                         n0 * BN, pol_stream);
+      }
+    }
+  }
+  // the prologue above touched only shared and tensor memory and weights
   pdl_wait_then_release();
   const bool skip = p.n_active != nullptr && *p.n_active == 0;
 
   if (skip) {
-    // nothing to do this step: fall through to the teardown
+    // nothing to do this step: land the early weight tiles, then teardown
+    if (warp == 0 && lane == 0)
+      for (int s = 0; s < pre; ++s) {
+        mbar_arrive(&full[s]);
+        mbar_wait_bounded(&full[s], 0u, nullptr);
+      }
   } else if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -158,9 +200,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t* sa = smem + stage * Cfg::kStageBytes;
           uint8_t* sb = sa + Cfg::kABytes;
-          mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-          tma_load_2d(sa, &tmA, &full[stage], kb * kBK, m * kBM);
-          tma_load_2d(sb, &tmB, &full[stage], kb * kBK, n * BN);
+          if (issued < pre) {
+            // this stage's B tile is already in flight
+            mbar_arrive_expect_tx(&full[stage], Cfg::kABytes);
+            tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+            tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
+            tma_load_2d_hint(sb, &tmB, &full[stage], kb * kBKe, n * BN, pol_stream);
+          }
           ++issued;
           if (++stage == Cfg::kStages) {
             stage = 0;
@@ -170,20 +218,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!ok) {
         // let the copies already in flight land before the CTA exits
-        int st = stage, ph = phase;
-        for (int i = 0; i < Cfg::kStages && i < issued; ++i) {
-          if (--st < 0) {
-            st = Cfg::kStages - 1;
-            ph ^= 1;
+        if (issued < pre) {
+          // early B tiles without their A: arrive so the phase can complete
+          for (int s = issued; s < pre; ++s) mbar_arrive(&full[s]);
+          for (int s = 0; s < pre; ++s) mbar_wait_bounded(&full[s], 0u, nullptr);
+        } else {
+          int st = stage, ph = phase;
+          for (int i = 0; i < Cfg::kStages && i < issued; ++i) {
+            if (--st < 0) {
+              st = Cfg::kStages - 1;
+              ph ^= 1;
+            }
+            mbar_wait_bounded(&full[st], (uint32_t)ph, nullptr);
           }
-          mbar_wait_bounded(&full[st], (uint32_t)ph, nullptr);
         }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -202,10 +256,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
           const uint32_t sb = sa + Cfg::kABytes;
+          // four instructions of 32 bytes of K per 128-byte k-block
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            umma_bf16(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
-                      (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (F8)
+              umma_e4m3(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
+                        (kb > kb0 || k > 0) ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
+                        (kb > kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           if (++stage == Cfg::kStages) {
@@ -239,6 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int lm_row = -1, lm_canvas = 0, lm_pos = 0, lm_step = 0;
     bool lm_live = false;
     float lm_inv_t = 1.f;
+    float lm_a = 0.f;   // F8: the row's scale
     if constexpr (EPI == EPI_LM) {
       m = blockIdx.x % p.m_tiles;
       lm_row = m * kBM + quad * 32 + lane;
@@ -247,6 +307,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       lm_live = lm_row < p.M && (p.done == nullptr || p.done[lm_canvas] == 0);
       lm_step = lm_live ? p.epi.step[lm_canvas] : 0;
       lm_inv_t = lm_inv_temp(p.epi, lm_step);
+      if constexpr (F8) lm_a = lm_live ? p.epi.row_scale[lm_row] : 0.f;
     }
     for (int it = 0; get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag)) break;
@@ -262,6 +323,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float v[32];
             tmem_ld32(taddr + c, v);
             const int col0 = n * BN + c;
+            if constexpr (F8) {
+              if (p.epi.col_scale != nullptr)
+                scale_chunk(v, row < p.M ? p.epi.row_scale[row] : 0.f, p.epi.col_scale + col0);
+            }
             if (row < p.M) {
               if (col0 + 32 <= p.N) {
                 float4* dst = reinterpret_cast<float4*>(orow + col0);
@@ -279,6 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = cb; c < cb + kHalfN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
+            if constexpr (F8) scale_chunk(v, lm_a, p.epi.col_scale + n * BN + c);
             if (lm_live)
               rs_update<32>(rs, v, n * BN + c, lm_inv_t, p.epi, lm_canvas, lm_pos, lm_step);
           }
@@ -420,20 +486,20 @@ int tc_grid(int units, int m_tiles, int n_tiles, int epi, int num_sms) {
   return units < num_sms ? units : num_sms;
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool F8 = false>
 cudaError_t launch_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const TcParams& p,
                       int num_sms, cudaStream_t st) {
   using Cfg = TcCfg<BN>;
   static bool attr_set = false;   // per process; one device is used per process
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int grid = tc_grid(p.units, p.m_tiles, p.n_tiles, EPI, num_sms);
-  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kGemmThreads), Cfg::kSmem, st, tmA,
-                    tmB, p);
+  return launch_pdl(gemm_tc_kernel<BN, EPI, F8>, dim3(grid), dim3(kGemmThreads), Cfg::kSmem, st,
+                    tmA, tmB, p);
 }
 
 }  // namespace
@@ -447,7 +513,8 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.m_tiles = (plan.M + kBM - 1) / kBM;
   p.n_tiles = (plan.N + plan.BN - 1) / plan.BN;
   p.splits = plan.splits;
-  p.kblocks = (plan.K + kBK - 1) / kBK;
+  const int kbe = plan.f8 ? 2 * kBK : kBK;   // elements per k-block
+  p.kblocks = (plan.K + kbe - 1) / kbe;
   p.units = p.m_tiles * p.n_tiles * p.splits;
   p.out = io.out;
   p.part = io.part;
@@ -457,6 +524,16 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.done = io.done;
   p.n_active = io.n_active;
   p.err = io.err;
+  if (plan.f8) {
+    // e4m3 operands: the LM head and its full-logit inspection only
+    if (plan.epi == EPI_LM)
+      return plan.BN == 128 ? launch_tc<128, EPI_LM, true>(tmA, tmB, p, num_sms, st)
+                            : launch_tc<256, EPI_LM, true>(tmA, tmB, p, num_sms, st);
+    if (plan.epi == EPI_F32)
+      return plan.BN == 128 ? launch_tc<128, EPI_F32, true>(tmA, tmB, p, num_sms, st)
+                            : launch_tc<256, EPI_F32, true>(tmA, tmB, p, num_sms, st);
+    return cudaErrorInvalidValue;
+  }
   if (plan.BN == 128) {
     return plan.epi == EPI_LM ? launch_tc<128, EPI_LM>(tmA, tmB, p, num_sms, st)
                               : launch_tc<128, EPI_F32>(tmA, tmB, p, num_sms, st);

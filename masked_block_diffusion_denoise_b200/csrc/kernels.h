@@ -19,6 +19,7 @@ struct GemmPlan {
   int BN;       // 128 or 256 (tcgen05); 64 (fp32 SIMT)
   int splits;   // K splits (EPI_F32 only)
   int epi;      // EPI_F32 / EPI_LM
+  int f8 = 0;       // e4m3 operands (tcgen05 only; EPI_LM and EPI_F32)
 };
 
 struct ModelDims;
@@ -98,6 +99,11 @@ cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint6
 
 // lens[b] += n for b < B
 cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st);
+
+// e4m3 rows with one float32 scale each (bf16 input, cols % 8 == 0); rows of
+// finished canvases (row / C, when done is given) are skipped
+cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, float* scale, int C,
+                               const uint8_t* done, const int* n_active, cudaStream_t st);
 
 // ---- attention.cu ------------------------------------------------------------
 struct AttnPlan {

@@ -33,6 +33,9 @@ struct LmEpi {
   uint32_t seed_lo, seed_hi;
   const int32_t* step;   // [B] steps taken (sampling counter and anneal)
   int n_tiles;    // partials per row
+  // e4m3 LM head: logit = acc * (row_scale[r] * col_scale[v]); null otherwise
+  const float* row_scale;
+  const float* col_scale;   // padded with zeros to whole vocabulary tiles
 };
 
 struct RowState {

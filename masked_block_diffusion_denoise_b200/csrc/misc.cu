@@ -1,6 +1,8 @@
 // Element-wise kernels around the GEMMs: RoPE table, embedding gather, the
 // projection epilogues (split-K sum, rotary embedding, KV-cache write,
 // residual), KV copy-in and canvas initialisation.
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 
 namespace dlm {
@@ -140,6 +142,52 @@ __global__ void add_len_all_kernel(int32_t* lens, int B, int n) {
   if (b < B) lens[b] += n;
 }
 
+// e4m3 quantisation of bf16 rows: s = max|x| / 448 (1 for an all-zero row),
+// q = e4m3(x / s), round to nearest even, saturating.  One CTA per row;
+// rows of finished canvases (row / C) are skipped.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(
+    const __nv_bfloat16* __restrict__ x, int rows, int cols, uint8_t* __restrict__ q,
+    float* __restrict__ scale, int C, const uint8_t* __restrict__ done, const int* n_active) {
+  pdl_wait_then_release();
+  if (n_active != nullptr && *n_active == 0) return;
+  const int r = blockIdx.x;
+  if (r >= rows || (done != nullptr && done[r / C])) return;
+  const __nv_bfloat16* xr = x + (size_t)r * cols;
+  float amax = 0.f;
+  for (int i = threadIdx.x * 8; i < cols; i += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = wmax[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, wmax[w]);
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  uint8_t* qr = q + (size_t)r * cols;
+  for (int i = threadIdx.x * 8; i < cols; i += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+      const uint32_t lo = __nv_cvt_float_to_fp8(__fdiv_rn(f.x, s), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float_to_fp8(__fdiv_rn(f.y, s), __NV_SATFINITE, __NV_E4M3);
+      packed[u >> 1] |= (lo | (hi << 8)) << (16 * (u & 1));
+    }
+    *reinterpret_cast<uint2*>(qr + i) = make_uint2(packed[0], packed[1]);
+  }
+  if (threadIdx.x == 0) scale[r] = s;
+}
+
 __global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint32_t s0,
                                    uint32_t s1, int32_t* tokens, uint8_t* committed,
                                    int32_t* step, uint8_t* done, int32_t* eos_pos,
@@ -238,6 +286,13 @@ cudaError_t canvas_init(const ModelDims& md, int B, int C, int corruption, uint6
                                             (uint32_t)(seed >> 32), tokens, committed, step,
                                             done, eos_pos, prev_cand, stable);
   return cudaGetLastError();
+}
+
+cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, float* scale, int C,
+                               const uint8_t* done, const int* n_active, cudaStream_t st) {
+  if (cols % 8 != 0) return cudaErrorInvalidValue;
+  return launch_pdl(quantize_rows_kernel, dim3(rows), dim3(256), 0, st,
+                    (const __nv_bfloat16*)x, rows, cols, q, scale, C, done, n_active);
 }
 
 cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st) {

@@ -74,8 +74,12 @@ class StepShape:
         return self.canvas * len(self.prefix_lens)
 
 
-def step_work(s: StepShape, lm_tile: int = 128, part_bytes: int = 24) -> Dict[str, Dict[str, float]]:
-    """Algorithmic bytes and flops of each stage of one denoise step."""
+def step_work(s: StepShape, lm_tile: int = 128, part_bytes: int = 24,
+              lm_elem_bytes: int = 0) -> Dict[str, Dict[str, float]]:
+    """Algorithmic bytes and flops of each stage of one denoise step.
+    lm_elem_bytes = 1: the e4m3 LM head (one-byte weights and input rows, a
+    float32 scale per vocabulary row and per input row, and the quantisation
+    of the input rows); 0: the head in the model's element type."""
     e = s.elem_bytes
     M, d, V = s.rows, s.d_model, s.vocab
     qd, kvd = s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
@@ -94,9 +98,13 @@ def step_work(s: StepShape, lm_tile: int = 128, part_bytes: int = 24) -> Dict[st
                "flop": 2.0 * M * qd * d},
         "lm_head": {"bytes": float(V * d * e + M * d * e + M * ntiles * part_bytes),
                     "flop": 2.0 * M * d * V},
+        "quantize": {"bytes": 0.0, "flop": 0.0},
         "reduce": {"bytes": float(M * ntiles * part_bytes + 12 * M), "flop": 0.0},
         "commit": {"bytes": float(M * (4 + 1 + 4 + 4 + 4) * 2), "flop": 0.0},
     }
+    if lm_elem_bytes == 1:
+        out["lm_head"]["bytes"] = float(V * d + M * d + 4 * V + 4 * M + M * ntiles * part_bytes)
+        out["quantize"]["bytes"] = float(M * d * e + M * d + 4 * M)
     out["step"] = {"bytes": sum(v["bytes"] for v in out.values()),
                    "flop": sum(v["flop"] for v in out.values())}
     return out

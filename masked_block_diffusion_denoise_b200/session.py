@@ -108,7 +108,8 @@ class Session:
         desc = dlm_model_desc(shape.d_model, shape.n_heads, shape.n_kv_heads, shape.head_dim,
                               shape.vocab, DLM_BF16 if shape.dtype == "bf16" else DLM_F32,
                               float(shape.rope_theta), shape.mask_id, shape.eos_id,
-                              max_batch, max_prefix, max_canvas)
+                              max_batch, max_prefix, max_canvas,
+                              1 if getattr(shape, "lm_fp8", False) else 0)
         wts = dlm_weights(*(self.w[k].data_ptr() for k in
                             ("emb", "w_q", "w_k", "w_v", "w_o", "w_lm")))
         torch.cuda.synchronize(self.device)

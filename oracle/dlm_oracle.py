@@ -197,6 +197,46 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
     return (w @ v) / w.sum(axis=1, keepdims=True)
 
 
+# ---------------------------------------------------------------------------
+# FP8 LM head (NLD tutorial section 8.6: online BF16 -> FP8 quantisation of
+# the weights, KV cache kept in BF16; course section 15: low-bit weight paths
+# on Blackwell).  READING: one float32 scale per row, s = max|x| / 448 (1 for
+# an all-zero row), q = e4m3(x / s) with the division in float32.  The
+# tensor cores take both operands in 8 bits, so the LM head's input rows are
+# quantised the same way (per row).
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def round_to_e4m3(x) -> np.ndarray:
+    """Nearest value of the e4m3 format -- sign, 4 exponent bits (bias 7), 3
+    mantissa bits, no infinities, largest finite 448 -- ties to even;
+    magnitudes beyond 448 saturate to 448.  Values are float64."""
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    _, e = np.frexp(a)                 # a = m * 2^e with m in [0.5, 1)
+    e = np.maximum(e - 1, -6)          # binade; below 2^-6 the subnormal spacing
+    step = np.ldexp(1.0, e - 3)        # grid spacing: 3 mantissa bits
+    r = np.minimum(np.rint(a / step) * step, E4M3_MAX)   # rint: ties to even
+    return np.copysign(r, x)
+
+
+def quantize_rows_e4m3(x) -> Tuple[np.ndarray, np.ndarray]:
+    """(q, s): q [rows][cols] the e4m3 values (float64), s [rows] float32.
+    Rows are independent; they are processed in blocks to bound memory."""
+    x = np.asarray(x)
+    q = np.empty(x.shape, dtype=F64)
+    s = np.empty(x.shape[0], dtype=np.float32)
+    for r0 in range(0, x.shape[0], 4096):
+        x32 = np.asarray(x[r0:r0 + 4096], dtype=np.float32)
+        amax = np.abs(x32).max(axis=1)
+        sb = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        q[r0:r0 + 4096] = round_to_e4m3((x32 / sb[:, None]).astype(np.float32))
+        s[r0:r0 + 4096] = sb
+    return q, s
+
+
 @dataclass
 class ModelDims:
     d_model: int
@@ -208,11 +248,13 @@ class ModelDims:
     rope_theta: float = 1.0e6
     mask_id: int = 100
     eos_id: int = 11
+    lm_fp8: bool = False      # LM head with e4m3 weights and activations
 
     @classmethod
     def of(cls, shape) -> "ModelDims":
         return cls(shape.d_model, shape.n_heads, shape.n_kv_heads, shape.head_dim,
-                   shape.vocab, shape.dtype, shape.rope_theta, shape.mask_id, shape.eos_id)
+                   shape.vocab, shape.dtype, shape.rope_theta, shape.mask_id, shape.eos_id,
+                   bool(getattr(shape, "lm_fp8", False)))
 
 
 class OracleModel:
@@ -236,6 +278,8 @@ class OracleModel:
         self.w_v = conv(weights["w_v"])
         self.w_o = conv(weights["w_o"])
         self.w_lm = conv(weights["w_lm"])
+        if dims.lm_fp8:
+            self.lm_q, self.lm_scale = quantize_rows_e4m3(self.w_lm)
         self.store = round_to_bf16 if dims.dtype == "bf16" else round_to_f32
         self.k_cache: Dict[int, np.ndarray] = {}
         self.v_cache: Dict[int, np.ndarray] = {}
@@ -304,6 +348,12 @@ class OracleModel:
         return self.store(x + o @ self.w_o.T)
 
     def logits(self, y: np.ndarray) -> np.ndarray:
+        if self.dims.lm_fp8:
+            # the e4m3 head: both operands quantised per row, the products
+            # summed exactly, then one float32 factor a_r * s_v per logit
+            qy, a = quantize_rows_e4m3(y)
+            w = (a[:, None] * self.lm_scale[None, :]).astype(np.float32)
+            return (qy @ self.lm_q.T) * w.astype(F64)
         return y @ self.w_lm.T
 
     def forward(self, seq: int, tokens) -> Dict[str, np.ndarray]:

@@ -71,6 +71,27 @@ int main(void) {
                      ctypes.sizeof(dlm.dlm_canvas_stats)]
 
 
+def test_enum_values_match_header():
+    """Every DLM_* enumerator of the header has the binding's value."""
+    dlm = _library()
+    header = open(os.path.join(ROOT, "include", "dlm.h")).read()
+    names = sorted(set(re.findall(r"\b(DLM_[A-Z0-9_]+)\s*=", header)))
+    code = "#include <stdio.h>\n#include \"dlm.h\"\nint main(void) {\n"
+    code += "".join('  printf("%%d\\n", (int)%s);\n' % n for n in names)
+    code += "  return 0;\n}\n"
+    import tempfile
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "e.c")
+        exe = os.path.join(td, "e")
+        open(c, "w").write(code)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = list(map(int, subprocess.run([exe], capture_output=True, text=True,
+                                            check=True).stdout.split()))
+    assert len(names) > 20
+    for n, v in zip(names, vals):
+        assert getattr(dlm, n) == v, n
+
+
 def _desc(dlm, **kw):
     base = dict(d_model=256, n_heads=4, n_kv_heads=2, head_dim=128, vocab=1000,
                 dtype=dlm.DLM_BF16, rope_theta=1e6, mask_id=100, eos_id=11, max_batch=2,

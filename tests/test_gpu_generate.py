@@ -40,7 +40,10 @@ def test_generate_tiny_fp32_free_running(mode):
     wl = base.replace(prefix_cap=base.prefix_len[1] + N_BLOCKS * base.canvas)
     over = {}
     if mode == "stop":
-        over = dict(stability_steps=1, stop_entropy=100.0)
+        # the argmax of this random model changes between steps, so only
+        # stability 0 freezes (the stable-step count is covered bit-exactly
+        # by the commit tests)
+        over = dict(stability_steps=0, stop_entropy=100.0)
     if mode == "uniform":
         over = dict(corruption="uniform", seed=7)
     if mode == "edit":

@@ -156,6 +156,13 @@ SMALL = {
     # uniform corruption, quota from ceil(C/S)
     "small_uniform": W.small_workload("small_uniform", corruption="uniform", steps=7, quota=0,
                                       seed=3),
+    # e4m3 LM head, one M tile (128-wide vocabulary tiles, ragged vocabulary)
+    "small_fp8": W.small_workload("small_fp8", steps=6, quota=0, lm_fp8=True, seed=4),
+    # e4m3 LM head over two M tiles (256-wide vocabulary tiles), uniform corruption
+    "small_fp8_mtiles": W.small_workload("small_fp8_mtiles", n_heads=8, n_kv_heads=2, batch=4,
+                                         canvas=64, steps=4, quota=0, prefix_len=(64, 300),
+                                         prefix_cap=320, vocab=3000, lm_fp8=True,
+                                         corruption="uniform"),
 }
 
 
@@ -410,7 +417,36 @@ def test_kv_append_tokens_bf16():
 # full-size shapes: one step, sampled outputs
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("name", ["8b_b1", "encdec"])
+def test_fp8_quantisation_bit_exact():
+    """The e4m3 copies of the LM head's weights and of a step's input rows,
+    and their scales, equal the oracle's quantisation bit for bit."""
+    wl = SMALL["small_fp8"]
+    sess, om, _ = make_pair(wl)
+    try:
+        from masked_block_diffusion_denoise_b200 import (DLM_BUF_LM_Q, DLM_BUF_LM_SCALE,
+                                                         DLM_BUF_Y_Q, DLM_BUF_Y_SCALE)
+        sh = wl.shape
+        V, d = sh.vocab, sh.d_model
+        as_e4m3 = lambda t: t.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        q = as_e4m3(sess.buffer(DLM_BUF_LM_Q, (V, d), torch.uint8))
+        sc = sess.buffer(DLM_BUF_LM_SCALE, (V,), torch.float32).cpu().numpy()
+        assert np.array_equal(q, om.lm_q) and np.array_equal(sc, om.lm_scale)
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib = lib_params(wl)
+        sess.init(cv, p_lib)
+        sess.step(cv, p_lib)
+        sess.check()
+        M = wl.batch * wl.canvas
+        y = to64(sess.buffer(DLM_BUF_Y, (M, d), torch.bfloat16))
+        qy = as_e4m3(sess.buffer(DLM_BUF_Y_Q, (M, d), torch.uint8))
+        sy = sess.buffer(DLM_BUF_Y_SCALE, (M,), torch.float32).cpu().numpy()
+        ref_q, ref_s = O.quantize_rows_e4m3(y)
+        assert np.array_equal(qy, ref_q) and np.array_equal(sy, ref_s)
+    finally:
+        sess.close()
+
+
+@pytest.mark.parametrize("name", ["8b_b1", "encdec", "8b_b1_fp8"])
 def test_full_size_step_sampled(name):
     wl = W.WORKLOADS[name]
     sess, om, _ = make_pair(wl)

@@ -60,6 +60,7 @@ class ModelShape:
     rope_theta: float = 1.0e6
     mask_id: int = 100
     eos_id: int = 11
+    lm_fp8: bool = False           # LM head in e4m3 (weights and its input rows)
 
     @property
     def q_dim(self) -> int:
@@ -128,16 +129,22 @@ WORKLOADS: Dict[str, Workload] = {
                           prefix_len=(1024, 1024), prefix_cap=1024, entropy_bound=0.1,
                           t_max=0.8, t_min=0.4),
 }
+# the same workloads with the e4m3 LM head (online FP8 weight quantisation)
+for _name in ("8b_b1", "batched", "encdec"):
+    _w = WORKLOADS[_name]
+    WORKLOADS[_name + "_fp8"] = _w.replace(name=_name + "_fp8",
+                                           shape=dataclasses.replace(_w.shape, lm_fp8=True))
 
 
 def small_workload(name: str = "small", *, d_model=256, n_heads=4, n_kv_heads=2,
                    head_dim=128, vocab=4096 + 96, batch=2, canvas=32, steps=8,
-                   prefix_len=(200, 333), prefix_cap=384, dtype="bf16", **kw) -> Workload:
+                   prefix_len=(200, 333), prefix_cap=384, dtype="bf16", lm_fp8=False,
+                   **kw) -> Workload:
     """A reduced workload that the oracle finishes in seconds; by default the
     vocabulary, prefix lengths and canvas are not multiples of the kernels'
     tile sizes, so every tiling has a ragged tail."""
     shape = ModelShape(d_model=d_model, n_heads=n_heads, n_kv_heads=n_kv_heads,
-                       head_dim=head_dim, vocab=vocab, dtype=dtype)
+                       head_dim=head_dim, vocab=vocab, dtype=dtype, lm_fp8=lm_fp8)
     return Workload(name, shape, batch=batch, canvas=canvas, steps=steps,
                     prefix_len=prefix_len, prefix_cap=prefix_cap, **kw)
 
