@@ -11,14 +11,21 @@
 // that share the KV head times the C canvas positions (GQA grouping), so each
 // K/V tile is read once for all of them.  K and V stream from HBM with TMA;
 // S = Q K^T and O += P V run on the tensor cores with S and O in tensor
-// memory; the online softmax keeps one query row per thread.  Splits write
-// unnormalised partials that a second kernel combines (log-sum-exp).
+// memory; the online softmax keeps one query row per thread.  The key splits
+// of one (row tile, sequence x KV head) either form a thread-block cluster
+// and combine their unnormalised partials through distributed shared memory
+// at the end (up to 8 splits), or write them to global memory for a second
+// kernel (log-sum-exp).
 #include <math_constants.h>
+
+#include <cooperative_groups.h>
 
 #include "kernels.h"
 
 namespace dlm {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int kDh = 128;
 constexpr int kKeys = 128;                    // keys per tile (the N of S = Q K^T)
@@ -41,8 +48,16 @@ struct AttnParams {
   const int* n_active;
   int* err;
   int H, Hkv, G, C, R, chunk, nsplit;
+  int cluster;   // > 1: the nsplit CTAs of a (row tile, plane) form a cluster and combine in it
   float scale_log2;
 };
+
+// cluster exchange area (in the K/V ring, free once the last tile is done):
+// unnormalised O rows with a stride of 132 floats (16-byte aligned rows for
+// vector reads by the peers), then (max, sum) per row
+constexpr int kXoStride = kDh + 4;
+constexpr int kXoBytes = kRowsCta * kXoStride * 4;
+constexpr int kMaxCluster = 8;
 
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
 //   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
@@ -69,9 +84,11 @@ __global__ void __launch_bounds__(192, 1)
   if (p.done != nullptr && p.done[b]) return;
   const int n_keys = p.lens[b] + p.C;
   const int k_begin = split * p.chunk;
-  if (k_begin >= n_keys) return;
+  // a split past the keys exits at once, except in a cluster, where it still
+  // takes part in the exchange (with no rows of its own)
+  if (k_begin >= n_keys && p.cluster <= 1) return;
   const int k_end = min(k_begin + p.chunk, n_keys);
-  const int n_tiles = (k_end - k_begin + kKeys - 1) / kKeys;
+  const int n_tiles = k_end > k_begin ? (k_end - k_begin + kKeys - 1) / kKeys : 0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -175,7 +192,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         umma_commit(&s_full[t & 1]);
       };
-      bool ok = mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+      bool ok = n_tiles > 0 && mbar_wait_bounded(&kv_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -287,10 +304,12 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait_bounded(pv_done, (uint32_t)((n_tiles - 1) & 1), abort_flag)) {
+    float ov[kDh];
+    bool have = false;
+    if (ok && n_tiles > 0 &&
+        mbar_wait_bounded(pv_done, (uint32_t)((n_tiles - 1) & 1), abort_flag)) {
       tc_fence_after();
-      const int r = rt * kRowsCta + row;
-      float ov[kDh];
+      have = true;
       {
         uint32_t raw[kDh / 32][32];
 #pragma unroll
@@ -302,6 +321,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) ov[c * 32 + j] = __uint_as_float(raw[c][j]);
       }
+    }
+    if (p.cluster > 1) {
+      // this split's rows for the cluster: unnormalised O, running max and sum
+      fence_proxy_async_smem();
+      float* xo = reinterpret_cast<float*>(ring) + row * kXoStride;
+#pragma unroll
+      for (int j = 0; j < kDh; ++j) xo[j] = have ? ov[j] : 0.f;
+      reinterpret_cast<float2*>(ring + kXoBytes)[row] =
+          have ? make_float2(m_run, l_run) : make_float2(-CUDART_INF_F, 0.f);
+    } else if (have) {
+      const int r = rt * kRowsCta + row;
       if (r < p.R) {
         if (p.nsplit == 1) {
           const int i = r / p.G, hh = r - i * p.G;
@@ -326,6 +356,64 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
+  }
+
+  if (p.cluster > 1) {
+    // every split's rows are in its shared memory; CTA q of the cluster
+    // combines rows q*ceil(128/n) .. of the tile for all splits (fixed order).
+    // All peer reads of an item are issued before any of them is used.
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int n = p.cluster;
+    const int q = (int)cluster.block_rank();
+    const int per = (kRowsCta + n - 1) / n;
+    const int r0 = q * per, r1 = min(kRowsCta, r0 + per);
+    const float* xo_self = reinterpret_cast<const float*>(ring);
+    const float2* xml_self = reinterpret_cast<const float2*>(ring + kXoBytes);
+    const float* xo_p[kMaxCluster];
+    const float2* xml_p[kMaxCluster];
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j) {
+      const int jj = j < n ? j : 0;
+      xo_p[j] = cluster.map_shared_rank(xo_self, jj);
+      xml_p[j] = cluster.map_shared_rank(xml_self, jj);
+    }
+    for (int it = tid; it < (r1 - r0) * (kDh / 4); it += blockDim.x) {
+      const int lr = r0 + it / (kDh / 4);
+      const int c4 = (it % (kDh / 4)) * 4;
+      const int r = rt * kRowsCta + lr;
+      if (r >= p.R) continue;
+      float2 ml[kMaxCluster];
+      float4 ov4[kMaxCluster];
+#pragma unroll
+      for (int j = 0; j < kMaxCluster; ++j) {
+        ml[j] = j < n ? xml_p[j][lr] : make_float2(-CUDART_INF_F, 0.f);
+        ov4[j] = j < n ? *reinterpret_cast<const float4*>(xo_p[j] + lr * kXoStride + c4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int j = 0; j < kMaxCluster; ++j) M = fmaxf(M, ml[j].x);
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < kMaxCluster; ++j) {
+        const float w = ml[j].x == -CUDART_INF_F ? 0.f : fast_exp2(ml[j].x - M);
+        L = fmaf(w, ml[j].y, L);
+        acc.x = fmaf(w, ov4[j].x, acc.x);
+        acc.y = fmaf(w, ov4[j].y, acc.y);
+        acc.z = fmaf(w, ov4[j].z, acc.z);
+        acc.w = fmaf(w, ov4[j].w, acc.w);
+      }
+      const float inv = 1.f / L;
+      const int i = r / p.G, hh = r - i * p.G;
+      __nv_bfloat16* dst = p.o + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + c4;
+      uint2 w2;
+      w2.x = pack_bf16(acc.x * inv, acc.y * inv);
+      w2.y = pack_bf16(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(dst) = w2;
+    }
+    cluster.sync();   // the peers have finished reading this CTA's rows
   }
 
   tc_fence_before();
@@ -501,8 +589,28 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.R = ap.R;
   p.chunk = ap.chunk;
   p.nsplit = ap.nsplit;
+  p.cluster = ap.cluster;
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
+  if (ap.cluster > 1) {
+    // the splits of a (row tile, plane) as one cluster: no partials, no combine kernel
+    if (ap.cluster != ap.nsplit || ap.cluster > 8) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = kAttnSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)ap.cluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmK, tmV, p);
+  }
   cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kAttnSmem, st, tmK, tmV, p);
   if (e != cudaSuccess || ap.nsplit == 1) return e;
   const int rows_per_block = 8;
@@ -510,6 +618,35 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   return launch_pdl(attn_combine_kernel, g2, dim3(32 * rows_per_block), 0, st,
                     (const float*)opart, (const float2*)ml, (__nv_bfloat16*)o, lens, done,
                     n_active, md.H, md.Hkv, ap.G, ap.C, ap.R, ap.chunk, ap.nsplit);
+}
+
+int attn_cluster_capacity(int n) {
+  // clusters of n attention CTAs (one SM each) that can be resident at once
+  static int cap[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  if (n < 2 || n > 8) return 0;
+  if (cap[n] >= 0) return cap[n];
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kAttnSmem) != cudaSuccess) {
+    cudaGetLastError();
+    return cap[n] = 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n, 1, 1);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kAttnSmem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)n;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int num = 0;
+  if (cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    num = 0;
+  }
+  return cap[n] = num;
 }
 
 cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,

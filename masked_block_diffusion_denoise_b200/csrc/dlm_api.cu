@@ -85,6 +85,7 @@ struct dlm_ctx {
   std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> maps;
   CUtensorMap tmK{}, tmV{};
   std::vector<GraphEntry> graphs;
+  std::map<std::vector<int>, AttnPlan> plans;   // attention split plans
   cudaStream_t cap = nullptr;
   std::string msg;
   int launches = 0;
@@ -215,15 +216,25 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
     p.BN = 256;
     return p;
   }
+  // one M tile: weight-read bound; split K over as many CTAs as fit in one
+  // wave (a second wave of short CTAs costs more pipeline fill than it saves)
   p.BN = 128;
-  p.splits = pick_splits(cdiv(N, p.BN), cdiv(K, 64), ctx->num_sms, 16);
+  const int tiles = cdiv(N, p.BN);
+  p.splits = tiles >= ctx->num_sms
+                 ? 1
+                 : std::max(1, std::min({16, ctx->num_sms / tiles, std::max(1, cdiv(K, 64) / 2)}));
   return p;
 }
 
-// Split plan of the attention: every chunk size (whole 128-key tiles) is
-// costed by list-scheduling the CTAs in launch order (split fastest, one CTA
-// per SM) with a per-tile time, a per-CTA fixed time and the combine's cost
-// per partial; ragged prefixes (lens, host) are taken as they are.
+// Split plan of the attention.  For every split count (with the smallest
+// chunk of whole 128-key tiles that gives it) the CTAs are list-scheduled in
+// launch order (split fastest) onto the SMs with a per-CTA and a per-tile
+// time; ragged prefixes (lens, host) are taken as they are.  Up to 8 splits
+// may combine inside a thread-block cluster (an exchange cost per CTA) when
+// the whole grid fits in one wave of resident clusters; otherwise splits
+// write partials for the combine kernel (a write cost per CTA, the kernel, a
+// cost per partial).  Costs in microseconds, from B200 measurements: a tile
+// takes ~1.2 us in a lone CTA and ~1.7 us when every SM streams K/V.
 AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int max_len_all) {
   AttnPlan a{};
   a.B = B;
@@ -235,13 +246,32 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
   const int sms = std::min(std::max(ctx->num_sms, 1), 1024);
   const int max_keys = max_len_all + C;
   const int max_tiles = cdiv(max_keys, 128);
-  const double t_tile = 2.0, t_cta = 2.0, t_comb = 3.0, t_part = 0.02;   // microseconds
+  const double t_tile = 1.5, t_cta = 3.0, t_xchg = 1.5, t_pw = 1.5, t_comb = 4.0, t_part = 0.03;
   double best = -1.0;
-  double sm_free[1024];   // no heap: this also runs inside dlm_attention_noalloc
+  double sm_free[1024];   // no heap allocation: this also runs inside dlm_attention_noalloc
+  // diagnostic switch: DLM_ATTN_CLUSTER=0 keeps every split plan on the
+  // partials + combine kernel path
+  const char* cl_env = std::getenv("DLM_ATTN_CLUSTER");
+  const bool cluster_ok = cl_env == nullptr || std::strcmp(cl_env, "0") != 0;
+  // diagnostic switch: DLM_ATTN_TILES=k plans only chunks of k key tiles
+  const char* ct_env = std::getenv("DLM_ATTN_TILES");
+  const int only_ct = ct_env != nullptr ? std::atoi(ct_env) : 0;
+  int last_nsplit = 0;
   for (int ct = 1; ct <= max_tiles; ++ct) {
+    if (only_ct > 0 && ct != std::min(only_ct, max_tiles)) continue;
     const int chunk = ct * 128;
     const int nsplit = cdiv(max_keys, chunk);
-    if (nsplit > 64) continue;
+    if (nsplit > 64) continue;   // the combine kernel holds up to 64 splits
+    if (nsplit == last_nsplit) continue;   // a larger chunk for the same split count
+    last_nsplit = nsplit;
+    const long ctas = (long)B * Hkv * a.rtiles * nsplit;
+    int cl = 1;
+    if (nsplit > 1 && nsplit <= 8 && cluster_ok) {
+      const int cap = attn_cluster_capacity(nsplit);
+      if (cap > 0 && ctas <= (long)cap * nsplit) cl = nsplit;
+    }
+    const double per_cta = t_cta + (cl > 1 ? t_xchg : (nsplit > 1 ? t_pw : 0.0));
+    // SMs as a min-heap of finish times (negated for the max-heap functions)
     std::fill(sm_free, sm_free + sms, 0.0);
     long partials = 0;
     double makespan = 0.0;
@@ -250,23 +280,39 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
       for (int rt = 0; rt < a.rtiles; ++rt) {
         for (int sp = 0; sp < nsplit; ++sp) {
           const int k0 = sp * chunk;
-          if (k0 >= keys) continue;   // exits at once
-          const int tiles = cdiv(std::min(chunk, keys - k0), 128);
-          double* it = std::min_element(sm_free, sm_free + sms);
-          *it += t_cta + tiles * t_tile;
-          makespan = std::max(makespan, *it);
+          if (k0 >= keys && cl == 1) continue;   // exits at once
+          const int tiles = k0 < keys ? cdiv(std::min(chunk, keys - k0), 128) : 0;
+          std::pop_heap(sm_free, sm_free + sms);   // earliest free SM to the back
+          sm_free[sms - 1] -= per_cta + tiles * t_tile;
+          makespan = std::max(makespan, -sm_free[sms - 1]);
+          std::push_heap(sm_free, sm_free + sms);
           ++partials;
         }
       }
     }
-    const double cost = makespan + (nsplit > 1 ? t_comb + t_part * partials : 0.0);
+    const double cost = makespan + (nsplit > 1 && cl == 1 ? t_comb + t_part * partials : 0.0);
     if (best < 0.0 || cost < best - 1e-9) {
       best = cost;
       a.chunk = chunk;
       a.nsplit = nsplit;
+      a.cluster = cl;
     }
   }
   return a;
+}
+
+// plan_attention, remembered per (batch, canvas, prefix lengths)
+AttnPlan plan_attention_cached(dlm_ctx* ctx, int B, int C, int max_len_all) {
+  std::vector<int> key(ctx->lens_h.begin(), ctx->lens_h.begin() + B);
+  key.push_back(B);
+  key.push_back(C);
+  key.push_back(max_len_all);
+  auto it = ctx->plans.find(key);
+  if (it != ctx->plans.end()) return it->second;
+  const AttnPlan ap = plan_attention(ctx, B, C, ctx->lens_h.data(), max_len_all);
+  if (ctx->plans.size() > 256) ctx->plans.clear();
+  ctx->plans.emplace(std::move(key), ap);
+  return ap;
 }
 
 int max_len(const dlm_ctx* ctx, int batch) {
@@ -276,7 +322,7 @@ int max_len(const dlm_ctx* ctx, int batch) {
 }
 
 int ensure_attn_scratch(dlm_ctx* ctx, const AttnPlan& ap) {
-  if (ap.nsplit <= 1) return DLM_OK;
+  if (ap.nsplit <= 1 || ap.cluster > 1) return DLM_OK;
   const size_t slots = (size_t)ap.B * ctx->md.Hkv * ap.nsplit * ap.R;
   if (slots * ctx->md.Dh > ctx->opart_floats) {
     if (ctx->opart) {
@@ -384,7 +430,8 @@ int run_gemm(dlm_ctx* ctx, const void* A, const void* B, int Brows, const GemmPl
   cudaError_t e;
   if (ctx->bf16) {
     const bool u8 = plan.f8 != 0;
-    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K, 128, u8);
+    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K,
+                                  (uint32_t)gemm_tc_a_rows(plan.M), u8);
     const CUtensorMap* tb =
         map2d(ctx, B, (uint64_t)Brows, (uint64_t)plan.K, (uint32_t)plan.BN, u8);
     if (ta == nullptr || tb == nullptr)
@@ -474,7 +521,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
   if (ctx->bf16) {
     e = attention_bf16(md, ap, ctx->tmK, ctx->tmV, ctx->q, ctx->o, ctx->opart, ctx->ml,
                        ctx->lens_d, c->done, ctx->n_active, ctx->err, st);
-    ctx->launches += ap.nsplit > 1 ? 2 : 1;
+    ctx->launches += ap.nsplit > 1 && ap.cluster <= 1 ? 2 : 1;
   } else {
     e = attention_f32(md, batch, C, (const float*)ctx->q, (const float*)ctx->kc,
                       (const float*)ctx->vc, (float*)ctx->o, ctx->lens_d, c->done,
@@ -812,7 +859,7 @@ int dlm_denoise_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
   if (int rc = check_canvas(ctx, c, p)) return rc;
-  AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
+  AttnPlan ap = plan_attention_cached(ctx, batch, p->canvas, max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
   ctx->launches = 0;
@@ -825,7 +872,7 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   ctx->msg.clear();
   if (int rc = check_params(ctx, p, batch)) return rc;
   if (int rc = check_canvas(ctx, c, p)) return rc;
-  AttnPlan ap = plan_attention(ctx, batch, p->canvas, ctx->lens_h.data(), max_len(ctx, batch));
+  AttnPlan ap = plan_attention_cached(ctx, batch, p->canvas, max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
   // the graph bakes in pointers, sizes, parameters and the attention plan
@@ -937,7 +984,7 @@ int dlm_generate(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     pk.seed = p->seed + (unsigned long long)k;   // block k's random streams
     CK(canvas_init(ctx->md, batch, C, pk.corruption, pk.seed, c->tokens, c->committed, c->step,
                    c->done, c->eos_pos, c->prev_cand, c->stable, st));
-    AttnPlan ap = plan_attention(ctx, batch, C, ctx->lens_h.data(), max_len(ctx, batch));
+    AttnPlan ap = plan_attention_cached(ctx, batch, C, max_len(ctx, batch));
     if (ctx->bf16)
       if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
     ctx->launches = 0;
@@ -1137,7 +1184,7 @@ int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cach
   cudaDeviceGetAttribute(&plan_ctx.num_sms, cudaDevAttrMultiProcessorCount, dev);
   const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, nullptr, max_len);
   const long slots = (long)batch * n_kv_heads * ap.nsplit * ap.R;
-  if (ap.nsplit > 1 && slots > kNoAllocSlots) {
+  if (ap.nsplit > 1 && ap.cluster <= 1 && slots > kNoAllocSlots) {
     g_create_error = "attention_noalloc: the split plan needs " + std::to_string(slots) +
                      " partial row slots; the static array holds " +
                      std::to_string(kNoAllocSlots);

@@ -36,20 +36,40 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;   // one 128-byte swizzle atom of bf16 per row
 
+// Shared memory: a ring of `stages` stages, each [B tile: BN rows x 128 B]
+// [A tile: a_rows x 128 B], then a pad, the barriers and the row-state
+// exchange.  With one M tile the A box holds only the rows in use (rounded up
+// to 8); the MMA still reads 128 A rows, and rows past a_rows -- whatever
+// follows in shared memory -- feed only accumulator rows the epilogue never
+// reads.  The pad of (128 - a_rows) x 128 bytes keeps those reads of the last
+// stage inside the allocation.  Smaller A tiles leave room for more stages
+// of weights in flight.
 template <int BN>
 struct TcCfg {
-  static constexpr int kStages = (BN == 128) ? 6 : 4;
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kMaxStages = 16;
+  static constexpr int kBBytes = BN * 128;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kSmem =
-      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + 128 * 32 /*row states*/;
+  static constexpr int kBarBytes = 512;       // mbarriers, TMEM slot, abort flag
+  static constexpr int kXchBytes = 128 * 32;  // row states of the EPI_LM hand-over
+  static constexpr int kSmem = 232448;        // the opt-in maximum per block
 };
+
+__host__ __device__ constexpr int tc_stage_bytes(int BN, int a_rows) { return (BN + a_rows) * 128; }
+__host__ __device__ constexpr int tc_bar_offset(int BN, int a_rows, int stages) {
+  return stages * tc_stage_bytes(BN, a_rows) + (128 - a_rows) * 128;
+}
+template <int BN>
+constexpr int tc_stages(int a_rows) {
+  using Cfg = TcCfg<BN>;
+  const int room = Cfg::kSmem - 1024 - Cfg::kBarBytes - Cfg::kXchBytes - (128 - a_rows) * 128;
+  const int n = room / tc_stage_bytes(BN, a_rows);
+  return n < Cfg::kMaxStages ? n : Cfg::kMaxStages;
+}
 
 struct TcParams {
   int M, N, K;
   int m_tiles, n_tiles, splits, units, kblocks;
+  int a_rows, stages;    // A box rows (multiple of 8, <= 128), ring stages
   float* out;
   LmPart* part;
   LmEpi epi;
@@ -121,9 +141,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kStages * Cfg::kStageBytes);
-  uint64_t* empty = full + Cfg::kStages;
-  uint64_t* tfull = empty + Cfg::kStages;
+  const int stages = p.stages;
+  const int stage_bytes = tc_stage_bytes(BN, p.a_rows);
+  const uint32_t a_bytes = (uint32_t)p.a_rows * 128u;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_bar_offset(BN, p.a_rows, stages));
+  uint64_t* empty = full + Cfg::kMaxStages;
+  uint64_t* tfull = empty + Cfg::kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -133,7 +156,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < Cfg::kStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -164,12 +187,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     pol_stream = l2_evict_first_policy();
     int m0, n0, kb0, kb1, sp0;
     if (get_unit<EPI>(p, 0, m0, n0, kb0, kb1, sp0)) {
-      pre = min(Cfg::kStages, kb1 - kb0);
+      pre = min(stages, kb1 - kb0);
       for (int s = 0; s < pre; ++s) {
         const int kb = kb0 + s;
         mbar_expect_tx(&full[s], Cfg::kBBytes);
-        tma_load_2d_hint(smem + s * Cfg::kStageBytes + Cfg::kABytes, &tmB, &full[s], kb * kBKe,
-                         n0 * BN, pol_stream);
+        tma_load_2d_hint(smem + s * stage_bytes, &tmB, &full[s], kb * kBKe, n0 * BN, pol_stream);
       }
     }
   }
@@ -198,19 +220,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * Cfg::kStageBytes;
-          uint8_t* sb = sa + Cfg::kABytes;
+          uint8_t* sb = smem + stage * stage_bytes;
+          uint8_t* sa = sb + Cfg::kBBytes;
           if (issued < pre) {
             // this stage's B tile is already in flight
-            mbar_arrive_expect_tx(&full[stage], Cfg::kABytes);
+            mbar_arrive_expect_tx(&full[stage], a_bytes);
             tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
           } else {
-            mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+            mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
             tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
             tma_load_2d_hint(sb, &tmB, &full[stage], kb * kBKe, n * BN, pol_stream);
           }
           ++issued;
-          if (++stage == Cfg::kStages) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -224,9 +246,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int s = 0; s < pre; ++s) mbar_wait_bounded(&full[s], 0u, nullptr);
         } else {
           int st = stage, ph = phase;
-          for (int i = 0; i < Cfg::kStages && i < issued; ++i) {
+          for (int i = 0; i < stages && i < issued; ++i) {
             if (--st < 0) {
-              st = Cfg::kStages - 1;
+              st = stages - 1;
               ph ^= 1;
             }
             mbar_wait_bounded(&full[st], (uint32_t)ph, nullptr);
@@ -254,8 +276,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
-          const uint32_t sb = sa + Cfg::kABytes;
+          const uint32_t sb = smem_u32(smem + stage * stage_bytes);
+          const uint32_t sa = sb + Cfg::kBBytes;
           // four instructions of 32 bytes of K per 128-byte k-block
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -267,7 +289,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         (kb > kb0 || k > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
-          if (++stage == Cfg::kStages) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
@@ -453,7 +475,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if constexpr (EPI == EPI_LM) {
       // the two warpgroups' states of a row: warpgroup 1 hands its state over
       // through shared memory, warpgroup 0 combines (fixed order) and stores
-      RowState* xch = reinterpret_cast<RowState*>(reinterpret_cast<uint8_t*>(full) + 256);
+      RowState* xch = reinterpret_cast<RowState*>(reinterpret_cast<uint8_t*>(full) + Cfg::kBarBytes);
       const int lr = quad * 32 + lane;
       if (wg == 1) xch[lr] = rs;
       asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -516,6 +538,8 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   const int kbe = plan.f8 ? 2 * kBK : kBK;   // elements per k-block
   p.kblocks = (plan.K + kbe - 1) / kbe;
   p.units = p.m_tiles * p.n_tiles * p.splits;
+  p.a_rows = gemm_tc_a_rows(plan.M);
+  p.stages = plan.BN == 128 ? tc_stages<128>(p.a_rows) : tc_stages<256>(p.a_rows);
   p.out = io.out;
   p.part = io.part;
   p.epi = io.epi;
@@ -547,6 +571,8 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
 }
 
 int gemm_tc_smem_bytes(int BN) { return BN == 128 ? TcCfg<128>::kSmem : TcCfg<256>::kSmem; }
+
+int gemm_tc_a_rows(int M) { return M >= kBM ? kBM : ((M + 7) / 8) * 8; }
 
 int gemm_tc_lm_partials(const GemmPlan& plan, int num_sms) {
   const int m_tiles = (plan.M + kBM - 1) / kBM;

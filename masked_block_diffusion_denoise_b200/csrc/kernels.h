@@ -50,6 +50,8 @@ struct GemmIO {
 cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPlan& plan,
                     const GemmIO& io, int num_sms, cudaStream_t st);
 int gemm_tc_smem_bytes(int BN);
+// rows of the A (activation) box: all rows in use, rounded up to 8, at most 128
+int gemm_tc_a_rows(int M);
 // LM partials per row written by the EPI_LM launch of `plan` (one per CTA slot)
 int gemm_tc_lm_partials(const GemmPlan& plan, int num_sms);
 
@@ -108,8 +110,12 @@ cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, fl
 // ---- attention.cu ------------------------------------------------------------
 struct AttnPlan {
   int B, C, G, R, rtiles;   // G = H / Hkv, R = G * C query rows per (seq, kv head)
-  int chunk, nsplit;        // keys per split (multiple of 64), splits per (seq, kv head)
+  int chunk, nsplit;        // keys per split (multiple of 128), splits per (seq, kv head)
+  int cluster = 1;          // nsplit (<= 8) when the splits combine inside a cluster
 };
+
+// clusters of n (2..8) attention CTAs that fit on the device at once (0: none)
+int attn_cluster_capacity(int n);
 
 // bf16: TMA-fed mma.sync flash attention over [prefix ; canvas] keys, split-KV
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,

@@ -14,48 +14,79 @@
 namespace dlm {
 namespace {
 
-// combine the n_part partials of one row (a warp) into cand / conf / entropy
+// combine the n_part partials of one row (a warp) into cand / conf / entropy:
+//   M = max_j m_j,  S = sum_j s_j e^{m_j - M},  T = sum_j e^{m_j - M} (t_j + s_j (m_j - M)),
+//   winner = the partial with the largest g (lowest index on ties).
+// The partials are taken in chunks of 32 * kU: a chunk's maximum is a warp
+// maximum, after which every lane's terms are independent of one another (no
+// chain of pairwise merges); the lane sums and the winner meet in fixed
+// butterflies, so the result does not depend on timing.
 __device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, int32_t* cand,
                            float* conf, float* ent) {
-  RowState acc;
-  rs_init(acc);
-  // issue all loads of a batch before combining (independent L2 reads)
-  constexpr int kU = 8;
+  constexpr int kU = 5;   // one chunk covers one partial per SM of a 148-SM part
+  float M = -CUDART_INF_F, s_l = 0.f, t_l = 0.f;
+  float g_b = -CUDART_INF_F, zw_b = -CUDART_INF_F;
+  int idx_b = 0x7fffffff;
   for (int j0 = 0; j0 < n_part; j0 += 32 * kU) {
     LmPart q[kU];
+    bool ok[kU];
+    float mloc = -CUDART_INF_F;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int j = j0 + lane + 32 * u;
-      if (j < n_part) q[u] = pr[j];
+      ok[u] = j < n_part;
+      if (ok[u]) {
+        q[u] = pr[j];
+        ok[u] = q[u].m != -CUDART_INF_F;   // a tile with every column excluded
+      }
+      if (ok[u]) mloc = fmaxf(mloc, q[u].m);
     }
 #pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, off));
+    const float Mn = fmaxf(M, mloc);
+    if (Mn == -CUDART_INF_F) continue;   // warp-uniform
+    if (M != -CUDART_INF_F && Mn > M) {
+      const float a = __expf(M - Mn);
+      t_l = (t_l + s_l * (M - Mn)) * a;
+      s_l *= a;
+    }
+    M = Mn;
+#pragma unroll
     for (int u = 0; u < kU; ++u) {
-      if (j0 + lane + 32 * u < n_part) {
-        RowState x{q[u].m, q[u].s, q[u].t, q[u].g, q[u].zw, q[u].idx};
-        acc = rs_combine(acc, x);
+      if (ok[u]) {
+        const float d = q[u].m - M;
+        const float w = __expf(d);
+        s_l = fmaf(q[u].s, w, s_l);
+        t_l = fmaf(w, fmaf(q[u].s, d, q[u].t), t_l);
+        const bool better = q[u].g > g_b || (q[u].g == g_b && q[u].idx < idx_b);
+        g_b = better ? q[u].g : g_b;
+        zw_b = better ? q[u].zw : zw_b;
+        idx_b = better ? q[u].idx : idx_b;
       }
     }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    RowState o;
-    o.m = __shfl_xor_sync(0xffffffffu, acc.m, off);
-    o.s = __shfl_xor_sync(0xffffffffu, acc.s, off);
-    o.t = __shfl_xor_sync(0xffffffffu, acc.t, off);
-    o.g = __shfl_xor_sync(0xffffffffu, acc.g, off);
-    o.zw = __shfl_xor_sync(0xffffffffu, acc.zw, off);
-    o.idx = __shfl_xor_sync(0xffffffffu, acc.idx, off);
-    acc = rs_combine(acc, o);   // symmetric: every lane ends with the same value
+    s_l += __shfl_xor_sync(0xffffffffu, s_l, off);
+    t_l += __shfl_xor_sync(0xffffffffu, t_l, off);
+    const float g_o = __shfl_xor_sync(0xffffffffu, g_b, off);
+    const float zw_o = __shfl_xor_sync(0xffffffffu, zw_b, off);
+    const int idx_o = __shfl_xor_sync(0xffffffffu, idx_b, off);
+    const bool take = g_o > g_b || (g_o == g_b && idx_o < idx_b);
+    g_b = take ? g_o : g_b;
+    zw_b = take ? zw_o : zw_b;
+    idx_b = take ? idx_o : idx_b;
   }
   if (lane == 0) {
-    if (acc.idx == 0x7fffffff || !(acc.s > 0.f)) {
+    if (idx_b == 0x7fffffff || !(s_l > 0.f)) {
       *cand = 0;
       *conf = 0.f;
       *ent = 0.f;
     } else {
-      *cand = acc.idx;
-      *conf = expf(acc.zw - acc.m) / acc.s;
-      *ent = logf(acc.s) - acc.t / acc.s;
+      *cand = idx_b;
+      *conf = expf(zw_b - M) / s_l;
+      *ent = logf(s_l) - t_l / s_l;
     }
   }
 }
@@ -212,18 +243,37 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   const int nU = __syncthreads_count(open);
   const int nthr = __syncthreads_count(open && !a.eb && conf[base + i] >= a.threshold);
 
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      const int ixj = i ^ j;
-      if (i < P && ixj > i) {
-        const unsigned long long x = keys[i], y = keys[ixj];
-        const bool up = (i & k) == 0;
-        if ((x > y) == up) {
-          keys[i] = y;
-          keys[ixj] = x;
+  if (P == 32) {
+    // up to 32 keys: a bitonic network inside warp 0, in registers (the keys
+    // are unique -- position in the low word -- so any sorting network gives
+    // the same order)
+    if (i < 32) {
+      unsigned long long x = keys[i];
+      for (int k = 2; k <= 32; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+          const bool up = (i & k) == 0;
+          const bool low = (i & j) == 0;
+          x = (low == up) ? (x < y ? x : y) : (x < y ? y : x);
         }
       }
-      __syncthreads();
+      keys[i] = x;
+    }
+    __syncthreads();
+  } else {
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const int ixj = i ^ j;
+        if (i < P && ixj > i) {
+          const unsigned long long x = keys[i], y = keys[ixj];
+          const bool up = (i & k) == 0;
+          if ((x > y) == up) {
+            keys[i] = y;
+            keys[ixj] = x;
+          }
+        }
+        __syncthreads();
+      }
     }
   }
 
@@ -299,7 +349,7 @@ cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed
   int P = 32;
   while (P < a.C) P <<= 1;
   if (P > kMaxC) return cudaErrorInvalidValue;
-  if (part != nullptr && P < 512) P = 512;   // enough warps for the row reductions
+  if (part != nullptr) P = 1024;   // 32 warps for the row reductions
   return launch_pdl(commit_kernel, dim3(a.B), dim3(P), 0, st, a, tokens, committed, step, done,
                     eos_pos, prev_cand, stable, part, n_part, cand, conf, ent, stats, n_active, err);
 }

@@ -188,6 +188,24 @@ def test_small_block_stagewise(name):
         sess.close()
 
 
+@pytest.mark.parametrize("cluster", ["1", "0"])
+def test_attention_split_paths(cluster, monkeypatch):
+    """The split-KV attention both ways: splits combined inside a thread-block
+    cluster, and splits written as partials for the combine kernel
+    (DLM_ATTN_CLUSTER=0); ragged prefixes leave some splits without keys."""
+    monkeypatch.setenv("DLM_ATTN_CLUSTER", cluster)
+    wl = W.small_workload("split_paths", n_heads=8, n_kv_heads=2, batch=3, canvas=16, steps=2,
+                          quota=0, prefix_len=(20, 1500), prefix_cap=1600, seed=6)
+    sess, om, _ = make_pair(wl)
+    try:
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        sess.init(cv, p_lib)
+        check_one_step(sess, om, wl, cv, p_lib, p_or)
+    finally:
+        sess.close()
+
+
 def test_tiny_fp32_reference_config():
     """The tiny fp32 configuration: batch 1, d 256, 4 heads of 64, vocab 4096,
     prefix of 128 random ids appended through the clean pass, canvas 32,
