@@ -141,17 +141,32 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   pdl_wait_then_release();
-  // query tile -> shared memory, two 64-column halves, 128-byte swizzle
-  for (int idx = tid; idx < kRowsCta * 16; idx += blockDim.x) {
-    const int lr = idx >> 4, ch = idx & 15;
-    const int r = rt * kRowsCta + lr;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (r < p.R) {
-      const int i = r / p.G, hh = r - i * p.G;
-      val = *reinterpret_cast<const uint4*>(
-          p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8);
+  // query tile -> shared memory, two 64-column halves, 128-byte swizzle; every
+  // load of a thread is issued before the first store (one L2 round trip)
+  {
+    constexpr int kQChunks = kRowsCta * 16;                  // 16-byte chunks
+    constexpr int kPer = (kQChunks + 191) / 192;             // per thread at 192 threads
+    uint4 val[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = tid + u * 192;
+      const int lr = idx >> 4, ch = idx & 15;
+      const int r = rt * kRowsCta + lr;
+      val[u] = make_uint4(0, 0, 0, 0);
+      if (idx < kQChunks && r < p.R) {
+        const int i = r / p.G, hh = r - i * p.G;
+        val[u] = *reinterpret_cast<const uint4*>(
+            p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8);
+      }
     }
-    *reinterpret_cast<uint4*>(qs + (ch >> 3) * kHalf + sw128_off(lr, ch & 7)) = val;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = tid + u * 192;
+      if (idx < kQChunks) {
+        const int lr = idx >> 4, ch = idx & 15;
+        *reinterpret_cast<uint4*>(qs + (ch >> 3) * kHalf + sw128_off(lr, ch & 7)) = val[u];
+      }
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
