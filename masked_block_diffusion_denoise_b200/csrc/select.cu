@@ -22,7 +22,8 @@ namespace {
 // chain of pairwise merges); the lane sums and the winner meet in fixed
 // butterflies, so the result does not depend on timing.
 __device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, int32_t* cand,
-                           float* conf, float* ent) {
+                           float* conf, float* ent, int32_t* cand_sm, float* conf_sm,
+                           float* ent_sm) {
   constexpr int kU = 5;   // one chunk covers one partial per SM of a 148-SM part
   float M = -CUDART_INF_F, s_l = 0.f, t_l = 0.f;
   float g_b = -CUDART_INF_F, zw_b = -CUDART_INF_F;
@@ -79,15 +80,19 @@ __device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, 
     idx_b = take ? idx_o : idx_b;
   }
   if (lane == 0) {
-    if (idx_b == 0x7fffffff || !(s_l > 0.f)) {
-      *cand = 0;
-      *conf = 0.f;
-      *ent = 0.f;
-    } else {
-      *cand = idx_b;
-      *conf = expf(zw_b - M) / s_l;
-      *ent = logf(s_l) - t_l / s_l;
+    int32_t c = 0;
+    float f = 0.f, h = 0.f;
+    if (idx_b != 0x7fffffff && s_l > 0.f) {
+      c = idx_b;
+      f = expf(zw_b - M) / s_l;
+      h = logf(s_l) - t_l / s_l;
     }
+    *cand = c;
+    *conf = f;
+    *ent = h;
+    *cand_sm = c;   // the block's own copy for the selection
+    *conf_sm = f;
+    *ent_sm = h;
   }
 }
 
@@ -133,24 +138,30 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   if (n_active != nullptr && *n_active == 0) return;
   const int b = blockIdx.x;
   if (done[b]) return;
-  if (part != nullptr) {
-    // a6: the cross-tile reduction of this canvas's rows, one warp per row
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int i = warp; i < a.C; i += nw) {
-      const size_t row = (size_t)b * a.C + i;
-      reduce_row(part + row * n_part, n_part, lane, cand + row, conf + row, ent + row);
-    }
-    __syncthreads();
-  }
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
   __shared__ uint8_t com[kMaxC];
+  __shared__ int32_t cand_s[kMaxC];   // this canvas's candidates, confidences, entropies
+  __shared__ float conf_s[kMaxC], ent_s[kMaxC];
   __shared__ int e_s, k_s, krule_s;
   const int i = threadIdx.x;
   const int C = a.C;
   int P = 32;               // keys sorted: the next power of two >= C
   while (P < C) P <<= 1;
   const size_t base = (size_t)b * C;
+  if (part != nullptr) {
+    // a6: the cross-tile reduction of this canvas's rows, one warp per row
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int r = warp; r < C; r += nw) {
+      const size_t row = base + r;
+      reduce_row(part + row * n_part, n_part, lane, cand + row, conf + row, ent + row,
+                 cand_s + r, conf_s + r, ent_s + r);
+    }
+  } else if (i < C) {
+    cand_s[i] = cand[base + i];
+    conf_s[i] = conf[base + i];
+    ent_s[i] = ent[base + i];
+  }
   const int s = step[b];
   if (i < C) {
     tok[i] = tokens[base + i];
@@ -169,8 +180,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     const int lim = e0 < 0 ? C : e0;
     bool ed = false;
     if (i < lim && com[i]) {
-      int c = cand[base + i];
-      if (c != tok[i] && conf[base + i] + 0.0f >= a.edit_thr) {
+      int c = cand_s[i];
+      if (c != tok[i] && conf_s[i] + 0.0f >= a.edit_thr) {
         if (c < 0 || c >= a.V) {
           raise_error(err, DLM_EBOUNDS);
           c = 0;
@@ -188,12 +199,12 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     // mean entropy (float32, summed in position order) below the bound the
     // canvas freezes: every open position commits its candidate
     __shared__ int freeze_s;
-    const bool same = (i >= C) || (cand[base + i] == prev_cand[base + i]);
+    const bool same = (i >= C) || (cand_s[i] == prev_cand[base + i]);
     const int all_same = __syncthreads_and(same);
-    if (i < C) prev_cand[base + i] = cand[base + i];
+    if (i < C) prev_cand[base + i] = cand_s[i];
     if (i == 0) {
       float total = 0.f;
-      for (int j = 0; j < C; ++j) total = __fadd_rn(total, ent[base + j] + 0.0f);
+      for (int j = 0; j < C; ++j) total = __fadd_rn(total, ent_s[j] + 0.0f);
       const float mean = __fdiv_rn(total, (float)C);
       const int st = all_same ? stable[b] + 1 : 0;
       stable[b] = st;
@@ -203,7 +214,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     if (freeze_s) {
       const bool opened = i < C && !com[i];
       if (opened) {
-        int c = cand[base + i];
+        int c = cand_s[i];
         if (c < 0 || c >= a.V) {
           raise_error(err, DLM_EBOUNDS);
           c = 0;
@@ -236,12 +247,12 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   const bool open = (i < C) && !com[i];
   unsigned long long key = ~0ull;
   if (open) {
-    const uint32_t hi = a.eb ? ordered_bits(ent[base + i]) : ~ordered_bits(conf[base + i]);
+    const uint32_t hi = a.eb ? ordered_bits(ent_s[i]) : ~ordered_bits(conf_s[i]);
     key = ((unsigned long long)hi << 32) | (unsigned)i;
   }
   if (i < P) keys[i] = key;
   const int nU = __syncthreads_count(open);
-  const int nthr = __syncthreads_count(open && !a.eb && conf[base + i] >= a.threshold);
+  const int nthr = __syncthreads_count(open && !a.eb && conf_s[i] >= a.threshold);
 
   if (P == 32) {
     // up to 32 keys: a bitonic network inside warp 0, in registers (the keys
@@ -284,7 +295,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
       float run = 0.f;
       for (int j = 0; j < nU; ++j) {
         const int pos = (int)(keys[j] & 0xffffffffu);
-        run = __fadd_rn(run, ent[base + pos] + 0.0f);
+        run = __fadd_rn(run, ent_s[pos] + 0.0f);
         if (run <= a.bound)
           ++k;
         else
@@ -303,7 +314,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   const int k = k_s;
   if (i < k) {
     const int pos = (int)(keys[i] & 0xffffffffu);
-    int c = cand[base + pos];
+    int c = cand_s[pos];
     if (c < 0 || c >= a.V) {
       raise_error(err, DLM_EBOUNDS);
       c = 0;

@@ -153,3 +153,45 @@ def test_generate_rejects_overflow():
         assert dlm_kv_length(sess.ctx, 0) == wl.prefix_len[1]
     finally:
         sess.close()
+
+
+@pytest.mark.parametrize("lm_fp8", [False, True])
+def test_generate_bf16_every_option(lm_fp8):
+    """Two blocks with uniform corruption, adaptive stopping and token editing
+    together (bf16, and with the e4m3 LM head): every position of every block
+    is committed, no id is out of range, the counters add up, and the clean
+    passes cached each block's own tokens."""
+    base = W.small_workload("gen_all", batch=2, canvas=32, steps=5, quota=0, corruption="uniform",
+                            prefix_len=(60, 200), lm_fp8=lm_fp8, seed=8)
+    wl = base.replace(prefix_cap=base.prefix_len[1] + 2 * base.canvas)
+    sess, om, _ = make_pair(wl)
+    try:
+        C, B, sh = wl.canvas, wl.batch, wl.shape
+        L0 = [om.kv_len(b) for b in range(B)]
+        p = lib_params(wl, stability_steps=0, stop_entropy=0.05, editing=1,
+                       editing_threshold=0.0)
+        cv = sess.new_canvas(B, C)
+        out, n = sess.generate(cv, p, 2, eos_early_stop=False)
+        sess.check()
+        out = out.cpu().numpy()
+        st = cv.numpy()
+        assert n == 2 and ((out >= 0) & (out < sh.vocab)).all()
+        assert st["committed"].all() and st["done"].all()
+        stats = st["stats"]
+        # per block every position is committed once: by the sampler, a freeze or the EOS fill
+        for b in range(B):
+            assert stats[b][1] + stats[b][4] + stats[b][3] == 2 * C
+            assert stats[b][0] <= 2 * wl.steps
+        Lcap = sess.max_prefix + sess.max_canvas
+        kc = sess.buffer(DLM_BUF_K_CACHE, (B, sh.n_kv_heads, Lcap, sh.head_dim), torch.bfloat16)
+        half = sh.head_dim // 2
+        for b in range(B):
+            assert dlm_kv_length(sess.ctx, b) == L0[b] + 2 * C
+            om.kv_append_tokens(b, out[b])
+            xe = om.embed(out[b])
+            tk = abs_terms(xe, om.w_k).reshape(-1, sh.n_kv_heads, sh.head_dim).transpose(1, 0, 2)
+            tk = np.concatenate([tk[..., :half] + tk[..., half:]] * 2, axis=-1)
+            assert_storage_close(to64(kc[b, :, L0[b]:L0[b] + 2 * C]), om.k_cache[b][:, L0[b]:],
+                                 "bf16", what="K", terms=tk)
+    finally:
+        sess.close()
