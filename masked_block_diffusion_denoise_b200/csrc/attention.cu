@@ -14,7 +14,7 @@
 // memory; the online softmax keeps one query row per thread.  The key splits
 // of one (row tile, sequence x KV head) either form a thread-block cluster
 // and combine their unnormalised partials through distributed shared memory
-// at the end (up to 8 splits), or write them to global memory for a second
+// at the end (up to 16 splits), or write them to global memory for a second
 // kernel (log-sum-exp).
 #include <math_constants.h>
 
@@ -57,7 +57,7 @@ struct AttnParams {
 // vector reads by the peers), then (max, sum) per row
 constexpr int kXoStride = kDh + 4;
 constexpr int kXoBytes = kRowsCta * kXoStride * 4;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;   // 9..16: non-portable cluster sizes
 
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
 //   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
@@ -577,17 +577,25 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(int H, int Hkv, int C, in
 
 }  // namespace
 
+// the attention kernel's function attributes: its shared memory, and
+// clusters of up to 16 CTAs (beyond the portable 8), once per process
+cudaError_t attn_set_attributes() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaErrorNotReady) {
+    done = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kAttnSmem);
+    if (done == cudaSuccess)
+      done = cudaFuncSetAttribute(attn_tc_kernel,
+                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  }
+  return done;
+}
+
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const void* q, void* o, float* opart,
                            float2* ml, const int32_t* lens, const uint8_t* done,
                            const int* n_active, int* err, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (cudaError_t e = attn_set_attributes(); e != cudaSuccess) return e;
   AttnParams p;
   p.q = (const __nv_bfloat16*)q;
   p.o = (__nv_bfloat16*)o;
@@ -609,7 +617,7 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
   if (ap.cluster > 1) {
     // the splits of a (row tile, plane) as one cluster: no partials, no combine kernel
-    if (ap.cluster != ap.nsplit || ap.cluster > 8) return cudaErrorInvalidValue;
+    if (ap.cluster != ap.nsplit || ap.cluster > kMaxCluster) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(192);
@@ -637,11 +645,15 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
 
 int attn_cluster_capacity(int n) {
   // clusters of n attention CTAs (one SM each) that can be resident at once
-  static int cap[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
-  if (n < 2 || n > 8) return 0;
+  static int cap[kMaxCluster + 1];
+  static bool init = false;
+  if (!init) {
+    for (int i = 0; i <= kMaxCluster; ++i) cap[i] = -1;
+    init = true;
+  }
+  if (n < 2 || n > kMaxCluster) return 0;
   if (cap[n] >= 0) return cap[n];
-  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kAttnSmem) != cudaSuccess) {
+  if (attn_set_attributes() != cudaSuccess) {
     cudaGetLastError();
     return cap[n] = 0;
   }

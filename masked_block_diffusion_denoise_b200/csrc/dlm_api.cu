@@ -229,7 +229,7 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
 // Split plan of the attention.  For every split count (with the smallest
 // chunk of whole 128-key tiles that gives it) the CTAs are list-scheduled in
 // launch order (split fastest) onto the SMs with a per-CTA and a per-tile
-// time; ragged prefixes (lens, host) are taken as they are.  Up to 8 splits
+// time; ragged prefixes (lens, host) are taken as they are.  Up to 16 splits
 // may combine inside a thread-block cluster (an exchange cost per CTA) when
 // the whole grid fits in one wave of resident clusters; otherwise splits
 // write partials for the combine kernel (a write cost per CTA, the kernel, a
@@ -266,7 +266,7 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
     last_nsplit = nsplit;
     const long ctas = (long)B * Hkv * a.rtiles * nsplit;
     int cl = 1;
-    if (nsplit > 1 && nsplit <= 8 && cluster_ok) {
+    if (nsplit > 1 && nsplit <= 16 && cluster_ok) {
       const int cap = attn_cluster_capacity(nsplit);
       if (cap > 0 && ctas <= (long)cap * nsplit) cl = nsplit;
     }

@@ -111,10 +111,10 @@ cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, fl
 struct AttnPlan {
   int B, C, G, R, rtiles;   // G = H / Hkv, R = G * C query rows per (seq, kv head)
   int chunk, nsplit;        // keys per split (multiple of 128), splits per (seq, kv head)
-  int cluster = 1;          // nsplit (<= 8) when the splits combine inside a cluster
+  int cluster = 1;          // nsplit (<= 16) when the splits combine inside a cluster
 };
 
-// clusters of n (2..8) attention CTAs that fit on the device at once (0: none)
+// clusters of n (2..16) attention CTAs that fit on the device at once (0: none)
 int attn_cluster_capacity(int n);
 
 // bf16: TMA-fed mma.sync flash attention over [prefix ; canvas] keys, split-KV
