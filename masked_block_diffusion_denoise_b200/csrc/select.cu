@@ -135,9 +135,12 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
   pdl_wait_then_release();
-  if (n_active != nullptr && *n_active == 0) return;
+  // the active count and this canvas's flag in one round trip
   const int b = blockIdx.x;
-  if (done[b]) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int na = n_active != nullptr ? *n_active : 1;
+  const uint8_t dn = done[b];
+  if (na == 0 || dn) return;
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
   __shared__ uint8_t com[kMaxC];
@@ -149,9 +152,17 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   int P = 32;               // keys sorted: the next power of two >= C
   while (P < C) P <<= 1;
   const size_t base = (size_t)b * C;
+  // the canvas state is loaded into registers first (its loads overlap the
+  // reduction) and stored to shared memory after it
+  const int s = step[b];
+  int32_t tok_r = 0;
+  uint8_t com_r = 0;
+  if (i < C) {
+    tok_r = tokens[base + i];
+    com_r = committed[base + i];
+  }
   if (part != nullptr) {
     // a6: the cross-tile reduction of this canvas's rows, one warp per row
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int r = warp; r < C; r += nw) {
       const size_t row = base + r;
       reduce_row(part + row * n_part, n_part, lane, cand + row, conf + row, ent + row,
@@ -162,10 +173,9 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     conf_s[i] = conf[base + i];
     ent_s[i] = ent[base + i];
   }
-  const int s = step[b];
   if (i < C) {
-    tok[i] = tokens[base + i];
-    com[i] = committed[base + i];
+    tok[i] = tok_r;
+    com[i] = com_r;
   }
   __syncthreads();
 
