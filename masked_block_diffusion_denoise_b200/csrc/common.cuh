@@ -138,7 +138,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------------------
-// TMA tensor copies (no cluster multicast anywhere in this library)
+// TMA tensor copies: every load fills only the issuing CTA's own shared memory
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
