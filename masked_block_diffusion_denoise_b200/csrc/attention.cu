@@ -49,6 +49,7 @@ struct AttnParams {
   int* err;
   int H, Hkv, G, C, R, chunk, nsplit;
   int cluster;   // > 1: the nsplit CTAs of a (row tile, plane) form a cluster and combine in it
+  int q_tma;     // the query tile by TMA (tmQ: q as [positions][H][Dh], box 64 x G x 128/G)
   float scale_log2;
 };
 
@@ -72,7 +73,7 @@ constexpr int kMaxCluster = 16;   // 9..16: non-portable cluster sizes
 // overwrite P(t) before P(t) V(t) has read it.
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                   const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
   // Before the wait for the previous kernel this CTA reads only data of
   // kernels that finished before that one started (cache lengths, done
   // flags, the active count) and the cached prefix: barriers, tensor memory
@@ -101,7 +102,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 1;
   uint64_t* mma_done = pv_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* q_full = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
+    mbar_init(q_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -131,9 +134,11 @@ __global__ void __launch_bounds__(192, 1)
     tma_load_3d(base + 3 * kHalf, &tmV, &kv_full[st], 64, key0, plane);
   };
   int pre = 0;   // tiles issued before the wait (prefix keys only)
+  const bool q_by_tma = p.q_tma != 0 && n_tiles > 0;   // a split without keys needs no query
   if (warp == 0 && lane == 0) {
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
+    if (q_by_tma) tma_prefetch(&tmQ);
     const int n_prefix = p.lens[b];
     while (pre < kStages && pre < n_tiles && k_begin + (pre + 1) * kKeys <= n_prefix) {
       issue_kv(pre);
@@ -141,9 +146,20 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   pdl_wait_then_release();
-  // query tile -> shared memory, two 64-column halves, 128-byte swizzle; every
-  // load of a thread is issued before the first store (one L2 round trip)
-  {
+  if (q_by_tma) {
+    // the query tile: positions b*C + rt*128/G .., the G heads of KV head g,
+    // two 64-column halves with the 128-byte swizzle; rows past R (the next
+    // canvas's positions, or zero fill past the buffer) are never stored
+    if (warp == 0 && lane == 0) {
+      const int z0 = b * p.C + rt * (kRowsCta / p.G);
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      tma_load_3d(qs, &tmQ, q_full, 0, g * p.G, z0);
+      tma_load_3d(qs + kHalf, &tmQ, q_full, 64, g * p.G, z0);
+    }
+  } else {
+    // query tile -> shared memory, two 64-column halves, 128-byte swizzle;
+    // every load of a thread is issued before the first store
+
     constexpr int kQChunks = kRowsCta * 16;                  // 16-byte chunks
     constexpr int kPer = (kQChunks + 191) / 192;             // per thread at 192 threads
     uint4 val[kPer];
@@ -190,6 +206,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
           mbar_wait_bounded(&kv_full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
       }
+      if (q_by_tma) mbar_wait_bounded(q_full, 0, nullptr);   // the query tile has landed
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -207,7 +224,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         umma_commit(&s_full[t & 1]);
       };
-      bool ok = n_tiles > 0 && mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+      bool ok = n_tiles > 0 && (!q_by_tma || mbar_wait_bounded(q_full, 0, abort_flag)) &&
+                mbar_wait_bounded(&kv_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -592,8 +610,8 @@ cudaError_t attn_set_attributes() {
 }
 
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
-                           const CUtensorMap& tmV, const void* q, void* o, float* opart,
-                           float2* ml, const int32_t* lens, const uint8_t* done,
+                           const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q, void* o,
+                           float* opart, float2* ml, const int32_t* lens, const uint8_t* done,
                            const int* n_active, int* err, cudaStream_t st) {
   if (cudaError_t e = attn_set_attributes(); e != cudaSuccess) return e;
   AttnParams p;
@@ -613,6 +631,8 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.chunk = ap.chunk;
   p.nsplit = ap.nsplit;
   p.cluster = ap.cluster;
+  p.q_tma = tmQ != nullptr && ap.G > 0 && kRowsCta % ap.G == 0 ? 1 : 0;
+  const CUtensorMap qmap = tmQ != nullptr ? *tmQ : tmK;   // unread without q_tma
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
   if (ap.cluster > 1) {
@@ -632,9 +652,9 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmK, tmV, p);
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmK, tmV, qmap, p);
   }
-  cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kAttnSmem, st, tmK, tmV, p);
+  cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kAttnSmem, st, tmK, tmV, qmap, p);
   if (e != cudaSuccess || ap.nsplit == 1) return e;
   const int rows_per_block = 8;
   dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);

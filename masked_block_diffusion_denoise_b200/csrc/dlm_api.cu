@@ -84,6 +84,8 @@ struct dlm_ctx {
   dlm_canvas_stats* h_stats = nullptr;
   std::map<std::tuple<const void*, uint64_t, uint64_t, uint32_t>, CUtensorMap> maps;
   CUtensorMap tmK{}, tmV{};
+  CUtensorMap tmQ{};
+  bool has_tmQ = false;   // the query tile by TMA (G divides 128)
   std::vector<GraphEntry> graphs;
   std::map<std::vector<int>, AttnPlan> plans;   // attention split plans
   cudaStream_t cap = nullptr;
@@ -160,6 +162,22 @@ bool map_kv(CUtensorMap* m, void* base, uint64_t planes, uint64_t Lcap, uint64_t
   cuuint32_t box[3] = {64, 128, 1};   // 64 head-dim columns x 128 keys (one attention tile half)
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q [positions][H][Dh] as a 3-D map whose box (64 columns, the G heads of a KV
+// head, 128/G positions) is one 64-column half of a 128-row attention query
+// tile; G must divide 128
+bool map_q(CUtensorMap* m, void* q, uint64_t positions, uint64_t H, uint64_t Dh, uint32_t G) {
+  if (G == 0 || 128 % G != 0) return false;
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {Dh, H, positions};
+  cuuint64_t strides[2] = {Dh * 2, H * Dh * 2};
+  cuuint32_t box[3] = {64, G, 128 / G};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -519,7 +537,8 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
   // a3: attention over [prefix ; canvas]
   STAGE(DLM_STAGE_ATTENTION, false);
   if (ctx->bf16) {
-    e = attention_bf16(md, ap, ctx->tmK, ctx->tmV, ctx->q, ctx->o, ctx->opart, ctx->ml,
+    e = attention_bf16(md, ap, ctx->tmK, ctx->tmV, ctx->has_tmQ ? &ctx->tmQ : nullptr, ctx->q,
+                       ctx->o, ctx->opart, ctx->ml,
                        ctx->lens_d, c->done, ctx->n_active, ctx->err, st);
     ctx->launches += ap.nsplit > 1 && ap.cluster <= 1 ? 2 : 1;
   } else {
@@ -778,6 +797,8 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
     if (!map_kv(&ctx->tmK, ctx->kc, planes, ctx->Lcap, d.head_dim) ||
         !map_kv(&ctx->tmV, ctx->vc, planes, ctx->Lcap, d.head_dim))
       return bail(fail(ctx, DLM_ECUDA, "cuTensorMapEncodeTiled (KV cache) failed"));
+    ctx->has_tmQ = map_q(&ctx->tmQ, ctx->q, (uint64_t)ctx->Mmax, d.n_heads, d.head_dim,
+                         (uint32_t)(d.n_heads / d.n_kv_heads));
   }
   *out = ctx;
   return DLM_OK;
@@ -1198,7 +1219,11 @@ int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cach
   cudaStream_t st = (cudaStream_t)stream;
   if ((e = cudaMemsetAsync(sc.err, 0, sizeof(int), st)) != cudaSuccess)
     return cuda_fail(nullptr, "cudaMemsetAsync(error word)", e);
-  e = attention_bf16(plan_ctx.md, ap, tmK, tmV, q, o, sc.opart, sc.ml, lens, nullptr, nullptr,
+  CUtensorMap tmQ;
+  const bool has_q = map_q(&tmQ, const_cast<void*>(q), (uint64_t)batch * canvas, n_heads,
+                           head_dim, (uint32_t)(n_heads / n_kv_heads));
+  e = attention_bf16(plan_ctx.md, ap, tmK, tmV, has_q ? &tmQ : nullptr, q, o, sc.opart, sc.ml,
+                     lens, nullptr, nullptr,
                      sc.err, st);
   if (e != cudaSuccess) return cuda_fail(nullptr, "attention_noalloc launch", e);
   return DLM_OK;

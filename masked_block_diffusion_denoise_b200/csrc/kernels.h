@@ -118,9 +118,11 @@ struct AttnPlan {
 int attn_cluster_capacity(int n);
 
 // bf16: TMA-fed mma.sync flash attention over [prefix ; canvas] keys, split-KV
+// tmQ: q [positions][H][Dh] as a 3-D map with box (64, G, 128/G), used when G
+// divides 128 (else, or when null, the query tile is loaded with plain loads)
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
-                           const CUtensorMap& tmV, const void* q, void* o, float* opart,
-                           float2* ml, const int32_t* lens, const uint8_t* done,
+                           const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q, void* o,
+                           float* opart, float2* ml, const int32_t* lens, const uint8_t* done,
                            const int* n_active, int* err, cudaStream_t st);
 // fp32: one thread per query row
 cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,
