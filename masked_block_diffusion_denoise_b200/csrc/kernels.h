@@ -117,7 +117,9 @@ struct AttnPlan {
 // clusters of n (2..16) attention CTAs that fit on the device at once (0: none)
 int attn_cluster_capacity(int n);
 
-// bf16: TMA-fed mma.sync flash attention over [prefix ; canvas] keys, split-KV
+// bf16: tcgen05 flash attention over [prefix ; canvas] keys (S and O in tensor
+// memory, K/V by TMA), split over keys; up to 16 splits combine inside a
+// thread-block cluster, more write partials for the combine kernel.
 // tmQ: q [positions][H][Dh] as a 3-D map with box (64, G, 128/G), used when G
 // divides 128 (else, or when null, the query tile is loaded with plain loads)
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
