@@ -76,14 +76,17 @@ __global__ void __launch_bounds__(192, 1)
                    const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
   // Before the wait for the previous kernel this CTA reads only data of
   // kernels that finished before that one started (cache lengths, done
-  // flags, the active count) and the cached prefix: barriers, tensor memory
-  // and the K/V tiles that lie wholly inside the prefix are set up early;
-  // the query tile and tiles that reach the canvas slots follow the wait.
-  if (p.n_active != nullptr && *p.n_active == 0) return;
+  // flags, the active count; read through L2, where no stale copy can be
+  // left) and the cached prefix: barriers, tensor memory and the K/V tiles
+  // that lie wholly inside the prefix are set up early; the query tile and
+  // tiles that reach the canvas slots follow the wait.
   const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-  if (p.done != nullptr && p.done[b]) return;
-  const int n_keys = p.lens[b] + p.C;
+  const int na = p.n_active != nullptr ? __ldcg(p.n_active) : 1;
+  const bool dn = p.done != nullptr && __ldcg(p.done + b) != 0;
+  const int len_b = __ldcg(p.lens + b);
+  if (na == 0 || dn) return;
+  const int n_keys = len_b + p.C;
   const int k_begin = split * p.chunk;
   // a split past the keys exits at once, except in a cluster, where it still
   // takes part in the exchange (with no rows of its own)
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
     if (q_by_tma) tma_prefetch(&tmQ);
-    const int n_prefix = p.lens[b];
+    const int n_prefix = len_b;
     while (pre < kStages && pre < n_tiles && k_begin + (pre + 1) * kKeys <= n_prefix) {
       issue_kv(pre);
       ++pre;

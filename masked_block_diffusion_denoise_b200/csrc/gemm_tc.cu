@@ -179,17 +179,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   // The weights (B) do not depend on the previous kernel: before waiting for
   // it, the producer puts the B tiles of the first ring stages in flight
-  // (expected bytes raised, no arrival yet); the A tiles follow the wait.
-  // Weights are read once per launch: they stream through L2 with evict_first.
+  // (expected bytes raised, no arrival yet).  Right after the wait, before
+  // anything else, it issues those stages' A tiles; the active count is read
+  // only then, so its round trip overlaps the A loads.  Weights are read once
+  // per launch: they stream through L2 with evict_first.
   int pre = 0;
   uint64_t pol_stream = 0;
+  int m_first = 0, kb_first = 0;
   if (warp == 0 && lane == 0) {
     pol_stream = l2_evict_first_policy();
-    int m0, n0, kb0, kb1, sp0;
-    if (get_unit<EPI>(p, 0, m0, n0, kb0, kb1, sp0)) {
-      pre = min(stages, kb1 - kb0);
+    int n0, kb1, sp0;
+    if (get_unit<EPI>(p, 0, m_first, n0, kb_first, kb1, sp0)) {
+      pre = min(stages, kb1 - kb_first);
       for (int s = 0; s < pre; ++s) {
-        const int kb = kb0 + s;
+        const int kb = kb_first + s;
         mbar_expect_tx(&full[s], Cfg::kBBytes);
         tma_load_2d_hint(smem + s * stage_bytes, &tmB, &full[s], kb * kBKe, n0 * BN, pol_stream);
       }
@@ -197,15 +200,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   // the prologue above touched only shared and tensor memory and weights
   pdl_wait_then_release();
+  if (warp == 0 && lane == 0) {
+    // the A tiles of the stages whose B tiles are in flight (the A buffer is
+    // always allocated, so these loads are issued even when the step turns
+    // out to have nothing to do)
+    for (int s = 0; s < pre; ++s) {
+      mbar_arrive_expect_tx(&full[s], a_bytes);
+      tma_load_2d(smem + s * stage_bytes + Cfg::kBBytes, &tmA, &full[s], (kb_first + s) * kBKe,
+                  m_first * kBM);
+    }
+  }
   const bool skip = p.n_active != nullptr && *p.n_active == 0;
 
   if (skip) {
-    // nothing to do this step: land the early weight tiles, then teardown
+    // nothing to do this step: land the early tiles, then teardown
     if (warp == 0 && lane == 0)
-      for (int s = 0; s < pre; ++s) {
-        mbar_arrive(&full[s]);
-        mbar_wait_bounded(&full[s], 0u, nullptr);
-      }
+      for (int s = 0; s < pre; ++s) mbar_wait_bounded(&full[s], 0u, nullptr);
   } else if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -216,17 +226,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int m, n, kb0, kb1, split;
       for (int it = 0; ok && get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = smem + stage * stage_bytes;
-          uint8_t* sa = sb + Cfg::kBBytes;
-          if (issued < pre) {
-            // this stage's B tile is already in flight
-            mbar_arrive_expect_tx(&full[stage], a_bytes);
-            tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
-          } else {
+          // The first `pre` stages (their first use of the ring) are already
+          // in flight.  Their empty slots are not waited for: the MMA may have
+          // consumed and released them already, and a wait on the released
+          // phase would then wait for the next one.
+          if (issued >= pre) {
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sb = smem + stage * stage_bytes;
+            uint8_t* sa = sb + Cfg::kBBytes;
             mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
             tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
             tma_load_2d_hint(sb, &tmB, &full[stage], kb * kBKe, n * BN, pol_stream);
@@ -241,8 +251,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         // let the copies already in flight land before the CTA exits
         if (issued < pre) {
-          // early B tiles without their A: arrive so the phase can complete
-          for (int s = issued; s < pre; ++s) mbar_arrive(&full[s]);
           for (int s = 0; s < pre; ++s) mbar_wait_bounded(&full[s], 0u, nullptr);
         } else {
           int st = stage, ph = phase;

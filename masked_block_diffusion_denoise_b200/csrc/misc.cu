@@ -25,6 +25,12 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
                              T* __restrict__ x, int rows, int C, int d, int V, int B,
                              const uint8_t* __restrict__ done, int* n_active, int* err) {
   pdl_wait_then_release();
+  // this row's done flag and token are loaded together (and with block 0's
+  // loads of every canvas's flag for the active count)
+  const int r = blockIdx.x;
+  const bool row_ok = r < rows;
+  const bool dn = row_ok && done != nullptr && done[r / C] != 0;
+  int t = row_ok ? tokens[r] : 0;
   if (blockIdx.x == 0 && n_active != nullptr) {
     __shared__ int cnt;
     if (threadIdx.x == 0) cnt = 0;
@@ -35,10 +41,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
     __syncthreads();
     if (threadIdx.x == 0) *n_active = cnt;
   }
-  const int r = blockIdx.x;
-  if (r >= rows) return;
-  if (done != nullptr && done[r / C]) return;
-  int t = tokens[r];
+  if (!row_ok || dn) return;
   if (t < 0 || t >= V) {
     if (threadIdx.x == 0) raise_error(err, DLM_EBOUNDS);
     t = 0;
@@ -49,15 +52,19 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
   for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
 }
 
-// block (row, group of heads): one rotary pair (j, j + Dh/2) per thread
+// block (row, group of heads): one rotary pair (j, j + Dh/2) per thread.
+// The direct predecessor is always the GEMM that writes `part`; the active
+// count, done flags, cache lengths and the rotary table come from earlier
+// kernels, which have completed once this kernel may start (every kernel of
+// the chain lets its successor launch only after its own wait), so they are
+// read before the wait (through L2: a line left in L1 by an earlier step
+// would be stale) and only the partial sums after it.
 template <typename T>
 __global__ void __launch_bounds__(256)
     qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part, int splits, int rows, int C,
                         int seq_fixed, int head0, const int32_t* __restrict__ lens,
                         const float2* __restrict__ rope, T* __restrict__ q, T* __restrict__ kc,
                         T* __restrict__ vc, const uint8_t* __restrict__ done, const int* n_active) {
-  pdl_wait_then_release();
-  if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.x;
   const int half = md.Dh / 2;
   int seq, p_in;
@@ -67,17 +74,25 @@ __global__ void __launch_bounds__(256)
   } else {
     seq = r / C;
     p_in = r - seq * C;
-    if (done != nullptr && done[seq]) return;
   }
-  const int pos = lens[seq] + p_in;
+  // issued together: active count, done flag, cache length
+  const int na = n_active != nullptr ? __ldcg(n_active) : 1;
+  const bool dn = seq_fixed < 0 && done != nullptr && __ldcg(done + seq) != 0;
+  const int len = __ldcg(lens + seq);
   const int nheads = md.H + 2 * md.Hkv - head0;
   const int ncols = nheads * md.Dh;
   const int per_block = blockDim.x / half;
+  const int item = blockIdx.y * per_block * half + threadIdx.x;
+  const bool active = na != 0 && !dn && item < nheads * half;
+  const int hl = item / half, j = item - hl * half;
+  const int hh = hl + head0;
+  const int pos = len + p_in;
+  const bool rotate = rope != nullptr && hh < md.H + md.Hkv;
+  float2 cs = make_float2(1.f, 0.f);
+  if (active && rotate) cs = rope[(size_t)pos * half + j];
+  pdl_wait_then_release();
+  if (!active) return;
   {
-    const int item = blockIdx.y * per_block * half + threadIdx.x;
-    if (item >= nheads * half) return;
-    const int hl = item / half, j = item - hl * half;
-    const int hh = hl + head0;
     const int cb = hl * md.Dh;
     float a = 0.f, b = 0.f;
     for (int s = 0; s < splits; ++s) {
@@ -85,8 +100,7 @@ __global__ void __launch_bounds__(256)
       a += pr[j];
       b += pr[j + half];
     }
-    if (rope != nullptr && hh < md.H + md.Hkv) {
-      const float2 cs = rope[(size_t)pos * half + j];
+    if (rotate) {
       const float a2 = a * cs.x - b * cs.y;
       const float b2 = b * cs.x + a * cs.y;
       a = a2;
@@ -105,20 +119,24 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The direct predecessor is the GEMM that writes `part`; the active count,
+// done flags and x come from earlier kernels (complete once this kernel may
+// start) and are read before the wait, through L2.
 template <typename T>
 __global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, int rows, int d,
                                    int C, const T* __restrict__ x, T* __restrict__ y,
                                    const uint8_t* __restrict__ done, const int* n_active) {
-  pdl_wait_then_release();
-  if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.y;
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d) return;
-  if (done != nullptr && done[r / C]) return;
+  const size_t i = (size_t)r * d + c;
+  const int na = n_active != nullptr ? __ldcg(n_active) : 1;
+  const bool dn = done != nullptr && __ldcg(done + r / C) != 0;
+  const float xv = c < d ? to_f32(__ldcg(x + i)) : 0.f;
+  pdl_wait_then_release();
+  if (na == 0 || dn || c >= d) return;
   float acc = 0.f;
   for (int s = 0; s < splits; ++s) acc += part[((size_t)s * rows + r) * d + c];
-  const size_t i = (size_t)r * d + c;
-  y[i] = from_f32<T>(to_f32(x[i]) + acc);
+  y[i] = from_f32<T>(xv + acc);
 }
 
 template <typename T>

@@ -134,12 +134,31 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
-  pdl_wait_then_release();
-  // the active count and this canvas's flag in one round trip
+  // Inside a step (partials given) the direct predecessor is the LM head,
+  // which writes only the partials: the active count and the canvas state
+  // come from earlier kernels, complete once this kernel may start (every
+  // kernel of the chain lets its successor launch only after its own wait),
+  // and are read before the wait, through L2.  Given candidates (a call on
+  // its own) the predecessor is unknown and everything is read after it.
+  const bool early = part != nullptr;
+  if (!early) pdl_wait_then_release();
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int na = n_active != nullptr ? *n_active : 1;
-  const uint8_t dn = done[b];
+  const int i = threadIdx.x;
+  const int C = a.C;
+  const size_t base = (size_t)b * C;
+  // the active count, this canvas's flag and state in one round trip; the
+  // state goes to registers and reaches shared memory after the reduction
+  const int na = n_active != nullptr ? __ldcg(n_active) : 1;
+  const uint8_t dn = __ldcg(done + b);
+  const int s = __ldcg(step + b);
+  int32_t tok_r = 0;
+  uint8_t com_r = 0;
+  if (i < C) {
+    tok_r = __ldcg(tokens + base + i);
+    com_r = __ldcg(committed + base + i);
+  }
+  if (early) pdl_wait_then_release();
   if (na == 0 || dn) return;
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
@@ -147,20 +166,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   __shared__ int32_t cand_s[kMaxC];   // this canvas's candidates, confidences, entropies
   __shared__ float conf_s[kMaxC], ent_s[kMaxC];
   __shared__ int e_s, k_s, krule_s;
-  const int i = threadIdx.x;
-  const int C = a.C;
   int P = 32;               // keys sorted: the next power of two >= C
   while (P < C) P <<= 1;
-  const size_t base = (size_t)b * C;
-  // the canvas state is loaded into registers first (its loads overlap the
-  // reduction) and stored to shared memory after it
-  const int s = step[b];
-  int32_t tok_r = 0;
-  uint8_t com_r = 0;
-  if (i < C) {
-    tok_r = tokens[base + i];
-    com_r = committed[base + i];
-  }
   if (part != nullptr) {
     // a6: the cross-tile reduction of this canvas's rows, one warp per row
     for (int r = warp; r < C; r += nw) {
