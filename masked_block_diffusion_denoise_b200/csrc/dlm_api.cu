@@ -71,7 +71,7 @@ struct dlm_ctx {
   size_t opart_floats = 0;
   float2* ml = nullptr;
   size_t ml_count = 0;
-  LmPart* lmpart = nullptr;
+  float* lmpart = nullptr;   // LM-head partials, [M][kLmFields][n_part]
   int32_t* cand = nullptr;
   float *conf = nullptr, *ent = nullptr;
   float2* rope = nullptr;
@@ -731,7 +731,8 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if ((rc = dalloc(ctx, &ctx->o, ctx->Mmax * qd * es))) return bail(rc);
   if ((rc = dalloc(ctx, &ctx->y, ctx->Mmax * dm * es))) return bail(rc);
   const int lm_tile = ctx->bf16 ? 128 : 64;
-  if ((rc = dalloc(ctx, &ctx->lmpart, (size_t)ctx->Mmax * cdiv(d.vocab, lm_tile) * sizeof(LmPart))))
+  if ((rc = dalloc(ctx, &ctx->lmpart,
+                   (size_t)ctx->Mmax * cdiv(d.vocab, lm_tile) * kLmFields * sizeof(float))))
     return bail(rc);
   if ((rc = dalloc(ctx, &ctx->cand, ctx->Mmax * sizeof(int32_t)))) return bail(rc);
   if ((rc = dalloc(ctx, &ctx->conf, ctx->Mmax * sizeof(float)))) return bail(rc);

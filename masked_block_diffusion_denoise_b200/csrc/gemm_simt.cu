@@ -13,7 +13,7 @@ constexpr int kTK = 16;
 struct SimtParams {
   int M, N, K, splits, n_tiles;
   float* out;
-  LmPart* part;
+  float* part;   // EPI_LM partials, [M][kLmFields][n_tiles]
   LmEpi epi;
   const uint8_t* done;
   const int* n_active;
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
             for (int j = 0; j < 32; ++j) v[j] = Ts[threadIdx.x][c + j];
             rs_update<32>(rs, v, n0 + c, inv_t, p.epi, canvas, pos, step);
           }
-          rs_store(p.part + (size_t)row * p.n_tiles + blockIdx.x, rs);
+          rs_store(p.part, p.n_tiles, (size_t)row, blockIdx.x, rs);
         }
       }
     }

@@ -22,7 +22,7 @@
 //   EPI_LM   the LM head's fused vocabulary reduction.  CTA c keeps m tile
 //            c % m_tiles and walks vocabulary tiles c / m_tiles + k * slots;
 //            each epilogue thread folds every tile of its row into one row
-//            state and writes one LmPart per (row, CTA); logits never leave
+//            state and writes one partial per (row, CTA); logits never leave
 //            the SM.  CTAs with the same slot read the same weight slab at
 //            about the same time (L2 reuse across m tiles).
 #include <cstdio>
@@ -71,7 +71,7 @@ struct TcParams {
   int m_tiles, n_tiles, splits, units, kblocks;
   int a_rows, stages;    // A box rows (multiple of 8, <= 128), ring stages
   float* out;
-  LmPart* part;
+  float* part;           // EPI_LM partials, [M][kLmFields][slots]
   LmEpi epi;
   ProjEpi proj;
   const uint8_t* done;   // [B] canvases that are finished (LM rows skipped)
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (wg == 0) {
         const RowState both = rs_combine(rs, xch[lr]);
         const int slots = gridDim.x / p.m_tiles;
-        if (lm_live) rs_store(p.part + (size_t)lm_row * slots + blockIdx.x / p.m_tiles, both);
+        if (lm_live) rs_store(p.part, slots, (size_t)lm_row, blockIdx.x / p.m_tiles, both);
       }
     }
   }

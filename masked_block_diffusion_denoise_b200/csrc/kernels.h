@@ -38,7 +38,7 @@ struct ProjEpi {
 
 struct GemmIO {
   float* out = nullptr;        // EPI_F32: [splits][M][N]
-  LmPart* part = nullptr;      // EPI_LM:  [M][n_tiles]
+  float* part = nullptr;       // EPI_LM:  [M][kLmFields][n_part]
   LmEpi epi{};
   ProjEpi proj{};
   const uint8_t* done = nullptr;
@@ -153,7 +153,7 @@ struct SelectArgs {
 // given cand / conf / ent.
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
                         uint8_t* done, int32_t* eos_pos, int32_t* prev_cand, int32_t* stable,
-                        const LmPart* part, int n_part, int32_t* cand, float* conf, float* ent,
+                        const float* part, int n_part, int32_t* cand, float* conf, float* ent,
                         dlm_canvas_stats* stats, const int* n_active, int* err, cudaStream_t st);
 
 }  // namespace dlm

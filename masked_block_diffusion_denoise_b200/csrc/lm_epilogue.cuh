@@ -20,6 +20,11 @@ struct LmPart {
   int idx;
 };
 
+// Partials are stored field-major within a row, [row][kLmFields][n_part]
+// floats (idx as its int bits): a warp that reads one field of 32
+// consecutive partials of a row reads one contiguous 128-byte line.
+constexpr int kLmFields = 6;
+
 enum { LM_GREEDY = 0, LM_SAMPLE_FIXED = 1, LM_SAMPLE_ANNEAL = 2 };
 
 struct LmEpi {
@@ -135,15 +140,16 @@ __device__ __forceinline__ void rs_update(RowState& r, const float (&v)[N], int 
   }
 }
 
-__device__ __forceinline__ void rs_store(LmPart* dst, const RowState& r) {
-  LmPart p;
-  p.m = r.m;
-  p.s = r.s;
-  p.t = r.t;
-  p.g = r.g;
-  p.zw = r.zw;
-  p.idx = r.idx;
-  *dst = p;
+// partial j of row `row` (n_part partials per row)
+__device__ __forceinline__ void rs_store(float* part, int n_part, size_t row, int j,
+                                         const RowState& r) {
+  float* d = part + row * kLmFields * (size_t)n_part + j;
+  d[0] = r.m;
+  d[n_part] = r.s;
+  d[2 * n_part] = r.t;
+  d[3 * n_part] = r.g;
+  d[4 * n_part] = r.zw;
+  d[5 * n_part] = __int_as_float(r.idx);
 }
 
 // combine two partial states (the order of arguments fixes the tie rule:

@@ -21,7 +21,7 @@ namespace {
 // maximum, after which every lane's terms are independent of one another (no
 // chain of pairwise merges); the lane sums and the winner meet in fixed
 // butterflies, so the result does not depend on timing.
-__device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, int32_t* cand,
+__device__ void reduce_row(const float* __restrict__ pr, int n_part, int lane, int32_t* cand,
                            float* conf, float* ent, int32_t* cand_sm, float* conf_sm,
                            float* ent_sm) {
   constexpr int kU = 5;   // one chunk covers one partial per SM of a 148-SM part
@@ -37,7 +37,13 @@ __device__ void reduce_row(const LmPart* __restrict__ pr, int n_part, int lane, 
       const int j = j0 + lane + 32 * u;
       ok[u] = j < n_part;
       if (ok[u]) {
-        q[u] = pr[j];
+        // field-major row: each field of 32 partials is one 128-byte line
+        q[u].m = pr[j];
+        q[u].s = pr[n_part + j];
+        q[u].t = pr[2 * n_part + j];
+        q[u].g = pr[3 * n_part + j];
+        q[u].zw = pr[4 * n_part + j];
+        q[u].idx = __float_as_int(pr[5 * n_part + j]);
         ok[u] = q[u].m != -CUDART_INF_F;   // a tile with every column excluded
       }
       if (ok[u]) mloc = fmaxf(mloc, q[u].m);
@@ -130,7 +136,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               uint8_t* __restrict__ committed, int32_t* __restrict__ step,
                               uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
                               int32_t* __restrict__ prev_cand, int32_t* __restrict__ stable,
-                              const LmPart* __restrict__ part, int n_part,
+                              const float* __restrict__ part, int n_part,
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     // a6: the cross-tile reduction of this canvas's rows, one warp per row
     for (int r = warp; r < C; r += nw) {
       const size_t row = base + r;
-      reduce_row(part + row * n_part, n_part, lane, cand + row, conf + row, ent + row,
+      reduce_row(part + row * kLmFields * (size_t)n_part, n_part, lane, cand + row, conf + row, ent + row,
                  cand_s + r, conf_s + r, ent_s + r);
     }
   } else if (i < C) {
@@ -372,7 +378,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
 
 cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed, int32_t* step,
                         uint8_t* done, int32_t* eos_pos, int32_t* prev_cand, int32_t* stable,
-                        const LmPart* part, int n_part, int32_t* cand, float* conf, float* ent,
+                        const float* part, int n_part, int32_t* cand, float* conf, float* ent,
                         dlm_canvas_stats* stats, const int* n_active, int* err, cudaStream_t st) {
   int P = 32;
   while (P < a.C) P <<= 1;
