@@ -14,8 +14,9 @@
 // memory; the online softmax keeps one query row per thread.  The key splits
 // of one (row tile, sequence x KV head) either form a thread-block cluster
 // and combine their unnormalised partials through distributed shared memory
-// at the end (up to 16 splits), or write them to global memory for a second
-// kernel (log-sum-exp).
+// at the end (up to 16 splits: each CTA bulk-copies to every peer the rows
+// that peer combines), or write them to global memory for a second kernel
+// (log-sum-exp).
 #include <math_constants.h>
 
 #include <cooperative_groups.h>
@@ -54,11 +55,17 @@ struct AttnParams {
 };
 
 // cluster exchange area (in the K/V ring, free once the last tile is done):
-// unnormalised O rows with a stride of 132 floats (16-byte aligned rows for
-// vector reads by the peers), then (max, sum) per row
+// this split's rows, unnormalised O (128 floats) then (max, sum) in the
+// row's pad, 132 floats (528 bytes) a row; then the receive area, where
+// peer j's copy of the rows this CTA combines lands at slot j.
 constexpr int kXoStride = kDh + 4;
-constexpr int kXoBytes = kRowsCta * kXoStride * 4;
+constexpr int kXoRowBytes = kXoStride * 4;
+constexpr int kXoBytes = kRowsCta * kXoRowBytes;
 constexpr int kMaxCluster = 16;   // 9..16: non-portable cluster sizes
+constexpr int kRecvOff = kXoBytes;
+static_assert(kRecvOff + (kRowsCta + kMaxCluster) * kXoRowBytes <= kStages * kStageBytes,
+              "exchange areas exceed the K/V ring");
+static_assert(kXoRowBytes % 16 == 0 && kRecvOff % 16 == 0, "bulk copies need 16-byte units");
 
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
 //   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
@@ -106,7 +113,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* pv_done = p_full + 1;
   uint64_t* mma_done = pv_done + 1;
   uint64_t* q_full = mma_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
+  uint64_t* rx = q_full + 1;   // cluster exchange: the peers' rows have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rx + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -120,6 +128,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     mbar_init(q_full, 1);
+    mbar_init(rx, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -364,8 +373,9 @@ __global__ void __launch_bounds__(192, 1)
       float* xo = reinterpret_cast<float*>(ring) + row * kXoStride;
 #pragma unroll
       for (int j = 0; j < kDh; ++j) xo[j] = have ? ov[j] : 0.f;
-      reinterpret_cast<float2*>(ring + kXoBytes)[row] =
+      *reinterpret_cast<float2*>(xo + kDh) =
           have ? make_float2(m_run, l_run) : make_float2(-CUDART_INF_F, 0.f);
+      fence_proxy_async_smem();   // the rows are read by bulk copies (async proxy)
     } else if (have) {
       const int r = rt * kRowsCta + row;
       if (r < p.R) {
@@ -397,23 +407,32 @@ __global__ void __launch_bounds__(192, 1)
   if (p.cluster > 1) {
     // every split's rows are in its shared memory; CTA q of the cluster
     // combines rows q*ceil(128/n) .. of the tile for all splits (fixed order).
-    // All peer reads of an item are issued before any of them is used.
     cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
     const int n = p.cluster;
     const int q = (int)cluster.block_rank();
     const int per = (kRowsCta + n - 1) / n;
-    const int r0 = q * per, r1 = min(kRowsCta, r0 + per);
-    const float* xo_self = reinterpret_cast<const float*>(ring);
-    const float2* xml_self = reinterpret_cast<const float2*>(ring + kXoBytes);
-    const float* xo_p[kMaxCluster];
-    const float2* xml_p[kMaxCluster];
-#pragma unroll
-    for (int j = 0; j < kMaxCluster; ++j) {
-      const int jj = j < n ? j : 0;
-      xo_p[j] = cluster.map_shared_rank(xo_self, jj);
-      xml_p[j] = cluster.map_shared_rank(xml_self, jj);
+    const int r0 = min(kRowsCta, q * per), r1 = min(kRowsCta, r0 + per);
+    uint8_t* recv = ring + kRecvOff;
+    // every CTA copies, with one bulk copy per peer, the rows that peer
+    // combines into the peer's receive area; then each CTA combines from
+    // its own shared memory
+    if (tid == 0) mbar_arrive_expect_tx(rx, (uint32_t)((n - 1) * (r1 - r0) * kXoRowBytes));
+    cluster.sync();   // rows written, receive barriers armed
+    if (tid < n && tid != q) {
+      const int a0 = min(kRowsCta, tid * per), a1 = min(kRowsCta, a0 + per);
+      if (a1 > a0)
+        bulk_copy_to_peer(cluster_addr(smem_u32(recv + q * per * kXoRowBytes), tid),
+                          smem_u32(ring + a0 * kXoRowBytes), (uint32_t)((a1 - a0) * kXoRowBytes),
+                          cluster_addr(smem_u32(rx), tid));
     }
+    // the copies into this CTA land before it reads them -- or, after an
+    // abort, before it exits
+    if (!mbar_wait_bounded(rx, 0, abort_flag)) mbar_wait_bounded(rx, 0, nullptr);
+    const float* xo_p[kMaxCluster];   // split j's row r0 + i: xo_p[j] + i * kXoStride
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j)
+      xo_p[j] = j == q ? reinterpret_cast<const float*>(ring + r0 * kXoRowBytes)
+                       : reinterpret_cast<const float*>(recv + (j < n ? j : 0) * per * kXoRowBytes);
     for (int it = tid; it < (r1 - r0) * (kDh / 4); it += blockDim.x) {
       const int lr = r0 + it / (kDh / 4);
       const int c4 = (it % (kDh / 4)) * 4;
@@ -423,9 +442,9 @@ __global__ void __launch_bounds__(192, 1)
       float4 ov4[kMaxCluster];
 #pragma unroll
       for (int j = 0; j < kMaxCluster; ++j) {
-        ml[j] = j < n ? xml_p[j][lr] : make_float2(-CUDART_INF_F, 0.f);
-        ov4[j] = j < n ? *reinterpret_cast<const float4*>(xo_p[j] + lr * kXoStride + c4)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* src = xo_p[j] + (lr - r0) * kXoStride;
+        ml[j] = j < n ? *reinterpret_cast<const float2*>(src + kDh) : make_float2(-CUDART_INF_F, 0.f);
+        ov4[j] = j < n ? *reinterpret_cast<const float4*>(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       float M = -CUDART_INF_F;
 #pragma unroll
@@ -449,7 +468,9 @@ __global__ void __launch_bounds__(192, 1)
       w2.y = pack_bf16(acc.z * inv, acc.w * inv);
       *reinterpret_cast<uint2*>(dst) = w2;
     }
-    cluster.sync();   // the peers have finished reading this CTA's rows
+    // every copy into every CTA of the cluster has landed (each CTA arrives
+    // after its receive barrier): the rows may be released
+    cluster.sync();
   }
 
   tc_fence_before();

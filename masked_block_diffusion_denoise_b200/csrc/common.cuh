@@ -366,6 +366,25 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
+// distributed shared memory: the address of a shared-memory location in the
+// CTA of rank `rank` of this cluster, and a bulk copy from this CTA's shared
+// memory into another CTA's, completing (bytes) on an mbarrier of that CTA
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_local,
+                                                  uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(dst_cluster),
+      "r"(src_local), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // small conversions
 // ---------------------------------------------------------------------------
 
