@@ -370,11 +370,14 @@ __global__ void __launch_bounds__(192, 1)
     if (p.cluster > 1) {
       // this split's rows for the cluster: unnormalised O, running max and sum
       fence_proxy_async_smem();
-      float* xo = reinterpret_cast<float*>(ring) + row * kXoStride;
+      // 16-byte stores: a warp's rows (528 bytes apart) fill all 32 banks
+      float4* xo = reinterpret_cast<float4*>(ring + row * kXoRowBytes);
 #pragma unroll
-      for (int j = 0; j < kDh; ++j) xo[j] = have ? ov[j] : 0.f;
-      *reinterpret_cast<float2*>(xo + kDh) =
-          have ? make_float2(m_run, l_run) : make_float2(-CUDART_INF_F, 0.f);
+      for (int c = 0; c < kDh / 4; ++c)
+        xo[c] = have ? make_float4(ov[4 * c], ov[4 * c + 1], ov[4 * c + 2], ov[4 * c + 3])
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+      xo[kDh / 4] = have ? make_float4(m_run, l_run, 0.f, 0.f)
+                         : make_float4(-CUDART_INF_F, 0.f, 0.f, 0.f);
       fence_proxy_async_smem();   // the rows are read by bulk copies (async proxy)
     } else if (have) {
       const int r = rt * kRowsCta + row;

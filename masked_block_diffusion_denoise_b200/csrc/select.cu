@@ -164,6 +164,26 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     tok_r = __ldcg(tokens + base + i);
     com_r = __ldcg(committed + base + i);
   }
+  // adaptive stopping's state and the counters, updated at the end, are
+  // read here too (kept in shared memory), so that no load is left for the
+  // end of the kernel
+  __shared__ int32_t prev_s[kMaxC];
+  __shared__ int32_t stable_s;
+  __shared__ dlm_canvas_stats st0;
+  const bool stopping = a.stop_entropy > 0.f;
+  if (stopping && i < C) prev_s[i] = __ldcg(prev_cand + base + i);
+  if (i == 0) {
+    if (stopping) stable_s = __ldcg(stable + b);
+    if (stats != nullptr) {
+      const int32_t* sp = reinterpret_cast<const int32_t*>(stats + b);
+      st0.steps_used = __ldcg(sp + 0);
+      st0.committed_by_sampler = __ldcg(sp + 1);
+      st0.forced_at_budget = __ldcg(sp + 2);
+      st0.eos_autofill = __ldcg(sp + 3);
+      st0.frozen = __ldcg(sp + 4);
+      st0.edited = __ldcg(sp + 5);
+    }
+  }
   if (early) pdl_wait_then_release();
   if (na == 0 || dn) return;
   __shared__ unsigned long long keys[kMaxC];
@@ -216,20 +236,20 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     nedit = __syncthreads_count(ed);
   }
 
-  if (a.stop_entropy > 0.f) {
+  if (stopping) {
     // adaptive stopping: the argmax of every position unchanged since the
     // previous step counts one stable step; with enough stable steps and a
     // mean entropy (float32, summed in position order) below the bound the
     // canvas freezes: every open position commits its candidate
     __shared__ int freeze_s;
-    const bool same = (i >= C) || (cand_s[i] == prev_cand[base + i]);
+    const bool same = (i >= C) || (cand_s[i] == prev_s[i]);
     const int all_same = __syncthreads_and(same);
     if (i < C) prev_cand[base + i] = cand_s[i];
     if (i == 0) {
       float total = 0.f;
       for (int j = 0; j < C; ++j) total = __fadd_rn(total, ent_s[j] + 0.0f);
       const float mean = __fdiv_rn(total, (float)C);
-      const int st = all_same ? stable[b] + 1 : 0;
+      const int st = all_same ? stable_s + 1 : 0;
       stable[b] = st;
       freeze_s = (st >= a.stability_steps && mean < a.stop_entropy) ? 1 : 0;
     }
@@ -257,10 +277,11 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
         step[b] = s + 1;
         eos_pos[b] = e;
         if (stats != nullptr) {
-          stats[b].steps_used += 1;
-          stats[b].frozen += nfrozen;
-          stats[b].eos_autofill += fill0 + fill1;
-          stats[b].edited += nedit;
+          dlm_canvas_stats& so = stats[b];
+          so.steps_used = st0.steps_used + 1;
+          so.frozen = st0.frozen + nfrozen;
+          so.eos_autofill = st0.eos_autofill + fill0 + fill1;
+          so.edited = st0.edited + nedit;
         }
       }
       return;
@@ -365,11 +386,12 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     step[b] = s + 1;
     eos_pos[b] = e;
     if (stats != nullptr) {
-      stats[b].steps_used += 1;
-      stats[b].committed_by_sampler += k;
-      stats[b].forced_at_budget += k - krule_s;
-      stats[b].eos_autofill += fill0 + fill1;
-      stats[b].edited += nedit;
+      dlm_canvas_stats& so = stats[b];
+      so.steps_used = st0.steps_used + 1;
+      so.committed_by_sampler = st0.committed_by_sampler + k;
+      so.forced_at_budget = st0.forced_at_budget + k - krule_s;
+      so.eos_autofill = st0.eos_autofill + fill0 + fill1;
+      so.edited = st0.edited + nedit;
     }
   }
 }
