@@ -324,6 +324,28 @@ int dlm_attention_noalloc(const void *q, const void *k_cache, const void *v_cach
  * DLM_ETIMEOUT / DLM_EBOUNDS set by a kernel); clears it. */
 int dlm_check(dlm_ctx *ctx, void *stream);
 
+/* ---- device timeline (tracing) ------------------------------------------
+ * A library built with `python -m masked_block_diffusion_denoise_b200.build
+ * --trace` (libdlm_trace.so, compiled with DLM_TRACE) stamps the GPU's
+ * global timer (%globaltimer, ns) per CTA in every kernel of the step: slot
+ * 0 the CTA's entry, 1 its exit (last warp out), 2 the programmatic-launch
+ * wait returned, 3.. kernel phases (GEMM: first / last ring stage full,
+ * first accumulator ready, last epilogue done; attention: query and first
+ * K/V tile loaded, O complete, cluster barrier, peers' rows received,
+ * combined; commit: rows reduced, keys sorted, done).  The table keeps the
+ * last launch of each kind; 0 = not reached.  Kinds: 0 embed, 1 QKV GEMM,
+ * 2 QKV epilogue, 3 attention, 4 attention combine, 5 Wo GEMM, 6 Wo
+ * epilogue, 7 row quantisation, 8 LM head, 9 commit.  The default build
+ * exports the same calls; they return DLM_ESTATE. */
+
+/* Table dimensions: kinds x ctas (linear CTA index) x slots. */
+int dlm_trace_layout(int *kinds, int *ctas, int *slots);
+/* Synchronise the device and copy the table (uint64, kinds*ctas*slots
+ * words, row-major) to host memory `table`; `words` is its capacity. */
+int dlm_trace_read(unsigned long long *table, size_t words);
+/* Zero the table (synchronises the device). */
+int dlm_trace_clear(void);
+
 /* Number of kernel launches one dlm_denoise_step made for this batch and
  * configuration (the last one issued), for launch accounting. */
 int dlm_launches_per_step(const dlm_ctx *ctx);

@@ -24,7 +24,9 @@ __all__ = [
     "dlm_decode_block", "dlm_decode_block_host", "dlm_commit", "dlm_generate", "dlm_debug_buffer",
     "dlm_debug_logits", "dlm_check", "dlm_launches_per_step", "dlm_last_error",
     "EXPORTED_SYMBOLS", "dlm_set_stage_events", "DLM_STAGE_EMBED", "DLM_STAGE_QKV",
-    "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT", "DLM_NUM_STAGES", "dlm_attention_noalloc",
+    "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT",
+    "DLM_NUM_STAGES", "dlm_attention_noalloc", "dlm_trace_layout", "dlm_trace_read",
+    "dlm_trace_clear",
 ]
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, DLM_ESTATE = \
@@ -113,6 +115,9 @@ _SIGS = {
     "dlm_attention_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
     "dlm_check": (_I, [_P, _P]),
     "dlm_launches_per_step": (_I, [_P]),
+    "dlm_trace_layout": (_I, [ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "dlm_trace_read": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_size_t]),
+    "dlm_trace_clear": (_I, []),
     "dlm_last_error": (ctypes.c_char_p, [_P]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGS)
@@ -273,3 +278,25 @@ def dlm_check(ctx, stream=None) -> int:
 
 def dlm_launches_per_step(ctx) -> int:
     return _check(ctx, lib().dlm_launches_per_step(ctx))
+
+
+def dlm_trace_layout():
+    """(kinds, ctas, slots) of the device timeline; DlmError(DLM_ESTATE)
+    unless the library is the DLM_TRACE build (see include/dlm.h)."""
+    k, c, s = _I(), _I(), _I()
+    _check(None, lib().dlm_trace_layout(ctypes.byref(k), ctypes.byref(c), ctypes.byref(s)))
+    return k.value, c.value, s.value
+
+
+def dlm_trace_read():
+    """The device timeline as a uint64 array [kinds][ctas][slots] (ns)."""
+    import numpy as np
+    k, c, s = dlm_trace_layout()
+    t = np.zeros(k * c * s, dtype=np.uint64)
+    _check(None, lib().dlm_trace_read(t.ctypes.data_as(ctypes.POINTER(ctypes.c_ulonglong)),
+                                      t.size))
+    return t.reshape(k, c, s)
+
+
+def dlm_trace_clear() -> int:
+    return _check(None, lib().dlm_trace_clear())

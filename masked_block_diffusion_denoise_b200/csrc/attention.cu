@@ -24,6 +24,9 @@
 #include "kernels.h"
 
 namespace dlm {
+
+DLM_TRACE_STORAGE(attn)
+
 namespace {
 
 namespace cg = cooperative_groups;
@@ -81,6 +84,10 @@ static_assert(kXoRowBytes % 16 == 0 && kRecvOff % 16 == 0, "bulk copies need 16-
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
+  // timeline marks: 2 wait returned, 3 query and first K/V tile in shared
+  // memory, 4 O complete, 5 cluster barrier passed, 6 peers' rows received,
+  // 7 combined
+  DLM_TRACE_CTA(TRACE_ATTENTION);
   // Before the wait for the previous kernel this CTA reads only data of
   // kernels that finished before that one started (cache lengths, done
   // flags, the active count; read through L2, where no stale copy can be
@@ -158,6 +165,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   pdl_wait_then_release();
+  if (tid == 0) DLM_TRACE_MARK(2);
   if (q_by_tma) {
     // the query tile: positions b*C + rt*128/G .., the G heads of KV head g,
     // two 64-column halves with the 128-byte swizzle; rows past R (the next
@@ -238,6 +246,7 @@ __global__ void __launch_bounds__(192, 1)
       };
       bool ok = n_tiles > 0 && (!q_by_tma || mbar_wait_bounded(q_full, 0, abort_flag)) &&
                 mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+      DLM_TRACE_MARK(3);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -355,6 +364,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait_bounded(pv_done, (uint32_t)((n_tiles - 1) & 1), abort_flag)) {
       tc_fence_after();
       have = true;
+      if (row == 0) DLM_TRACE_MARK(4);
       {
         uint32_t raw[kDh / 32][32];
 #pragma unroll
@@ -421,6 +431,7 @@ __global__ void __launch_bounds__(192, 1)
     // its own shared memory
     if (tid == 0) mbar_arrive_expect_tx(rx, (uint32_t)((n - 1) * (r1 - r0) * kXoRowBytes));
     cluster.sync();   // rows written, receive barriers armed
+    if (tid == 0) DLM_TRACE_MARK(5);
     if (tid < n && tid != q) {
       const int a0 = min(kRowsCta, tid * per), a1 = min(kRowsCta, a0 + per);
       if (a1 > a0)
@@ -431,6 +442,7 @@ __global__ void __launch_bounds__(192, 1)
     // the copies into this CTA land before it reads them -- or, after an
     // abort, before it exits
     if (!mbar_wait_bounded(rx, 0, abort_flag)) mbar_wait_bounded(rx, 0, nullptr);
+    if (tid == 0) DLM_TRACE_MARK(6);
     const float* xo_p[kMaxCluster];   // split j's row r0 + i: xo_p[j] + i * kXoStride
 #pragma unroll
     for (int j = 0; j < kMaxCluster; ++j)
@@ -471,6 +483,7 @@ __global__ void __launch_bounds__(192, 1)
       w2.y = pack_bf16(acc.z * inv, acc.w * inv);
       *reinterpret_cast<uint2*>(dst) = w2;
     }
+    if (tid == 0) DLM_TRACE_MARK(7);
     // every copy into every CTA of the cluster has landed (each CTA arrives
     // after its receive barrier): the rows may be released
     cluster.sync();
@@ -493,7 +506,9 @@ __global__ void attn_combine_kernel(const float* __restrict__ opart, const float
                                     __nv_bfloat16* __restrict__ o, const int32_t* __restrict__ lens,
                                     const uint8_t* __restrict__ done, const int* n_active, int H,
                                     int Hkv, int G, int C, int R, int chunk, int nsplit) {
+  DLM_TRACE_CTA(TRACE_ATTN_COMBINE);
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (n_active != nullptr && *n_active == 0) return;
   const int bg = blockIdx.x;
   const int b = bg / Hkv, g = bg - b * Hkv;

@@ -399,6 +399,58 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Device timeline, compiled in with -DDLM_TRACE only (every macro below is
+// empty otherwise).  Each kernel of the step stamps %globaltimer (ns) per
+// CTA into a table [kTraceKinds][kTraceCtas][kTraceSlots] of its translation
+// unit: slot 0 the CTA's entry, 1 its exit (the last warp out), 2 the
+// programmatic-launch wait returned, 3.. phases of the kernel.  The last
+// launch of each kind is what the table holds.
+// ---------------------------------------------------------------------------
+constexpr int kTraceKinds = 16;
+constexpr int kTraceCtas = 512;
+constexpr int kTraceSlots = 8;
+#ifdef DLM_TRACE
+__device__ __forceinline__ unsigned long long trace_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+struct TraceCta {
+  unsigned long long* row;
+  __device__ TraceCta(unsigned long long* table, int kind) {
+    const unsigned cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    row = (kind >= 0 && kind < kTraceKinds && cta < (unsigned)kTraceCtas)
+              ? table + ((size_t)kind * kTraceCtas + cta) * kTraceSlots
+              : nullptr;
+    if (row != nullptr && threadIdx.x == 0) row[0] = trace_now();
+  }
+  __device__ ~TraceCta() {
+    if (row != nullptr && (threadIdx.x & 31) == 0) atomicMax(row + 1, trace_now());
+  }
+  __device__ void mark(int slot) const {
+    if (row != nullptr) row[slot] = trace_now();
+  }
+};
+// the table of one translation unit and its host-side copy / clear
+#define DLM_TRACE_STORAGE(tu)                                                      \
+  static __device__ unsigned long long g_trace_tab[kTraceKinds * kTraceCtas * kTraceSlots]; \
+  cudaError_t trace_copy_##tu(unsigned long long* host) {                          \
+    return cudaMemcpyFromSymbol(host, g_trace_tab, sizeof(g_trace_tab));           \
+  }                                                                                \
+  cudaError_t trace_clear_##tu() {                                                 \
+    void* p = nullptr;                                                             \
+    cudaError_t e = cudaGetSymbolAddress(&p, g_trace_tab);                         \
+    return e != cudaSuccess ? e : cudaMemset(p, 0, sizeof(g_trace_tab));           \
+  }
+#define DLM_TRACE_CTA(kind) const TraceCta dlm_trace_cta(g_trace_tab, (kind))
+#define DLM_TRACE_MARK(slot) dlm_trace_cta.mark(slot)
+#else
+#define DLM_TRACE_STORAGE(tu)
+#define DLM_TRACE_CTA(kind) ((void)0)
+#define DLM_TRACE_MARK(slot) ((void)0)
+#endif
+
+// ---------------------------------------------------------------------------
 // programmatic dependent launch: a kernel of the step may start (and run its
 // shared-memory / TMEM prologue) while its predecessor finishes; before it
 // touches global memory it waits for the predecessor to complete, and only

@@ -519,6 +519,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.out = ctx->part;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
+    io.trace_kind = TRACE_QKV_GEMM;
     const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
     if (fused) {
       pl.epi = EPI_QKV;
@@ -557,6 +558,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.out = ctx->part;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
+    io.trace_kind = TRACE_WO_GEMM;
     const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
     if (fused) {
       pl.epi = EPI_RESID;
@@ -582,6 +584,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.done = c->done;
     io.n_active = ctx->n_active;
     io.err = ctx->err;
+    io.trace_kind = TRACE_LM_HEAD;
     if (ctx->lm_f8) {
       // e4m3 head: the rows are quantised first, the scales enter the epilogue
       e = quantize_rows_e4m3(ctx->y, rows, md.d, ctx->yq, ctx->s_y, C, c->done, ctx->n_active,
@@ -1132,6 +1135,56 @@ int dlm_set_stage_events(dlm_ctx* ctx, int stage, void* const* events, int n_pai
 
 const char* dlm_last_error(const dlm_ctx* ctx) {
   return ctx ? ctx->msg.c_str() : g_create_error.c_str();
+}
+
+int dlm_trace_layout(int* kinds, int* ctas, int* slots) {
+  if (kinds == nullptr || ctas == nullptr || slots == nullptr)
+    return fail(nullptr, DLM_EINVAL, "trace_layout: NULL pointer argument");
+  *kinds = kTraceKinds;
+  *ctas = kTraceCtas;
+  *slots = kTraceSlots;
+#ifdef DLM_TRACE
+  return DLM_OK;
+#else
+  return fail(nullptr, DLM_ESTATE, "trace: the library was built without DLM_TRACE");
+#endif
+}
+
+int dlm_trace_read(unsigned long long* table, size_t words) {
+  const size_t n = (size_t)kTraceKinds * kTraceCtas * kTraceSlots;
+  if (table == nullptr || words < n)
+    return fail(nullptr, DLM_EINVAL, "trace_read: table NULL or smaller than the layout");
+#ifdef DLM_TRACE
+  if (cudaError_t e = cudaDeviceSynchronize(); e != cudaSuccess)
+    return cuda_fail(nullptr, "trace_read", e);
+  // the tables of the translation units hold disjoint kinds: merge by max
+  std::vector<unsigned long long> part(n);
+  std::fill(table, table + n, 0ull);
+  cudaError_t (*copies[])(unsigned long long*) = {trace_copy_gemm, trace_copy_simt, trace_copy_attn,
+                                                  trace_copy_misc, trace_copy_sel};
+  for (auto copy : copies) {
+    if (cudaError_t e = copy(part.data()); e != cudaSuccess)
+      return cuda_fail(nullptr, "trace_read", e);
+    for (size_t i = 0; i < n; ++i) table[i] = std::max(table[i], part[i]);
+  }
+  return DLM_OK;
+#else
+  return fail(nullptr, DLM_ESTATE, "trace: the library was built without DLM_TRACE");
+#endif
+}
+
+int dlm_trace_clear(void) {
+#ifdef DLM_TRACE
+  cudaError_t (*clears[])() = {trace_clear_gemm, trace_clear_simt, trace_clear_attn,
+                               trace_clear_misc, trace_clear_sel};
+  for (auto clear : clears)
+    if (cudaError_t e = clear(); e != cudaSuccess) return cuda_fail(nullptr, "trace_clear", e);
+  if (cudaError_t e = cudaDeviceSynchronize(); e != cudaSuccess)
+    return cuda_fail(nullptr, "trace_clear", e);
+  return DLM_OK;
+#else
+  return fail(nullptr, DLM_ESTATE, "trace: the library was built without DLM_TRACE");
+#endif
 }
 
 }  // extern "C"

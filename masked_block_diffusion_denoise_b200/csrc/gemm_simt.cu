@@ -5,6 +5,9 @@
 #include "kernels.h"
 
 namespace dlm {
+
+DLM_TRACE_STORAGE(simt)
+
 namespace {
 
 constexpr int kT = 64;
@@ -17,13 +20,16 @@ struct SimtParams {
   LmEpi epi;
   const uint8_t* done;
   const int* n_active;
+  int trace_kind;
 };
 
 template <int EPI>
 __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A,
                                                        const float* __restrict__ B,
                                                        const SimtParams p) {
+  DLM_TRACE_CTA(p.trace_kind);
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (p.n_active != nullptr && *p.n_active == 0) return;
   __shared__ float As[kTK][kT + 4];
   __shared__ float Bs[kTK][kT + 4];
@@ -117,6 +123,7 @@ cudaError_t gemm_f32(const float* A, const float* B, const GemmPlan& plan, const
   p.epi.n_tiles = p.n_tiles;
   p.done = io.done;
   p.n_active = io.n_active;
+  p.trace_kind = io.trace_kind;
   dim3 grid(p.n_tiles, (plan.M + kT - 1) / kT, plan.epi == EPI_LM ? 1 : plan.splits);
   if (plan.epi == EPI_LM) return launch_pdl(gemm_f32_kernel<EPI_LM>, grid, dim3(256), 0, st, A, B, p);
   return launch_pdl(gemm_f32_kernel<EPI_F32>, grid, dim3(256), 0, st, A, B, p);

@@ -31,6 +31,9 @@
 #include "lm_epilogue.cuh"
 
 namespace dlm {
+
+DLM_TRACE_STORAGE(gemm)
+
 namespace {
 
 constexpr int kBM = 128;
@@ -77,6 +80,7 @@ struct TcParams {
   const uint8_t* done;   // [B] canvases that are finished (LM rows skipped)
   const int* n_active;   // whole launch skipped when *n_active == 0
   int* err;
+  int trace_kind;        // device timeline (DLM_TRACE builds), -1: not traced
 };
 
 __device__ __forceinline__ void unit_coords(const TcParams& p, int u, int& m, int& n, int& kb0,
@@ -138,6 +142,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
   constexpr int kBKe = F8 ? 2 * kBK : kBK;   // elements per k-block
+  // timeline marks: 2 wait returned, 3 / 4 first / last ring stage full,
+  // 5 first accumulator ready, 6 last tile's epilogue done
+  DLM_TRACE_CTA(p.trace_kind);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -201,6 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // the prologue above touched only shared and tensor memory and weights
   pdl_wait_then_release();
   if (warp == 0 && lane == 0) {
+    DLM_TRACE_MARK(2);
     // the A tiles of the stages whose B tiles are in flight (the A buffer is
     // always allocated, so these loads are issued even when the step turns
     // out to have nothing to do)
@@ -283,6 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          if (it == 0 && kb == kb0) DLM_TRACE_MARK(3);
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + stage * stage_bytes);
           const uint32_t sa = sb + Cfg::kBBytes;
@@ -303,6 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (!ok) break;
+        DLM_TRACE_MARK(4);
         umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
@@ -341,6 +351,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int it = 0; get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag)) break;
+      if (it == 0 && warp == 2 && lane == 0) DLM_TRACE_MARK(5);
       tc_fence_after();
       const int row0 = m * kBM + quad * 32;
       const int row = row0 + lane;
@@ -476,6 +487,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
+      if (warp == 2 && lane == 0) DLM_TRACE_MARK(6);
       if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -556,6 +568,7 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.done = io.done;
   p.n_active = io.n_active;
   p.err = io.err;
+  p.trace_kind = io.trace_kind;
   if (plan.f8) {
     // e4m3 operands: the LM head and its full-logit inspection only
     if (plan.epi == EPI_LM)

@@ -36,6 +36,34 @@ struct ProjEpi {
   void* y = nullptr;                 // EPI_RESID: [M][N]
 };
 
+// Device timeline (DLM_TRACE builds): one kind per kernel of the step
+enum TraceKind {
+  TRACE_EMBED = 0,
+  TRACE_QKV_GEMM = 1,
+  TRACE_QKV_EPILOGUE = 2,
+  TRACE_ATTENTION = 3,
+  TRACE_ATTN_COMBINE = 4,
+  TRACE_WO_GEMM = 5,
+  TRACE_WO_EPILOGUE = 6,
+  TRACE_QUANTIZE = 7,
+  TRACE_LM_HEAD = 8,
+  TRACE_COMMIT = 9,
+  TRACE_KINDS_USED = 10
+};
+#ifdef DLM_TRACE
+// each translation unit's table (see DLM_TRACE_STORAGE)
+cudaError_t trace_copy_gemm(unsigned long long* host);
+cudaError_t trace_clear_gemm();
+cudaError_t trace_copy_simt(unsigned long long* host);
+cudaError_t trace_clear_simt();
+cudaError_t trace_copy_attn(unsigned long long* host);
+cudaError_t trace_clear_attn();
+cudaError_t trace_copy_misc(unsigned long long* host);
+cudaError_t trace_clear_misc();
+cudaError_t trace_copy_sel(unsigned long long* host);
+cudaError_t trace_clear_sel();
+#endif
+
 struct GemmIO {
   float* out = nullptr;        // EPI_F32: [splits][M][N]
   float* part = nullptr;       // EPI_LM:  [M][kLmFields][n_part]
@@ -44,6 +72,7 @@ struct GemmIO {
   const uint8_t* done = nullptr;
   const int* n_active = nullptr;
   int* err = nullptr;
+  int trace_kind = -1;         // TraceKind of this launch, -1: not traced
 };
 
 // ---- gemm_tc.cu: bf16 tcgen05 GEMM ---------------------------------------

@@ -6,6 +6,9 @@
 #include "kernels.h"
 
 namespace dlm {
+
+DLM_TRACE_STORAGE(misc)
+
 namespace {
 
 // cos/sin of pos * theta^(-2j/Dh), evaluated in double precision (positions
@@ -24,7 +27,9 @@ template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ emb,
                              T* __restrict__ x, int rows, int C, int d, int V, int B,
                              const uint8_t* __restrict__ done, int* n_active, int* err) {
+  DLM_TRACE_CTA(TRACE_EMBED);
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   // this row's done flag and token are loaded together (and with block 0's
   // loads of every canvas's flag for the active count)
   const int r = blockIdx.x;
@@ -65,6 +70,7 @@ __global__ void __launch_bounds__(256)
                         int seq_fixed, int head0, const int32_t* __restrict__ lens,
                         const float2* __restrict__ rope, T* __restrict__ q, T* __restrict__ kc,
                         T* __restrict__ vc, const uint8_t* __restrict__ done, const int* n_active) {
+  DLM_TRACE_CTA(seq_fixed < 0 ? TRACE_QKV_EPILOGUE : -1);
   const int r = blockIdx.x;
   const int half = md.Dh / 2;
   int seq, p_in;
@@ -91,6 +97,7 @@ __global__ void __launch_bounds__(256)
   float2 cs = make_float2(1.f, 0.f);
   if (active && rotate) cs = rope[(size_t)pos * half + j];
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (!active) return;
   {
     const int cb = hl * md.Dh;
@@ -126,6 +133,7 @@ template <typename T>
 __global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, int rows, int d,
                                    int C, const T* __restrict__ x, T* __restrict__ y,
                                    const uint8_t* __restrict__ done, const int* n_active) {
+  DLM_TRACE_CTA(TRACE_WO_EPILOGUE);
   const int r = blockIdx.y;
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const size_t i = (size_t)r * d + c;
@@ -133,6 +141,7 @@ __global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, i
   const bool dn = done != nullptr && __ldcg(done + r / C) != 0;
   const float xv = c < d ? to_f32(__ldcg(x + i)) : 0.f;
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (na == 0 || dn || c >= d) return;
   float acc = 0.f;
   for (int s = 0; s < splits; ++s) acc += part[((size_t)s * rows + r) * d + c];
@@ -166,7 +175,9 @@ __global__ void add_len_all_kernel(int32_t* lens, int B, int n) {
 __global__ void __launch_bounds__(256) quantize_rows_kernel(
     const __nv_bfloat16* __restrict__ x, int rows, int cols, uint8_t* __restrict__ q,
     float* __restrict__ scale, int C, const uint8_t* __restrict__ done, const int* n_active) {
+  DLM_TRACE_CTA(TRACE_QUANTIZE);
   pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (n_active != nullptr && *n_active == 0) return;
   const int r = blockIdx.x;
   if (r >= rows || (done != nullptr && done[r / C])) return;

@@ -12,6 +12,9 @@
 #include "kernels.h"
 
 namespace dlm {
+
+DLM_TRACE_STORAGE(sel)
+
 namespace {
 
 // combine the n_part partials of one row (a warp) into cand / conf / entropy:
@@ -140,6 +143,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
+  // timeline marks: 2 wait returned, 3 rows reduced, 4 keys sorted, 5 done
+  DLM_TRACE_CTA(TRACE_COMMIT);
   // Inside a step (partials given) the direct predecessor is the LM head,
   // which writes only the partials: the active count and the canvas state
   // come from earlier kernels, complete once this kernel may start (every
@@ -185,6 +190,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     }
   }
   if (early) pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (na == 0 || dn) return;
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
@@ -211,6 +217,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     com[i] = com_r;
   }
   __syncthreads();
+  if (i == 0) DLM_TRACE_MARK(3);
 
   int fill0 = 0, fill1 = 0;
   const int e0 = eos_fill(tok, com, C, a.eos_id, &e_s, &fill0);
@@ -333,6 +340,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   }
 
   if (i == 0) {
+    DLM_TRACE_MARK(4);
     int k;
     if (a.eb) {
       k = 0;
@@ -382,6 +390,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   }
   const int all = __syncthreads_and(i >= C || com[i]);
   if (i == 0) {
+    DLM_TRACE_MARK(5);
     done[b] = all ? 1 : 0;
     step[b] = s + 1;
     eos_pos[b] = e;
