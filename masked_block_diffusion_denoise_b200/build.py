@@ -7,7 +7,9 @@ arch=compute_100a,code=sm_100a -lineinfo) and links one shared library
 against the shared CUDA runtime.  Sources are recompiled only when they, or a
 header, are newer than their object file.  --trace builds the device-timeline
 variant instead (-DDLM_TRACE, libdlm_trace.so; see dlm_trace_read in
-include/dlm.h).
+include/dlm.h); --bounds the index-checking variant (-DDLM_DEBUG_BOUNDS,
+libdlm_bounds.so: accesses whose index comes from device data are checked
+and a violation is reported as DLM_EBOUNDS instead of being made).
 """
 from __future__ import annotations
 
@@ -24,6 +26,8 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdlm.so")
 BUILD_TRACE = os.path.join(HERE, "_build_trace")
 LIB_TRACE = os.path.join(HERE, "libdlm_trace.so")
+BUILD_BOUNDS = os.path.join(HERE, "_build_bounds")
+LIB_BOUNDS = os.path.join(HERE, "libdlm_bounds.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -53,9 +57,15 @@ def _compile(src, obj, verbose, extra=()):
     return r.stderr
 
 
-def build(jobs: int = 0, verbose: bool = False, trace: bool = False) -> str:
-    build_dir, lib = (BUILD_TRACE, LIB_TRACE) if trace else (BUILD, LIB)
-    extra = ["-DDLM_TRACE"] if trace else []
+def build(jobs: int = 0, verbose: bool = False, trace: bool = False,
+          bounds: bool = False) -> str:
+    if trace and bounds:
+        raise ValueError("one variant at a time: trace or bounds")
+    build_dir, lib, extra = BUILD, LIB, []
+    if trace:
+        build_dir, lib, extra = BUILD_TRACE, LIB_TRACE, ["-DDLM_TRACE"]
+    if bounds:
+        build_dir, lib, extra = BUILD_BOUNDS, LIB_BOUNDS, ["-DDLM_DEBUG_BOUNDS"]
     os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest = max(os.path.getmtime(h) for h in _headers())
@@ -86,5 +96,7 @@ if __name__ == "__main__":
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--trace", action="store_true",
                     help="the device-timeline variant (libdlm_trace.so)")
+    ap.add_argument("--bounds", action="store_true",
+                    help="the index-checking variant (libdlm_bounds.so)")
     a = ap.parse_args()
-    print(build(a.jobs, a.verbose, a.trace))
+    print(build(a.jobs, a.verbose, a.trace, a.bounds))

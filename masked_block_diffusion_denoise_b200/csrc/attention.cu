@@ -54,6 +54,7 @@ struct AttnParams {
   int H, Hkv, G, C, R, chunk, nsplit;
   int cluster;   // > 1: the nsplit CTAs of a (row tile, plane) form a cluster and combine in it
   int q_tma;     // the query tile by TMA (tmQ: q as [positions][H][Dh], box 64 x G x 128/G)
+  int Lcap;      // key slots per plane in the cache
   float scale_log2;
 };
 
@@ -101,6 +102,8 @@ __global__ void __launch_bounds__(192, 1)
   const int len_b = __ldcg(p.lens + b);
   if (na == 0 || dn) return;
   const int n_keys = len_b + p.C;
+  // a cluster's CTAs share the plane, so this exit is uniform over a cluster
+  if (!DLM_IN_BOUNDS(n_keys - 1, p.Lcap, p.err)) return;
   const int k_begin = split * p.chunk;
   // a split past the keys exits at once, except in a cluster, where it still
   // takes part in the exchange (with no rows of its own)
@@ -576,7 +579,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(int H, int Hkv, int C, in
                                                        float* __restrict__ o,
                                                        const int32_t* __restrict__ lens,
                                                        const uint8_t* __restrict__ done,
-                                                       const int* n_active, float scale) {
+                                                       const int* n_active, float scale,
+                                                       int* err) {
   pdl_wait_then_release();
   if (n_active != nullptr && *n_active == 0) return;
   constexpr int KT = 32;
@@ -586,6 +590,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(int H, int Hkv, int C, in
   if (done != nullptr && done[b]) return;
   const int g = h / (H / Hkv);
   const int n_keys = lens[b] + C;
+  if (!DLM_IN_BOUNDS(n_keys - 1, Lcap, err)) return;
   const float* kbase = kc + ((size_t)b * Hkv + g) * Lcap * DH;
   const float* vbase = vc + ((size_t)b * Hkv + g) * Lcap * DH;
   for (int i0 = 0; i0 < C; i0 += blockDim.x) {
@@ -674,6 +679,7 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.nsplit = ap.nsplit;
   p.cluster = ap.cluster;
   p.q_tma = tmQ != nullptr && ap.G > 0 && kRowsCta % ap.G == 0 ? 1 : 0;
+  p.Lcap = md.Lcap;
   const CUtensorMap qmap = tmQ != nullptr ? *tmQ : tmK;   // unread without q_tma
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
@@ -740,19 +746,20 @@ int attn_cluster_capacity(int n) {
 
 cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,
                           const float* vcache, float* o, const int32_t* lens,
-                          const uint8_t* done, const int* n_active, cudaStream_t st) {
+                          const uint8_t* done, const int* n_active, int* err,
+                          cudaStream_t st) {
   const float scale = (float)(1.0 / sqrt((double)md.Dh));
   const int threads = 128;
   cudaError_t e;
   if (md.Dh == 64)
     e = launch_pdl(attn_f32_kernel<64>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
-                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale, err);
   else if (md.Dh == 128)
     e = launch_pdl(attn_f32_kernel<128>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
-                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale, err);
   else if (md.Dh == 32)
     e = launch_pdl(attn_f32_kernel<32>, dim3(B * md.H), dim3(threads), 0, st, md.H, md.Hkv, C,
-                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale);
+                   md.Lcap, q, kcache, vcache, o, lens, done, n_active, scale, err);
   else
     return cudaErrorInvalidValue;
   return e;

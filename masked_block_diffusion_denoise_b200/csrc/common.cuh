@@ -35,6 +35,21 @@ __device__ __forceinline__ void raise_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// Index check of the DLM_DEBUG_BOUNDS build (the stand-in for a memory
+// checker): at every global access whose index comes from device data (cache
+// lengths), true when 0 <= i < n; otherwise DLM_EBOUNDS is recorded and the
+// caller skips the access.  The default build compiles it to `true`.
+#ifdef DLM_DEBUG_BOUNDS
+__device__ __forceinline__ bool dlm_in_bounds(long long i, long long n, int* err) {
+  if (i >= 0 && i < n) return true;
+  raise_error(err, DLM_EBOUNDS);
+  return false;
+}
+#define DLM_IN_BOUNDS(i, n, err) dlm_in_bounds((long long)(i), (long long)(n), (err))
+#else
+#define DLM_IN_BOUNDS(i, n, err) true
+#endif
+
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): per round the words 0
 // and 2 are multiplied by the two round constants; the high halves are mixed

@@ -529,7 +529,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     if (int rc = run_gemm(ctx, ctx->x, ctx->w_qkv, ctx->Nqkv, pl, io, st)) return rc;
     if (!fused) {
       e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
-                       ctx->kc, ctx->vc, c->done, ctx->n_active, st);
+                       ctx->kc, ctx->vc, c->done, ctx->n_active, ctx->err, st);
       if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue", e);
       ++ctx->launches;
     }
@@ -545,7 +545,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
   } else {
     e = attention_f32(md, batch, C, (const float*)ctx->q, (const float*)ctx->kc,
                       (const float*)ctx->vc, (float*)ctx->o, ctx->lens_d, c->done,
-                      ctx->n_active, st);
+                      ctx->n_active, ctx->err, st);
     ++ctx->launches;
   }
   if (e != cudaSuccess) return cuda_fail(ctx, "attention", e);
@@ -632,7 +632,7 @@ int enqueue_clean_pass(dlm_ctx* ctx, const int32_t* tokens, int batch, int C, cu
   if (int rc = run_gemm(ctx, ctx->x, ctx->w_qkv, ctx->Nqkv, pl, io, st)) return rc;
   if (!fused) {
     e = qkv_epilogue(md, ctx->part, pl.splits, rows, C, -1, 0, ctx->lens_d, ctx->rope, ctx->q,
-                     ctx->kc, ctx->vc, nullptr, nullptr, st);
+                     ctx->kc, ctx->vc, nullptr, nullptr, ctx->err, st);
     if (e != cudaSuccess) return cuda_fail(ctx, "qkv epilogue (clean pass)", e);
   }
   e = add_len_all(ctx->lens_d, batch, C, st);
@@ -830,7 +830,7 @@ int dlm_kv_append(dlm_ctx* ctx, int seq, int n, const int32_t* tokens, const voi
   const ModelDims& md = ctx->md;
   if (tokens == nullptr) {
     if (k == nullptr || v == nullptr) return fail(ctx, DLM_EINVAL, "need tokens or k and v");
-    CK(kv_copy_in(md, seq, n, k, v, ctx->lens_d, ctx->kc, ctx->vc, st));
+    CK(kv_copy_in(md, seq, n, k, v, ctx->lens_d, ctx->kc, ctx->vc, ctx->err, st));
     CK(add_len(ctx->lens_d, seq, n, st));
   } else {
     const int Nkv = 2 * md.Hkv * md.Dh;
@@ -845,7 +845,7 @@ int dlm_kv_append(dlm_ctx* ctx, int seq, int n, const int32_t* tokens, const voi
       io.err = ctx->err;
       if (int rc = run_gemm(ctx, ctx->x, wkv, Nkv, pl, io, st)) return rc;
       CK(qkv_epilogue(md, ctx->part, pl.splits, rows, rows, seq, md.H, ctx->lens_d, ctx->rope,
-                      nullptr, ctx->kc, ctx->vc, nullptr, nullptr, st));
+                      nullptr, ctx->kc, ctx->vc, nullptr, nullptr, ctx->err, st));
       CK(add_len(ctx->lens_d, seq, rows, st));
     }
   }

@@ -398,8 +398,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
           for (int hc = cb / 128; hc < (cb + kHalfN) / 128; ++hc) {
             const int head = (n * BN) / 128 + hc;
-            const bool store = live && head < pe.H + 2 * pe.Hkv;
+            bool store = live && head < pe.H + 2 * pe.Hkv;
             const int pos = store ? pe.lens[seq] + p_in : 0;
+            if (store && !DLM_IN_BOUNDS(pos, pe.Lcap, p.err)) store = false;
             __nv_bfloat16* dst = nullptr;
             if (store) {
               if (head < pe.H) {

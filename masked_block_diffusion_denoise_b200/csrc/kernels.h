@@ -111,7 +111,7 @@ cudaError_t embed_rows(const ModelDims& md, const int32_t* tokens, const void* e
 cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
                          int seq_fixed, int head0, const int32_t* lens, const float2* rope,
                          void* q, void* kcache, void* vcache, const uint8_t* done,
-                         const int* n_active, cudaStream_t st);
+                         const int* n_active, int* err, cudaStream_t st);
 
 // y = x + sum of split-K partials of o W_o^T
 cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
@@ -120,7 +120,8 @@ cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int 
 
 // copy caller K/V [Hkv][n][Dh] into the cache of `seq` at slots lens[seq]..
 cudaError_t kv_copy_in(const ModelDims& md, int seq, int n, const void* k, const void* v,
-                       const int32_t* lens, void* kcache, void* vcache, cudaStream_t st);
+                       const int32_t* lens, void* kcache, void* vcache, int* err,
+                       cudaStream_t st);
 
 cudaError_t add_len(int32_t* lens, int seq, int n, cudaStream_t st);
 
@@ -158,7 +159,8 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
 // fp32: one thread per query row
 cudaError_t attention_f32(const ModelDims& md, int B, int C, const float* q, const float* kcache,
                           const float* vcache, float* o, const int32_t* lens,
-                          const uint8_t* done, const int* n_active, cudaStream_t st);
+                          const uint8_t* done, const int* n_active, int* err,
+                          cudaStream_t st);
 
 // ---- select.cu ------------------------------------------------------------------
 struct SelectArgs {

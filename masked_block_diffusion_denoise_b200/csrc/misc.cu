@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(256)
     qkv_epilogue_kernel(ModelDims md, const float* __restrict__ part, int splits, int rows, int C,
                         int seq_fixed, int head0, const int32_t* __restrict__ lens,
                         const float2* __restrict__ rope, T* __restrict__ q, T* __restrict__ kc,
-                        T* __restrict__ vc, const uint8_t* __restrict__ done, const int* n_active) {
+                        T* __restrict__ vc, const uint8_t* __restrict__ done, const int* n_active,
+                        int* err) {
   DLM_TRACE_CTA(seq_fixed < 0 ? TRACE_QKV_EPILOGUE : -1);
   const int r = blockIdx.x;
   const int half = md.Dh / 2;
@@ -89,12 +90,13 @@ __global__ void __launch_bounds__(256)
   const int ncols = nheads * md.Dh;
   const int per_block = blockDim.x / half;
   const int item = blockIdx.y * per_block * half + threadIdx.x;
-  const bool active = na != 0 && !dn && item < nheads * half;
+  bool active = na != 0 && !dn && item < nheads * half;
   const int hl = item / half, j = item - hl * half;
   const int hh = hl + head0;
   const int pos = len + p_in;
   const bool rotate = rope != nullptr && hh < md.H + md.Hkv;
   float2 cs = make_float2(1.f, 0.f);
+  if (active && !DLM_IN_BOUNDS(pos, md.Lcap, err)) active = false;
   if (active && rotate) cs = rope[(size_t)pos * half + j];
   pdl_wait_then_release();
   if (threadIdx.x == 0) DLM_TRACE_MARK(2);
@@ -151,9 +153,10 @@ __global__ void wo_epilogue_kernel(const float* __restrict__ part, int splits, i
 template <typename T>
 __global__ void kv_copy_kernel(int Hkv, int Lcap, int Dh, int seq, int n,
                                const T* __restrict__ k, const T* __restrict__ v,
-                               const int32_t* __restrict__ lens, T* kc, T* vc) {
+                               const int32_t* __restrict__ lens, T* kc, T* vc, int* err) {
   const int g = blockIdx.x, j = blockIdx.y;
   const int pos = lens[seq] + j;
+  if (!DLM_IN_BOUNDS(pos, Lcap, err)) return;
   const size_t src = ((size_t)g * n + j) * Dh;
   const size_t dst = (((size_t)seq * Hkv + g) * Lcap + pos) * Dh;
   for (int t = threadIdx.x; t < Dh; t += blockDim.x) {
@@ -262,17 +265,17 @@ cudaError_t embed_rows(const ModelDims& md, const int32_t* tokens, const void* e
 cudaError_t qkv_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
                          int seq_fixed, int head0, const int32_t* lens, const float2* rope,
                          void* q, void* kcache, void* vcache, const uint8_t* done,
-                         const int* n_active, cudaStream_t st) {
+                         const int* n_active, int* err, cudaStream_t st) {
   const int half = md.Dh / 2;
   const int per_block = 256 / half;   // heads per block
   dim3 grid(rows, (md.H + 2 * md.Hkv - head0 + per_block - 1) / per_block);
   if (md.esize == 2)
     return launch_pdl(qkv_epilogue_kernel<__nv_bfloat16>, grid, dim3(per_block * half), 0, st, md, part,
                       splits, rows, C, seq_fixed, head0, lens, rope, (__nv_bfloat16*)q,
-                      (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active);
+                      (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, done, n_active, err);
   return launch_pdl(qkv_epilogue_kernel<float>, grid, dim3(per_block * half), 0, st, md, part, splits,
                     rows, C, seq_fixed, head0, lens, rope, (float*)q, (float*)kcache,
-                    (float*)vcache, done, n_active);
+                    (float*)vcache, done, n_active, err);
 }
 
 cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int rows, int C,
@@ -287,17 +290,18 @@ cudaError_t wo_epilogue(const ModelDims& md, const float* part, int splits, int 
 }
 
 cudaError_t kv_copy_in(const ModelDims& md, int seq, int n, const void* k, const void* v,
-                       const int32_t* lens, void* kcache, void* vcache, cudaStream_t st) {
+                       const int32_t* lens, void* kcache, void* vcache, int* err,
+                       cudaStream_t st) {
   dim3 grid(md.Hkv, n);
   const int threads = md.Dh < 128 ? md.Dh : 128;
   if (md.esize == 2)
     kv_copy_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
         md.Hkv, md.Lcap, md.Dh, seq, n, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, lens,
-        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache);
+        (__nv_bfloat16*)kcache, (__nv_bfloat16*)vcache, err);
   else
     kv_copy_kernel<float><<<grid, threads, 0, st>>>(md.Hkv, md.Lcap, md.Dh, seq, n,
                                                     (const float*)k, (const float*)v, lens,
-                                                    (float*)kcache, (float*)vcache);
+                                                    (float*)kcache, (float*)vcache, err);
   return cudaGetLastError();
 }
 
