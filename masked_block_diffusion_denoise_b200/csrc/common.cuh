@@ -385,6 +385,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // CTA of rank `rank` of this cluster, and a bulk copy from this CTA's shared
 // memory into another CTA's, completing (bytes) on an mbarrier of that CTA
 // ---------------------------------------------------------------------------
+// one contiguous copy from global memory into this CTA's shared memory by the
+// bulk-copy engine (both addresses 16-byte aligned, bytes a multiple of 16),
+// completing (bytes) on an mbarrier of this CTA
+__device__ __forceinline__ void bulk_load_global(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                                 uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t cluster_addr(uint32_t local, int rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));

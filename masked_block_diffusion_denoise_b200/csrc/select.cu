@@ -112,6 +112,8 @@ __device__ __forceinline__ uint32_t ordered_bits(float x) {
 }
 
 constexpr int kMaxC = 1024;
+constexpr int kStageChunk = 32768;        // bytes per bulk copy of the partials
+constexpr int kStageMax = 160 * 1024;     // partials staged up to this size per canvas
 
 // positions after the first committed EOS become EOS and committed; returns
 // the EOS position (or -1) and, through *filled, how many were filled
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               uint8_t* __restrict__ committed, int32_t* __restrict__ step,
                               uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
                               int32_t* __restrict__ prev_cand, int32_t* __restrict__ stable,
-                              const float* __restrict__ part, int n_part,
+                              const float* __restrict__ part, int n_part, int stage_bytes,
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
                               const int* n_active, int* err) {
@@ -152,6 +154,19 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   // and are read before the wait, through L2.  Given candidates (a call on
   // its own) the predecessor is unknown and everything is read after it.
   const bool early = part != nullptr;
+  // stage_bytes > 0: this canvas's partials ([C][kLmFields][n_part] floats)
+  // come into shared memory by bulk copies, a few instructions instead of
+  // one load per field, partial and row from one SM
+  extern __shared__ __align__(128) uint8_t stage_raw[];
+  __shared__ uint64_t stage_bar;
+  const bool staged = part != nullptr && stage_bytes > 0;
+  if (staged) {
+    if (threadIdx.x == 0) {
+      mbar_init(&stage_bar, 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+  }
   if (!early) pdl_wait_then_release();
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -192,6 +207,13 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   if (early) pdl_wait_then_release();
   if (threadIdx.x == 0) DLM_TRACE_MARK(2);
   if (na == 0 || dn) return;
+  if (staged && i == 0) {
+    mbar_arrive_expect_tx(&stage_bar, (uint32_t)stage_bytes);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(part + base * kLmFields * (size_t)n_part);
+    for (int off = 0; off < stage_bytes; off += kStageChunk)
+      bulk_load_global(stage_raw + off, src + off, (uint32_t)min(kStageChunk, stage_bytes - off),
+                       &stage_bar);
+  }
   __shared__ unsigned long long keys[kMaxC];
   __shared__ int32_t tok[kMaxC];
   __shared__ uint8_t com[kMaxC];
@@ -201,10 +223,16 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   int P = 32;               // keys sorted: the next power of two >= C
   while (P < C) P <<= 1;
   if (part != nullptr) {
+    if (staged && !mbar_wait_bounded(&stage_bar, 0, nullptr)) {
+      raise_error(err, DLM_ETIMEOUT);
+      mbar_wait_bounded(&stage_bar, 0, nullptr);   // the copies land before the CTA exits
+    }
     // a6: the cross-tile reduction of this canvas's rows, one warp per row
     for (int r = warp; r < C; r += nw) {
       const size_t row = base + r;
-      reduce_row(part + row * kLmFields * (size_t)n_part, n_part, lane, cand + row, conf + row, ent + row,
+      const float* pr = staged ? reinterpret_cast<const float*>(stage_raw) + r * kLmFields * n_part
+                               : part + row * kLmFields * (size_t)n_part;
+      reduce_row(pr, n_part, lane, cand + row, conf + row, ent + row,
                  cand_s + r, conf_s + r, ent_s + r);
     }
   } else if (i < C) {
@@ -415,8 +443,21 @@ cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed
   while (P < a.C) P <<= 1;
   if (P > kMaxC) return cudaErrorInvalidValue;
   if (part != nullptr) P = 1024;   // 32 warps for the row reductions
-  return launch_pdl(commit_kernel, dim3(a.B), dim3(P), 0, st, a, tokens, committed, step, done,
-                    eos_pos, prev_cand, stable, part, n_part, cand, conf, ent, stats, n_active, err);
+  // the partials of a canvas go through shared memory when they fit and
+  // every canvas's block starts on a 16-byte boundary
+  int stage_bytes = 0;
+  if (part != nullptr) {
+    const long long bytes = (long long)a.C * kLmFields * n_part * (long long)sizeof(float);
+    if (bytes <= kStageMax && bytes % 16 == 0) stage_bytes = (int)bytes;
+  }
+  static cudaError_t attr = cudaErrorNotReady;   // per process; one device per process
+  if (attr == cudaErrorNotReady)
+    attr = cudaFuncSetAttribute(commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kStageMax);
+  if (attr != cudaSuccess) return attr;
+  return launch_pdl(commit_kernel, dim3(a.B), dim3(P), (size_t)stage_bytes, st, a, tokens,
+                    committed, step, done, eos_pos, prev_cand, stable, part, n_part, stage_bytes,
+                    cand, conf, ent, stats, n_active, err);
 }
 
 }  // namespace dlm
