@@ -169,6 +169,18 @@ def aggregate_rate(world, units_per_rank, ms_max):
 # our arm
 # ---------------------------------------------------------------------------
 
+def workload_config(workload, wl, lens, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    sh = wl.shape
+    return {"workload": workload, "batch": wl.batch, "canvas": wl.canvas,
+            "prefix": [int(min(lens)), int(max(lens))], "steps_per_block": wl.steps,
+            "threshold": wl.threshold, "quota": wl.quota_eff, "corruption": wl.corruption,
+            "d_model": sh.d_model, "heads": [sh.n_heads, sh.n_kv_heads, sh.head_dim],
+            "vocab": sh.vocab, "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2 (the LM head streams 1.07 GB of weights every step); "
+                  "no flush"}
+
+
 def run_ours(a):
     import torch
     import masked_block_diffusion_denoise_b200 as dlm
@@ -356,14 +368,7 @@ def run_ours(a):
             "dtype": ("bf16, LM head e4m3" if lm_fp8 else "bf16") if sh.dtype == "bf16" else "f32",
             "data": "synthetic: seeded random-init weights N(0,0.02), embeddings and prefix "
                     "K/V N(0,1), all-mask canvas",
-            "config": {"workload": a.workload, "batch": wl.batch, "canvas": wl.canvas,
-                       "prefix": [int(lens.min()), int(lens.max())], "steps_per_block": S,
-                       "threshold": wl.threshold, "quota": wl.quota_eff,
-                       "corruption": wl.corruption, "d_model": sh.d_model,
-                       "heads": [sh.n_heads, sh.n_kv_heads, sh.head_dim], "vocab": sh.vocab,
-                       "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (the LM head streams 1.07 GB of weights "
-                             "every step); no flush"},
+            "config": workload_config(a.workload, wl, lens, world),
             "committed_tokens_per_s": round(committed_all / (ms_max / 1e3), 1),
             "stages_us": {k: round(v, 2) for k, v in stages.items()},
             "step_algorithmic_bytes": work_["step"]["bytes"],
@@ -509,8 +514,7 @@ def run_reference(a):
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": round(1e3 * total / K, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": a.workload, "batch": wl.batch, "canvas": wl.canvas,
-                       "vocab": V},
+            "config": workload_config(a.workload, wl, W.make_prefix(wl)[0], world),
             "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": _threads(),
                              "kind": "oracle",
                              "sample": "each step: full forward to the LM-head input, LM head "
