@@ -237,6 +237,79 @@ def quantize_rows_e4m3(x) -> Tuple[np.ndarray, np.ndarray]:
     return q, s
 
 
+# ---------------------------------------------------------------------------
+# NVFP4 (the 4-bit option of the LM head; course "Diffusion LLMs" section 15
+# names NVFP4 as the Blackwell low-bit path; the pages give no recipe, so the
+# block layout below is a reading): e2m1 elements in blocks of 16 along the
+# reduction axis, one e4m3 scale per block, one float32 scale per row.
+# ---------------------------------------------------------------------------
+
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
+
+
+def round_to_e2m1(x) -> np.ndarray:
+    """Nearest value of the e2m1 format -- sign, 2 exponent bits (bias 1), 1
+    mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 -- ties to the even
+    mantissa bit; magnitudes beyond 6 saturate to 6.  Values are float64."""
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    _, e = np.frexp(a)                 # a = m * 2^e with m in [0.5, 1)
+    e = np.maximum(e - 1, 0)           # binade; below 1 the subnormal spacing
+    step = np.ldexp(1.0, e - 1)        # grid spacing: 1 mantissa bit
+    r = np.minimum(np.rint(a / step) * step, E2M1_MAX)   # rint: ties to even
+    return np.copysign(r, x)
+
+
+def quantize_rows_nvfp4(x) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """(q, sb, sr) for rows x [rows][cols] (cols a multiple of 16):
+    sr [rows] float32 = amax(row) / (448 * 6) (1 for a zero row), so that every
+    block scale is within the e4m3 range; sb [rows][cols/16] the e4m3 block
+    scales, e4m3(amax(block) / (6 * sr)) with the division in float32; q the
+    e2m1 elements, e2m1(x / (sb * sr)) with the product and the quotient in
+    float32 (0 in a block whose scale is 0).  x ~ q * sb * sr."""
+    x = np.asarray(x)
+    rows, cols = x.shape
+    if cols % NVFP4_BLOCK:
+        raise ValueError("cols must be a multiple of 16")
+    x32 = np.asarray(x, dtype=np.float32)
+    amax_r = np.abs(x32).max(axis=1)
+    sr = np.where(amax_r > 0, amax_r / np.float32(E4M3_MAX * E2M1_MAX),
+                  np.float32(1.0)).astype(np.float32)
+    xb = x32.reshape(rows, cols // NVFP4_BLOCK, NVFP4_BLOCK)
+    amax_b = np.abs(xb).max(axis=2)
+    sb = round_to_e4m3((amax_b / (np.float32(E2M1_MAX) * sr[:, None])).astype(np.float32))
+    scale = (sb.astype(np.float32) * sr[:, None]).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(scale[:, :, None] > 0, xb / scale[:, :, None], np.float32(0.0))
+    q = round_to_e2m1(ratio.astype(np.float32)).reshape(rows, cols)
+    return q, sb, sr
+
+
+def dequantize_rows_nvfp4(q, sb, sr) -> np.ndarray:
+    """q * sb * sr, float64."""
+    q = np.asarray(q, dtype=F64)
+    rows, cols = q.shape
+    s = np.repeat(np.asarray(sb, dtype=F64), NVFP4_BLOCK, axis=1) * np.asarray(sr, F64)[:, None]
+    return q * s
+
+
+def nvfp4_dot(qa, sba, sra, qb, sbb, srb) -> np.ndarray:
+    """Rows of A times rows of B, both NVFP4 along the reduction axis, the way
+    a block-scaled product runs: per block the exact sum of element products
+    times the two block scales, summed over blocks, times the two row scales.
+    Returns [rows_a][rows_b] float64."""
+    qa = np.asarray(qa, F64)
+    qb = np.asarray(qb, F64)
+    ra, cols = qa.shape
+    nb = cols // NVFP4_BLOCK
+    pa = qa.reshape(ra, nb, NVFP4_BLOCK)
+    pb = qb.reshape(qb.shape[0], nb, NVFP4_BLOCK)
+    blk = np.einsum("ikj,lkj->ilk", pa, pb)            # exact: products of e2m1 values
+    w = np.asarray(sba, F64)[:, None, :] * np.asarray(sbb, F64)[None, :, :]
+    return (blk * w).sum(axis=2) * (np.asarray(sra, F64)[:, None] * np.asarray(srb, F64)[None, :])
+
+
 @dataclass
 class ModelDims:
     d_model: int
