@@ -44,9 +44,9 @@ stores it.  Decisions that turn floats into integers take them in float32,
 the precision in which the kernel holds the values: confidence / entropy
 comparisons in the selection, the entropy prefix sum, temperature scaling.
 
-Readings of points the pages leave open are marked READING and listed in
-the design doc.  Pins (tests/test_oracle_*.py) tie every function to something
-other than itself; no function here is parity-unpinned.
+Readings of points the pages leave open are marked READING where they are
+taken.  Pins (tests/test_oracle_*.py) tie every function to something other
+than itself; no function here is parity-unpinned.
 """
 from __future__ import annotations
 
