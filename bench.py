@@ -1,17 +1,31 @@
 #!/usr/bin/env python
 """Throughput of the masked block-diffusion denoise step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 8b_b1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload batched]
     python bench.py --impl reference ...        # the CPU oracle, same line format
 
 One "step" is one denoising step over the whole batch: embed, QKV + RoPE,
 attention, output projection, fused LM-head reduction, cross-tile reduce,
-commit / re-noise.  Steps run as CUDA-graph replays of whole blocks
-(``dlm_decode_block``); a block of the 8B-shaped batch-1 workload is 32 steps.
-K steps are timed with CUDA events on the launch stream between a barrier and
-device synchronisation on both sides; with N ranks each rank decodes its own
-batch (weak scaling, no collective on the data path) and the time is the
-maximum over ranks.  Rank 0 prints one JSON line.
+commit / re-noise.  The default workload is the batched-serving shape (16
+canvases of 64 positions over prefixes of 1024-4096 keys, the 8B-class
+model), the largest single-GPU configuration.  Steps run as CUDA-graph
+replays: K steps are K // S whole blocks (``dlm_decode_block``, S steps each,
+every block from the same initial canvas) and the first K % S steps of one
+more block as one graph (``dlm_decode_steps``).  W warm-up steps (at least
+3) run the same way first; the graphs of the timed region are captured
+before it by one replay over finished canvases, which does no work.  K steps
+are timed with CUDA events on the launch stream between a barrier and device
+synchronisation on both sides; with N ranks each rank decodes its own batch
+(weak scaling, no collective on the data path) and the time is the maximum
+over ranks.  Rank 0 prints one JSON line.
+
+Besides the headline, the line carries: the LM head's roofline (HBM- or
+tensor-bound, by its arithmetic intensity) from CUDA events recorded around
+its launches inside the replayed graph; the attention + reduce/commit stages'
+achieved HBM bandwidth; ``e2e``, the same metric through the host-buffer
+entry point (``dlm_decode_block_host``: canvas state copied in and out every
+block, inside the timed region); and, at N = 1, ``configs``: one block of
+every other workload measured the same way.
 
 Inputs exceed L2: the LM head streams its 1.07 GB weight every step, so no
 L2 flush is needed between steps.
@@ -20,7 +34,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -43,12 +56,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1280)
+    ap.add_argument("--steps", type=int, default=320)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="8b_b1", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="batched", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload map of the other configurations")
     ap.add_argument("--profile", action="store_true",
                     help="a few eager steps only, for ncu captures")
     return ap.parse_args()
@@ -181,11 +196,180 @@ def workload_config(workload, wl, lens, world):
                   "no flush"}
 
 
+class Runner:
+    """One workload on one GPU: a library session with the workload's
+    weights and prefixes, a template canvas (initial state plus EOS plant)
+    and the working canvas the steps update."""
+
+    def __init__(self, wl, device, upload=None):
+        import torch
+        from masked_block_diffusion_denoise_b200.session import Session, sampler_params
+        self.torch = torch
+        self.wl = wl
+        sh = wl.shape
+        weights = W.make_weights(sh, seed=wl.seed) if upload is None else None
+        lens, toks, kp, vp = W.make_prefix(wl)
+        self.lens = [int(x) for x in lens]
+        self.sess = Session(sh, weights, max_batch=wl.batch, max_prefix=wl.prefix_cap,
+                            max_canvas=wl.canvas, device=device, upload=upload)
+        del weights
+        for b in range(wl.batch):
+            if toks is not None:
+                self.sess.kv_append_tokens(b, toks[b])
+            else:
+                n = int(lens[b])
+                self.sess.kv_append_kv(b, np.ascontiguousarray(kp[b][:, :n]),
+                                       np.ascontiguousarray(vp[b][:, :n]))
+        del kp, vp
+        self.p = sampler_params(canvas=wl.canvas, steps=wl.steps, threshold=wl.threshold,
+                                quota=wl.quota, corruption=wl.corruption,
+                                entropy_bound=wl.entropy_bound, temperature=wl.temperature,
+                                t_max=wl.t_max, t_min=wl.t_min, seed=wl.seed)
+        self.S = wl.steps
+        self.stream = torch.cuda.Stream(device)
+        self.tmpl = self.sess.new_canvas(wl.batch, wl.canvas)
+        with torch.cuda.stream(self.stream):
+            self.sess.init(self.tmpl, self.p, stream=self.stream)
+            for (b, slot) in W.make_eos_plant(wl):
+                self.tmpl.tokens[b, slot] = sh.eos_id
+                self.tmpl.committed[b, slot] = 1
+        self.stream.synchronize()
+        self.cv = self.sess.new_canvas(wl.batch, wl.canvas)
+
+    def reset(self, finished=False):
+        """The working canvas back to the initial state (or every canvas
+        marked done, so that a replay does no work)."""
+        c, t = self.cv, self.tmpl
+        for dst, src in ((c.tokens, t.tokens), (c.committed, t.committed), (c.step, t.step),
+                         (c.done, t.done), (c.eos_pos, t.eos_pos)):
+            dst.copy_(src, non_blocking=True)
+        if finished:
+            c.done.fill_(1)
+
+    def run(self, k):
+        """k steps: whole blocks, then the first k % S steps of one more
+        block, each a graph replay from the initial canvas."""
+        import masked_block_diffusion_denoise_b200 as dlm
+        full, rest = divmod(k, self.S)
+        st = self.stream
+        with self.torch.cuda.stream(st):
+            for _ in range(full):
+                self.reset()
+                self.sess.block(self.cv, self.p, stream=st)
+            if rest:
+                self.reset()
+                dlm.dlm_decode_steps(self.sess.ctx, self.cv.c, self.wl.batch, self.p, rest,
+                                     stats=self.cv.stats, stream=st)
+
+    def capture(self, k):
+        """Capture (and replay over finished canvases) the graphs run(k) uses."""
+        import masked_block_diffusion_denoise_b200 as dlm
+        full, rest = divmod(k, self.S)
+        st = self.stream
+        with self.torch.cuda.stream(st):
+            for n in ([self.S] if full else []) + ([rest] if rest else []):
+                self.reset(finished=True)
+                dlm.dlm_decode_steps(self.sess.ctx, self.cv.c, self.wl.batch, self.p, n,
+                                     stats=self.cv.stats, stream=st)
+        st.synchronize()
+
+    def timed(self, k):
+        """Device time (ms) of run(k) on the launch stream."""
+        torch = self.torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        self.run(k)
+        e1.record(self.stream)
+        self.stream.synchronize()
+        return e0.elapsed_time(e1)
+
+    def stage_us(self, stage, n_blocks):
+        """Mean duration (us) of one stage over the S steps of a block, from
+        events recorded around it inside the replayed graph (after n_blocks
+        blocks of replays, the last one read)."""
+        import masked_block_diffusion_denoise_b200 as dlm
+        torch = self.torch
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * self.S)]
+        for e in evs:            # torch creates the CUDA event on its first record
+            e.record(self.stream)
+        self.stream.synchronize()
+        dlm.dlm_set_stage_events(self.sess.ctx, stage, [e.cuda_event for e in evs])
+        self.run(n_blocks * self.S)
+        self.stream.synchronize()
+        dlm.dlm_set_stage_events(self.sess.ctx, 0, [])
+        return [1e3 * evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(self.S)]
+
+    def plan(self):
+        import masked_block_diffusion_denoise_b200 as dlm
+        if self.wl.shape.dtype != "bf16":
+            return None
+        return dlm.dlm_attention_plan(self.sess.ctx, self.wl.batch, self.wl.canvas)
+
+    def close(self):
+        self.sess.close()
+
+
+STAGES = ["embed", "qkv", "attention", "wo", "lm_head", "reduce+commit"]
+
+
+def kernel_figures(r, pk, n_blocks):
+    """Per-stage event times of one block and the rooflines they give: the
+    LM head against HBM or the bf16 tensor peak (by its arithmetic
+    intensity), attention + reduce/commit against HBM."""
+    wl = r.wl
+    sh = wl.shape
+    # a stage of a finished canvas does no work: average over the steps in
+    # which every canvas was still active (the first steps of the block)
+    times = {name: r.stage_us(i, n_blocks) for i, name in enumerate(STAGES)}
+    n_full = r.S
+    for (b, slot) in W.make_eos_plant(wl):
+        # the `slot` positions before a planted EOS take ceil(slot / quota) steps
+        n_full = min(n_full, max(1, -(-slot // max(1, wl.quota_eff))))
+    mean = {k: statistics.mean(v[:n_full]) for k, v in times.items()}
+    lm_fp8 = bool(getattr(sh, "lm_fp8", False))
+    es = 2 if sh.dtype == "bf16" else 4
+    shape = RL.StepShape(sh.d_model, sh.n_heads, sh.n_kv_heads, sh.head_dim, sh.vocab, es,
+                         wl.canvas, r.lens)
+    work = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256,
+                        lm_elem_bytes=1 if lm_fp8 else 0)
+    out = {"stages_us": {k: round(v, 2) for k, v in mean.items()},
+           "steps_averaged": n_full, "step_algorithmic_bytes": work["step"]["bytes"]}
+    if sh.dtype != "bf16":
+        return out, None
+    lm_s = mean["lm_head"] / 1e6
+    intensity = work["lm_head"]["flop"] / work["lm_head"]["bytes"]
+    if intensity < 250:
+        ach, peak, unit, bound = work["lm_head"]["bytes"] / lm_s / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
+        src = " hbm_gbs"
+    else:
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * (2 if lm_fp8 else 1)
+        ach, unit, bound = work["lm_head"]["flop"] / lm_s / 1e12, "TFLOP/s", "tensor"
+        src = " bf16_tflops_sustained" + (" x 2 (e4m3 : bf16 nominal ratio)" if lm_fp8 else "")
+    roof = {"kernel": "gemm_tc_kernel<EPI_LM%s> (LM head + fused vocab reduction)"
+                      % (", e4m3" if lm_fp8 else ""),
+            "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
+            "frac": round(ach / peak, 4), "traffic": _ncu_traffic(wl.name),
+            "peak_source": pk.get("source", "measured") + src,
+            "launch_us": round(mean["lm_head"], 2),
+            "algorithmic_bytes_per_launch": work["lm_head"]["bytes"],
+            "algorithmic_flop_per_launch": work["lm_head"]["flop"],
+            "launches_timed": n_full}
+    ac_bytes = work["attention"]["bytes"] + work["reduce"]["bytes"] + work["commit"]["bytes"]
+    ac_s = (mean["attention"] + mean["reduce+commit"]) / 1e6
+    out["attention_commit"] = {
+        "bound": "hbm", "bytes": ac_bytes, "us": round(ac_s * 1e6, 2),
+        "achieved_gbs": round(ac_bytes / ac_s / 1e9, 1), "peak": pk["hbm_gbs"],
+        "frac": round(ac_bytes / ac_s / 1e9 / pk["hbm_gbs"], 4),
+        "attention_gbs": round(work["attention"]["bytes"] / (mean["attention"] / 1e6) / 1e9, 1),
+        "attention_frac": round(work["attention"]["bytes"] / (mean["attention"] / 1e6) / 1e9
+                                / pk["hbm_gbs"], 4)}
+    return out, roof
+
+
 def run_ours(a):
     import torch
     import masked_block_diffusion_denoise_b200 as dlm
     from masked_block_diffusion_denoise_b200 import build as B
-    from masked_block_diffusion_denoise_b200.session import Session, sampler_params
 
     world, rank, local, pg = dist_init(a.gpus)
     device = torch.device("cuda", local)
@@ -196,195 +380,170 @@ def run_ours(a):
         barrier(pg, device)
     wl = W.WORKLOADS[a.workload]
     sh = wl.shape
-    weights = W.make_weights(sh, seed=wl.seed)
-    lens, toks, kp, vp = W.make_prefix(wl)
-    sess = Session(sh, weights, max_batch=wl.batch, max_prefix=wl.prefix_cap,
-                   max_canvas=wl.canvas, device=device)
-    for b in range(wl.batch):
-        if toks is not None:
-            sess.kv_append_tokens(b, toks[b])
-        else:
-            n = int(lens[b])
-            sess.kv_append_kv(b, np.ascontiguousarray(kp[b][:, :n]),
-                              np.ascontiguousarray(vp[b][:, :n]))
-    del kp, vp
-    p = sampler_params(canvas=wl.canvas, steps=wl.steps, threshold=wl.threshold,
-                       quota=wl.quota, corruption=wl.corruption,
-                       entropy_bound=wl.entropy_bound, temperature=wl.temperature,
-                       t_max=wl.t_max, t_min=wl.t_min, seed=wl.seed)
+    r = Runner(wl, device)
     S = wl.steps
-    stream = torch.cuda.Stream(device)
-    # template canvas: initial state (+ EOS plant), copied in before every block
-    tmpl = sess.new_canvas(wl.batch, wl.canvas)
-    with torch.cuda.stream(stream):
-        sess.init(tmpl, p, stream=stream)
-        for (b, slot) in W.make_eos_plant(wl):
-            tmpl.tokens[b, slot] = sh.eos_id
-            tmpl.committed[b, slot] = 1
-    stream.synchronize()
-    cv = sess.new_canvas(wl.batch, wl.canvas)
-
-    def reset(canvas):
-        for dst, src in ((canvas.tokens, tmpl.tokens), (canvas.committed, tmpl.committed),
-                         (canvas.step, tmpl.step), (canvas.done, tmpl.done),
-                         (canvas.eos_pos, tmpl.eos_pos)):
-            dst.copy_(src, non_blocking=True)
-
-    def run_steps(k, canvas):
-        """k steps: whole blocks as graph replays, the rest as single steps."""
-        full, rest = divmod(k, S)
-        with torch.cuda.stream(stream):
-            for _ in range(full):
-                reset(canvas)
-                sess.block(canvas, p, stream=stream)
-            if rest:
-                reset(canvas)
-                for _ in range(rest):
-                    sess.step(canvas, p, stream=stream)
 
     if a.profile:
-        with torch.cuda.stream(stream):
-            reset(cv)
+        with torch.cuda.stream(r.stream):
+            r.reset()
             for _ in range(max(1, a.steps)):
-                sess.step(cv, p, stream=stream)
-        stream.synchronize()
-        sess.check(stream)
+                r.sess.step(r.cv, r.p, stream=r.stream)
+        r.stream.synchronize()
+        r.sess.check(r.stream)
         if rank == 0:
             print(json.dumps({"profile": a.workload, "steps": a.steps}))
         return
 
     K, Wm = a.steps, max(a.warmup, 3)
-    run_steps(max(Wm, S), cv)            # warm-up (also captures the block graph)
-    stream.synchronize()
-    sess.check(stream)
-    launches_per_step = dlm.dlm_launches_per_step(sess.ctx)
+    r.run(Wm)                       # warm-up, the same graph replays as the timed steps
+    r.stream.synchronize()
+    r.capture(K)                    # the timed region's graphs, before it
+    r.sess.check(r.stream)
+    launches_per_step = dlm.dlm_launches_per_step(r.sess.ctx)
 
     # ---- timed region ----
     clocks = Clocks(local) if rank == 0 else None
-    stats0 = cv.stats.clone()
-    cv.stats.zero_()
+    r.cv.stats.zero_()
     barrier(pg, device)
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg, device)
-    e0.record(stream)
-    run_steps(K, cv)
-    e1.record(stream)
-    stream.synchronize()
+    ms = r.timed(K)
     barrier(pg, device)
     ck = clocks.stop() if clocks else None
-    sess.check(stream)
-    ms = e0.elapsed_time(e1)
+    r.sess.check(r.stream)
     ms_max = max_over_ranks(pg, ms, device)
-    committed = int(cv.stats[:, 1].sum().item())
+    committed = int(r.cv.stats[:, 1].sum().item())
     committed_all = max_over_ranks(pg, committed, device) * world
-    del stats0
 
-    # ---- roofline of the dominant kernel: LM-head launches of the timed pass
-    # configuration, events recorded inside the replayed graph ----
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * S)]
-    for e in evs:            # torch creates the CUDA event on its first record
-        e.record(stream)
-    stream.synchronize()
-    dlm.dlm_set_stage_events(sess.ctx, dlm.DLM_STAGE_LM_HEAD, [e.cuda_event for e in evs])
-    n_roof_blocks = max(3, min(20, K // S))
-    run_steps(n_roof_blocks * S, cv)
-    stream.synchronize()
-    lm_ms = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(S)]
-    stages = {}
-    names = ["embed", "qkv", "attention", "wo", "lm_head", "reduce+commit"]
-    for st, name in enumerate(names):
-        dlm.dlm_set_stage_events(sess.ctx, st, [e.cuda_event for e in evs])
-        run_steps(2 * S, cv)
-        stream.synchronize()
-        stages[name] = 1e3 * statistics.mean(evs[2 * i].elapsed_time(evs[2 * i + 1])
-                                             for i in range(S))
-    dlm.dlm_set_stage_events(sess.ctx, 0, [])
+    # ---- per-stage events inside the replayed graph ----
+    pk = peaks()
+    figs, roof = kernel_figures(r, pk, n_blocks=max(2, min(10, K // S)))
 
     # ---- end to end through the host-buffer entry point ----
     e2e = None
     if not a.no_e2e:
-        host = {k: getattr(tmpl, k).cpu().pin_memory() for k in
+        host = {k: getattr(r.tmpl, k).cpu().pin_memory() for k in
                 ("tokens", "committed", "step", "done", "eos_pos")}
         hstats = torch.zeros((wl.batch, 6), dtype=torch.int32).pin_memory()
         work = {k: v.clone().pin_memory() for k, v in host.items()}
-        n_blocks = max(1, K // S)
+        n_blocks = max(3, K // S)
         h2d = sum(v.numel() * v.element_size() for v in host.values()) + hstats.numel() * 4
         d2h = h2d
-        barrier(pg, device)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(n_blocks):
+
+        def host_block():
             for k in work:
                 work[k].copy_(host[k])
-            dlm.dlm_decode_block_host(sess.ctx, work["tokens"], work["committed"], work["step"],
-                                      work["done"], work["eos_pos"], wl.batch, p, stats=hstats,
-                                      stream=stream)
-        f1.record(stream)
-        stream.synchronize()
+            dlm.dlm_decode_block_host(r.sess.ctx, work["tokens"], work["committed"],
+                                      work["step"], work["done"], work["eos_pos"], wl.batch,
+                                      r.p, stats=hstats, stream=r.stream)
+        host_block()                # warm: the entry point's graph is captured here
+        hstats.zero_()
+        barrier(pg, device)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(r.stream)
+        for _ in range(n_blocks):
+            host_block()
+        f1.record(r.stream)
+        r.stream.synchronize()
         e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), device)
-        e2e = {"value": world * n_blocks * S / (e2e_ms / 1e3), "unit": "steps/s",
+        e2e = {"value": round(world * n_blocks * S / (e2e_ms / 1e3), 2), "unit": "steps/s",
                "h2d_bytes_per_step": h2d / S, "d2h_bytes_per_step": d2h / S,
-               "blocks": n_blocks, "call": "dlm_decode_block_host"}
+               "blocks": n_blocks, "call": "dlm_decode_block_host",
+               "committed_tokens_per_s": round(
+                   world * float(hstats[:, 1].sum().item()) / (e2e_ms / 1e3), 1)}
+    plan = r.plan()
 
+    line = None
     if rank == 0:
-        pk = peaks()
-        shape = RL.StepShape(sh.d_model, sh.n_heads, sh.n_kv_heads, sh.head_dim, sh.vocab, 2,
-                             wl.canvas, [int(x) for x in lens])
-        lm_fp8 = bool(getattr(sh, "lm_fp8", False))
-        work_ = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256,
-                             lm_elem_bytes=1 if lm_fp8 else 0)
-        lm_avg_s = statistics.mean(lm_ms) / 1e3
-        bound = "hbm" if work_["lm_head"]["flop"] / work_["lm_head"]["bytes"] < 250 else "tensor"
-        if bound == "hbm":
-            ach = work_["lm_head"]["bytes"] / lm_avg_s / 1e9
-            peak = pk["hbm_gbs"]
-            unit = "GB/s"
-        else:
-            ach = work_["lm_head"]["flop"] / lm_avg_s / 1e12
-            peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-            unit = "TFLOP/s"
-        roof = {"kernel": "gemm_tc_kernel<EPI_LM%s> (LM head + fused vocab reduction)"
-                          % (", e4m3" if lm_fp8 else ""),
-                "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
-                "frac": round(ach / peak, 4), "traffic": None,
-                "peak_source": pk.get("source", "measured") + (" hbm_gbs" if bound == "hbm"
-                                                               else " bf16_tflops_sustained"),
-                "launch_us": round(lm_avg_s * 1e6, 2),
-                "algorithmic_bytes_per_launch": work_["lm_head"]["bytes"],
-                "algorithmic_flop_per_launch": work_["lm_head"]["flop"],
-                "launches_timed": len(lm_ms)}
-        traffic = _ncu_traffic(a.workload)
-        if traffic is not None:
-            roof["traffic"] = traffic
         step_s = ms_max / 1e3 / K
         line = {
             "metric": "denoise steps/s", "value": round(aggregate_rate(world, K, ms_max), 2),
-            "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": max(Wm, S),
+            "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("bf16, LM head e4m3" if lm_fp8 else "bf16") if sh.dtype == "bf16" else "f32",
+            "dtype": ("bf16, LM head e4m3" if getattr(sh, "lm_fp8", False) else "bf16")
+                     if sh.dtype == "bf16" else "f32",
             "data": "synthetic: seeded random-init weights N(0,0.02), embeddings and prefix "
                     "K/V N(0,1), all-mask canvas",
-            "config": workload_config(a.workload, wl, lens, world),
+            "config": workload_config(a.workload, wl, r.lens, world),
             "committed_tokens_per_s": round(committed_all / (ms_max / 1e3), 1),
-            "stages_us": {k: round(v, 2) for k, v in stages.items()},
-            "step_algorithmic_bytes": work_["step"]["bytes"],
-            "step_hbm_frac": round(work_["step"]["bytes"] / step_s / 1e9 / pk["hbm_gbs"], 4),
+            "timing": "%d whole-block graph replays + one graph of %d steps, every block from "
+                      "the initial canvas" % divmod(K, S),
+            "stages_us": figs["stages_us"],
+            "stages_steps_averaged": figs["steps_averaged"],
+            "step_algorithmic_bytes": figs["step_algorithmic_bytes"],
+            "step_hbm_frac": round(figs["step_algorithmic_bytes"] / step_s / 1e9
+                                   / pk["hbm_gbs"], 4),
+            "attention_commit": figs.get("attention_commit"),
+            "attention_plan": plan,
             "roofline": roof,
             "gpu_launches": int(launches_per_step * K),
             "e2e": e2e,
             "clocks": ck,
         }
+    r.close()
+    del r
+    torch.cuda.empty_cache()
+    if rank == 0:
+        if world == 1 and not a.no_configs:
+            line["configs"] = measure_configs(a.workload, device, pk)
         if world == 1 and not a.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(line), flush=True)
-    sess.close()
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
+
+
+CONFIG_WORKLOADS = ["tiny", "8b_b1", "batched", "longctx", "encdec", "encdec_eb"]
+
+
+def measure_configs(skip, device, pk):
+    """One block (S steps, graph replay, after one warm-up block) of every
+    configuration, with its stage rooflines; weights are drawn once per
+    model shape."""
+    import torch
+    out = {}
+    uploads = {}
+    for name in CONFIG_WORKLOADS:
+        if name == skip:
+            out[name] = "the headline line"
+            continue
+        wl = W.WORKLOADS[name]
+        key = (wl.shape, wl.seed)
+        if key not in uploads:
+            from masked_block_diffusion_denoise_b200.session import host_to_device
+            uploads.clear()
+            torch.cuda.empty_cache()
+            w = W.make_weights(wl.shape, seed=wl.seed)
+            uploads[key] = {k: host_to_device(v, wl.shape.dtype, device) for k, v in w.items()}
+            del w
+        r = Runner(wl, device, upload=uploads[key])
+        try:
+            S = wl.steps
+            r.run(S)
+            r.stream.synchronize()
+            r.cv.stats.zero_()
+            ms = r.timed(S)
+            r.sess.check(r.stream)
+            committed = int(r.cv.stats[:, 1].sum().item())
+            figs, roof = kernel_figures(r, pk, n_blocks=2)
+            entry = {"steps_per_s": round(S / (ms / 1e3), 2), "ms_per_step": round(ms / S, 5),
+                     "committed_tokens_per_s": round(committed / (ms / 1e3), 1),
+                     "stages_us": figs["stages_us"]}
+            if roof is not None:
+                entry["lm_head"] = {k: roof[k] for k in ("bound", "achieved", "peak", "unit",
+                                                         "frac", "launch_us", "traffic")}
+                entry["attention_commit"] = figs["attention_commit"]
+                entry["attention_plan"] = r.plan()
+            out[name] = entry
+        finally:
+            r.close()
+    uploads.clear()
+    torch.cuda.empty_cache()
+    return out
 
 
 def _ncu_traffic(workload):
@@ -444,11 +603,12 @@ def _oracle_setup(wl, vocab_slice=None):
     return O, om, p, st
 
 
-def _oracle_step_timed(O, om, p, st, vocab_full):
-    """One oracle step; returns (seconds of forward-to-y, of LM head + scores,
-    of selection).  The LM head may cover a vocabulary slice."""
+def _oracle_step_timed(O, om, p, st, vocab_full, canvases=None):
+    """One oracle step over `canvases` (all when None); returns (seconds of
+    forward-to-y, of LM head + scores, of selection).  The LM head may cover
+    a vocabulary slice."""
     t_fwd = t_lm = t_sel = 0.0
-    for b in range(st.tokens.shape[0]):
+    for b in (range(st.tokens.shape[0]) if canvases is None else canvases):
         if st.done[b]:
             continue
         t0 = time.perf_counter()
@@ -490,9 +650,12 @@ def cpu_baseline(wl):
 
 def run_reference(a):
     """--impl reference: the oracle on this host, K timed steps after W
-    warm-up steps; each step computes the full forward to the LM-head input
-    and the LM head + scores on a vocabulary slice of 1/f of the rows of W_lm,
-    whose time is scaled by f (every other stage in full)."""
+    warm-up steps.  Each step is a bounded sample of the batch's step: the
+    first n_s = ceil(B / 8) canvases (every canvas up to a batch of 8), each
+    with its full forward to the LM-head input, the LM head + scores on a
+    vocabulary slice of 1/f of the rows of W_lm (that part's time scaled by f)
+    and its selection; the sampled canvases' time is scaled by B / n_s.  When
+    the sampled canvases are all done, their block starts over."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -501,14 +664,16 @@ def run_reference(a):
     V = wl.shape.vocab
     f = 32
     O, om, p, st = _oracle_setup(wl, vocab_slice=V // f)
+    n_s = -(-wl.batch // 8)
+    sample = list(range(n_s))
     K, Wm = a.steps, max(a.warmup, 3)
     total = 0.0
     for i in range(Wm + K):
-        if st.done.all():
+        if st.done[sample].all():
             st = O.init_canvas(wl.batch, p, wl.shape.mask_id, V)
-        fw, lm, sel = _oracle_step_timed(O, om, p, st, V)
+        fw, lm, sel = _oracle_step_timed(O, om, p, st, V, canvases=sample)
         if i >= Wm:
-            total += fw + lm * f + sel
+            total += (fw + lm * f + sel) * wl.batch / n_s
     value = K / total
     line = {"metric": "denoise steps/s", "value": round(value, 4), "unit": "steps/s",
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": round(1e3 * total / K, 3),
@@ -517,9 +682,11 @@ def run_reference(a):
             "config": workload_config(a.workload, wl, W.make_prefix(wl)[0], world),
             "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": _threads(),
                              "kind": "oracle",
-                             "sample": "each step: full forward to the LM-head input, LM head "
-                                       "and scores on 1/%d of the vocabulary, time scaled "
-                                       "by %d" % (f, f)},
+                             "sample": "each step: %d of the %d canvases, each with its full "
+                                       "forward to the LM-head input, LM head and scores on "
+                                       "1/%d of the vocabulary (that time scaled by %d) and "
+                                       "its selection; time scaled by %d/%d"
+                                       % (n_s, wl.batch, f, f, wl.batch, n_s)},
             "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -60,6 +60,7 @@ enum {
 
 enum { DLM_F32 = 0, DLM_BF16 = 1 };          /* model / weight element type  */
 enum { DLM_MASK = 0, DLM_UNIFORM = 1 };      /* corruption of uncommitted slots */
+enum { DLM_LM_MODEL = 0, DLM_LM_E4M3 = 1, DLM_LM_NVFP4 = 2 };   /* LM-head format  */
 
 typedef struct dlm_ctx dlm_ctx;
 
@@ -75,17 +76,25 @@ typedef struct {
   int max_batch;    /* sequences (canvases) per call                       */
   int max_prefix;   /* KV capacity per sequence for the finished prefix    */
   int max_canvas;   /* largest canvas length, <= 1024                       */
-  /* 1: e4m3 LM head (bf16 models, d_model % 16 == 0).  Online FP8
-   * quantisation of the head's weights (NLD tutorial, section 8.6; course
-   * "Diffusion LLMs", section 15: low-bit weights are the Blackwell path):
-   * dlm_create quantises W_lm per vocabulary row into a context-owned copy,
-   * scale s_v = max|W_v| / 448 (1 for a zero row), q = e4m3(W / s_v), round
-   * to nearest even, saturating; W_lm is not read afterwards.  The tensor
-   * cores take both operands in 8 bits, so every step quantises the head's
-   * input rows y the same way (a_r = max|y_r| / 448) and the logits are
-   * (sum_k qy_rk qW_vk) * (a_r * s_v), the factor rounded to float32.
-   * 0: the head in the model's element type. */
-  int lm_fp8;
+  /* Element format of the LM head (NLD tutorial, section 8.6: online FP8
+   * weight quantisation; course "Diffusion LLMs", section 15: low-bit
+   * weights, NVFP4 on Blackwell).  The tensor cores take both operands in
+   * the low-bit format, so every step quantises the head's input rows y the
+   * same way as the weights, which dlm_create quantises once per vocabulary
+   * row into a context-owned copy (W_lm is not read afterwards).
+   *   DLM_LM_MODEL  the model's element type.
+   *   DLM_LM_E4M3   (bf16 models, d_model % 16 == 0) scale s_v = max|W_v| /
+   *                 448 (1 for a zero row), q = e4m3(W / s_v), round to nearest
+   *                 even, saturating; the logits are (sum_k qy_rk qW_vk) *
+   *                 (a_r * s_v), the factor rounded to float32.
+   *   DLM_LM_NVFP4  (bf16 models, d_model % 256 == 0) a float32 row scale
+   *                 s = max|row| / (448 * 6) (1 for a zero row), an e4m3 scale
+   *                 per 16 elements e4m3(max|block| / (6 s)), elements
+   *                 e2m1(x / (block scale * s)) (0 in a block whose scale is
+   *                 0), every division and product in float32, round to
+   *                 nearest even, saturating; the logits are the block-scaled
+   *                 sums times the two row scales' product rounded to float32. */
+  int lm_quant;
 } dlm_model_desc;
 
 /* Device pointers, caller-owned, valid for the life of the context; element
@@ -217,6 +226,27 @@ int dlm_denoise_step(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
 int dlm_decode_block(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
                      const dlm_sampler_params *params, dlm_canvas_stats *stats, void *stream);
 
+/* The first n_steps (1 <= n_steps <= params->steps) denoising steps of
+ * dlm_decode_block as one CUDA graph, captured once per configuration and
+ * step count and replayed on `stream`.  Every step reads the canvas's own
+ * step counters on the device, so n_steps steps from any canvas state do
+ * what n_steps dlm_denoise_step calls would; dlm_decode_block is this call
+ * with n_steps = params->steps.  Same arguments otherwise; DLM_EINVAL for
+ * n_steps out of range. */
+int dlm_decode_steps(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
+                     const dlm_sampler_params *params, int n_steps, dlm_canvas_stats *stats,
+                     void *stream);
+
+/* The split plan of the canvas attention that dlm_denoise_step runs for
+ * `batch` canvases of `canvas` positions over the context's current prefix
+ * lengths (bf16 contexts): *nsplit key splits of *chunk keys (a multiple of
+ * 128) per (sequence, KV head, row tile); *cluster = nsplit when the splits
+ * combine inside one thread-block cluster, else 1 (partials and a combine
+ * kernel when nsplit > 1); *rows_per_cta query rows per CTA.  Host-only, no
+ * device work.  DLM_EINVAL for an fp32 context or sizes out of range. */
+int dlm_attention_plan(dlm_ctx *ctx, int batch, int canvas, int *nsplit, int *chunk,
+                       int *cluster, int *rows_per_cta);
+
 /* dlm_decode_block with HOST buffers: copies the canvas state in (host
  * arrays shaped as in dlm_canvas), runs the block, copies the canvas state
  * and `stats` (host, may be NULL) back, and synchronises `stream`.  The
@@ -259,20 +289,28 @@ int dlm_commit(dlm_ctx *ctx, const dlm_canvas *canvas, int batch,
  * DLM_BUF_Y [M][d] (model element type; M = batch * C, row b*C + i),
  * DLM_BUF_CAND int32 [M], DLM_BUF_CONF float [M], DLM_BUF_ENTROPY float [M],
  * DLM_BUF_K_CACHE / DLM_BUF_V_CACHE [max_batch][Hkv][max_prefix+max_canvas][Dh];
- * with lm_fp8 also DLM_BUF_LM_Q uint8 e4m3 [vocab][d] and DLM_BUF_LM_SCALE
- * float [vocab rounded up to 256] (zero padding), DLM_BUF_Y_Q uint8 e4m3
- * [M][d] and DLM_BUF_Y_SCALE float [M] (DLM_EINVAL without lm_fp8).
+ * with a low-bit LM head also DLM_BUF_LM_Q (the quantised weights: e4m3
+ * bytes [vocab][d], or NVFP4 e2m1 pairs [vocab][d/2] with element 2i in the
+ * low nibble), DLM_BUF_LM_SCALE float row scales [vocab rounded up to 256]
+ * (zero padding), DLM_BUF_Y_Q / DLM_BUF_Y_SCALE the last step's quantised
+ * rows and their scales ([M][d] or [M][d/2]; [M]); with the NVFP4 head
+ * DLM_BUF_LM_SF / DLM_BUF_Y_SF the e4m3 block scales in the layout the
+ * block-scaled tensor cores read: per 128-row block and 64-element k group a
+ * 512-byte chunk, byte (m % 32) * 16 + (m / 32) * 4 + s for row m of the
+ * block and its s-th 16-element block ([ceil(rows/128)][d/64][512]).
+ * DLM_EINVAL for a buffer the context does not have.
  * *ptr receives a device pointer owned by the context, *bytes its size. */
 enum { DLM_BUF_X = 0, DLM_BUF_Q = 1, DLM_BUF_O = 2, DLM_BUF_Y = 3, DLM_BUF_CAND = 4,
        DLM_BUF_CONF = 5, DLM_BUF_ENTROPY = 6, DLM_BUF_K_CACHE = 7, DLM_BUF_V_CACHE = 8,
-       DLM_BUF_LM_Q = 9, DLM_BUF_LM_SCALE = 10, DLM_BUF_Y_Q = 11, DLM_BUF_Y_SCALE = 12 };
+       DLM_BUF_LM_Q = 9, DLM_BUF_LM_SCALE = 10, DLM_BUF_Y_Q = 11, DLM_BUF_Y_SCALE = 12,
+       DLM_BUF_LM_SF = 13, DLM_BUF_Y_SF = 14 };
 int dlm_debug_buffer(dlm_ctx *ctx, int which, void **ptr, size_t *bytes);
 
 /* Full float32 logits of the rows in DLM_BUF_Y: `logits` (device float
  * [batch*canvas][vocab]) receives y W_lm^T from the same GEMM main loop as
- * the fused reduction (the store epilogue instead of the reduction); with
- * lm_fp8 the logits of the last step's quantised rows (DLM_BUF_Y_Q) with the
- * same scale factor as the step. */
+ * the fused reduction (the store epilogue instead of the reduction); with a
+ * low-bit head the logits of the last step's quantised rows (DLM_BUF_Y_Q)
+ * with the same scales as the step. */
 int dlm_debug_logits(dlm_ctx *ctx, int batch, int canvas, float *logits, void *stream);
 
 /* Stages of a step, for dlm_set_stage_events.  DLM_STAGE_COMMIT is the one
@@ -307,18 +345,28 @@ int dlm_set_stage_events(dlm_ctx *ctx, int stage, void *const *events, int n_pai
  *   lens     device int32 [batch]; max_len (host) must be >= every lens[b]
  *   o        device bf16 [batch*canvas][n_heads*head_dim], written
  * head_dim must be 128, n_heads a multiple of n_kv_heads, batch <= kv_batch,
- * max_len + canvas <= kv_capacity.  If the split plan needs more than the
- * 16384 slots (batch * n_kv_heads * splits * query-rows-per-KV-head) the call
- * fails with DLM_EINVAL and dlm_last_error(NULL) says how many it needed.
+ * max_len + canvas <= kv_capacity (else DLM_EINVAL, nothing launched).  The
+ * split plan is dlm_denoise_step's, restricted to plans whose partials fit
+ * the 16384 slots (batch * n_kv_heads * splits * query-rows-per-KV-head);
+ * one split needs none, so every valid size runs.
  * The first call on a device looks up the array's device address; make that
  * first call before any stream capture.  Every call shares the array, so
  * calls that overlap on the GPU (different streams, or other threads) race;
- * serialise them.  Launch errors are returned; a device-side wait that gives
- * up is recorded in a device word that each call clears first. */
+ * serialise them.  Launch errors are returned.  A device-side wait that gives
+ * up (DLM_ETIMEOUT) or a failed index check (DLM_EBOUNDS, index-checking
+ * build) is recorded in a device error word of the library, first error
+ * kept, until dlm_attention_noalloc_check reads and clears it. */
 int dlm_attention_noalloc(const void *q, const void *k_cache, const void *v_cache,
                           const int32_t *lens, int max_len, void *o, int batch, int canvas,
                           int n_heads, int n_kv_heads, int head_dim, int kv_batch,
                           int kv_capacity, void *stream);
+
+/* Synchronise `stream`, then read and clear the device error word of
+ * dlm_attention_noalloc on the current device: DLM_OK, or DLM_ETIMEOUT /
+ * DLM_EBOUNDS recorded by a kernel of an earlier call (the text is in
+ * dlm_last_error(NULL)); DLM_ECUDA if the runtime fails.  Like the array, the
+ * word is shared by every caller on the device. */
+int dlm_attention_noalloc_check(void *stream);
 
 /* Synchronise `stream` and return the device error word (DLM_OK, or
  * DLM_ETIMEOUT / DLM_EBOUNDS set by a kernel); clears it. */
@@ -345,6 +393,17 @@ int dlm_trace_layout(int *kinds, int *ctas, int *slots);
 int dlm_trace_read(unsigned long long *table, size_t words);
 /* Zero the table (synchronises the device). */
 int dlm_trace_clear(void);
+
+/* Failure-detection test hook (bf16 contexts).  The next n_launches
+ * tensor-core GEMM launches this context issues withhold their TMA loads:
+ * the MMA warp's bounded wait for the first ring stage then runs out (after
+ * 20 ms instead of the normal 2 s), the CTA stops issuing work, lets
+ * nothing in flight outlive it, frees its tensor memory and records
+ * DLM_ETIMEOUT in the context's error word (dlm_check returns it).  The
+ * rest of the step runs on the stale activations, so its results are
+ * meaningless; the context stays usable.  No device fault is involved.
+ * DLM_EINVAL for n_launches < 0 or an fp32 context. */
+int dlm_test_withhold_loads(dlm_ctx *ctx, int n_launches);
 
 /* Number of kernel launches one dlm_denoise_step made for this batch and
  * configuration (the last one issued), for launch accounting. */

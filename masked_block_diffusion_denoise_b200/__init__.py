@@ -17,7 +17,8 @@ __all__ = [
     "DLM_EBOUNDS", "DLM_ESTATE", "DLM_F32", "DLM_BF16", "DLM_MASK", "DLM_UNIFORM",
     "DLM_BUF_X", "DLM_BUF_Q", "DLM_BUF_O", "DLM_BUF_Y", "DLM_BUF_CAND", "DLM_BUF_CONF",
     "DLM_BUF_ENTROPY", "DLM_BUF_K_CACHE", "DLM_BUF_V_CACHE", "DLM_BUF_LM_Q", "DLM_BUF_LM_SCALE",
-    "DLM_BUF_Y_Q", "DLM_BUF_Y_SCALE",
+    "DLM_BUF_Y_Q", "DLM_BUF_Y_SCALE", "DLM_BUF_LM_SF", "DLM_BUF_Y_SF", "DLM_LM_MODEL",
+    "DLM_LM_E4M3", "DLM_LM_NVFP4",
     "dlm_model_desc", "dlm_weights", "dlm_sampler_params", "dlm_canvas", "dlm_canvas_stats",
     "DlmError", "lib", "library_path", "dlm_create", "dlm_destroy", "dlm_kv_append",
     "dlm_reset_kv", "dlm_kv_length", "dlm_canvas_init", "dlm_denoise_step",
@@ -25,8 +26,9 @@ __all__ = [
     "dlm_debug_logits", "dlm_check", "dlm_launches_per_step", "dlm_last_error",
     "EXPORTED_SYMBOLS", "dlm_set_stage_events", "DLM_STAGE_EMBED", "DLM_STAGE_QKV",
     "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT",
-    "DLM_NUM_STAGES", "dlm_attention_noalloc", "dlm_trace_layout", "dlm_trace_read",
-    "dlm_trace_clear",
+    "DLM_NUM_STAGES", "dlm_attention_noalloc", "dlm_attention_noalloc_check",
+    "dlm_trace_layout", "dlm_trace_read", "dlm_trace_clear", "dlm_decode_steps",
+    "dlm_attention_plan", "dlm_test_withhold_loads",
 ]
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, DLM_ESTATE = \
@@ -35,7 +37,8 @@ DLM_F32, DLM_BF16 = 0, 1
 DLM_MASK, DLM_UNIFORM = 0, 1
 (DLM_BUF_X, DLM_BUF_Q, DLM_BUF_O, DLM_BUF_Y, DLM_BUF_CAND, DLM_BUF_CONF, DLM_BUF_ENTROPY,
  DLM_BUF_K_CACHE, DLM_BUF_V_CACHE, DLM_BUF_LM_Q, DLM_BUF_LM_SCALE, DLM_BUF_Y_Q,
- DLM_BUF_Y_SCALE) = range(13)
+ DLM_BUF_Y_SCALE, DLM_BUF_LM_SF, DLM_BUF_Y_SF) = range(15)
+DLM_LM_MODEL, DLM_LM_E4M3, DLM_LM_NVFP4 = 0, 1, 2
 
 (DLM_STAGE_EMBED, DLM_STAGE_QKV, DLM_STAGE_ATTENTION, DLM_STAGE_WO, DLM_STAGE_LM_HEAD,
  DLM_STAGE_COMMIT, DLM_NUM_STAGES) = range(7)
@@ -54,7 +57,7 @@ class dlm_model_desc(ctypes.Structure):
                 ("rope_theta", ctypes.c_float), ("mask_id", ctypes.c_int),
                 ("eos_id", ctypes.c_int), ("max_batch", ctypes.c_int),
                 ("max_prefix", ctypes.c_int), ("max_canvas", ctypes.c_int),
-                ("lm_fp8", ctypes.c_int)]
+                ("lm_quant", ctypes.c_int)]
 
 
 class dlm_weights(ctypes.Structure):
@@ -103,6 +106,10 @@ _SIGS = {
                               ctypes.POINTER(dlm_sampler_params), _P, _P]),
     "dlm_decode_block": (_I, [_P, ctypes.POINTER(dlm_canvas), _I,
                               ctypes.POINTER(dlm_sampler_params), _P, _P]),
+    "dlm_decode_steps": (_I, [_P, ctypes.POINTER(dlm_canvas), _I,
+                              ctypes.POINTER(dlm_sampler_params), _I, _P, _P]),
+    "dlm_attention_plan": (_I, [_P, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "dlm_decode_block_host": (_I, [_P, _P, _P, _P, _P, _P, _I,
                                    ctypes.POINTER(dlm_sampler_params), _P, _P]),
     "dlm_commit": (_I, [_P, ctypes.POINTER(dlm_canvas), _I, ctypes.POINTER(dlm_sampler_params),
@@ -113,8 +120,10 @@ _SIGS = {
     "dlm_debug_logits": (_I, [_P, _I, _I, _P, _P]),
     "dlm_set_stage_events": (_I, [_P, _I, ctypes.POINTER(_P), _I]),
     "dlm_attention_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I, _P]),
+    "dlm_attention_noalloc_check": (_I, [_P]),
     "dlm_check": (_I, [_P, _P]),
     "dlm_launches_per_step": (_I, [_P]),
+    "dlm_test_withhold_loads": (_I, [_P, _I]),
     "dlm_trace_layout": (_I, [ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "dlm_trace_read": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_size_t]),
     "dlm_trace_clear": (_I, []),
@@ -214,6 +223,22 @@ def dlm_decode_block(ctx, canvas: dlm_canvas, batch: int, params: dlm_sampler_pa
                                               _stream(stream)))
 
 
+def dlm_decode_steps(ctx, canvas: dlm_canvas, batch: int, params: dlm_sampler_params,
+                     n_steps: int, stats=None, stream=None) -> int:
+    return _check(ctx, lib().dlm_decode_steps(ctx, ctypes.byref(canvas), batch,
+                                              ctypes.byref(params), n_steps, _ptr(stats),
+                                              _stream(stream)))
+
+
+def dlm_attention_plan(ctx, batch: int, canvas: int) -> dict:
+    """The attention split plan for the context's current prefix lengths."""
+    ns, ch, cl, rows = _I(), _I(), _I(), _I()
+    _check(ctx, lib().dlm_attention_plan(ctx, batch, canvas, ctypes.byref(ns), ctypes.byref(ch),
+                                         ctypes.byref(cl), ctypes.byref(rows)))
+    return {"nsplit": ns.value, "chunk": ch.value, "cluster": cl.value,
+            "rows_per_cta": rows.value}
+
+
 def dlm_decode_block_host(ctx, tokens, committed, step, done, eos_pos, batch: int,
                           params: dlm_sampler_params, stats=None, stream=None) -> int:
     """Host (CPU, ideally pinned) tensors in, results copied back in place."""
@@ -272,12 +297,27 @@ def dlm_attention_noalloc(q, k_cache, v_cache, lens, max_len: int, o, batch: int
     return rc
 
 
+def dlm_attention_noalloc_check(stream=None) -> int:
+    """Read and clear the device error word of dlm_attention_noalloc; raises
+    DlmError(DLM_ETIMEOUT / DLM_EBOUNDS) when a kernel recorded one."""
+    rc = lib().dlm_attention_noalloc_check(_stream(stream))
+    if rc != DLM_OK:
+        raise DlmError(rc, lib().dlm_last_error(None).decode())
+    return rc
+
+
 def dlm_check(ctx, stream=None) -> int:
     return _check(ctx, lib().dlm_check(ctx, _stream(stream)))
 
 
 def dlm_launches_per_step(ctx) -> int:
     return _check(ctx, lib().dlm_launches_per_step(ctx))
+
+
+def dlm_test_withhold_loads(ctx, n_launches: int) -> int:
+    """Failure-detection test hook: the next n GEMM launches issue no loads,
+    so their bounded waits run out and DLM_ETIMEOUT is recorded."""
+    return _check(ctx, lib().dlm_test_withhold_loads(ctx, n_launches))
 
 
 def dlm_trace_layout():

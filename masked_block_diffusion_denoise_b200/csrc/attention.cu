@@ -501,6 +501,365 @@ __global__ void __launch_bounds__(192, 1)
   if (tid == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
 }
 
+// ---------------------------------------------------------------------------
+// Two query-row tiles per CTA (256 rows): when a KV head has at least 256
+// query rows (G * C >= 256), one CTA takes two 128-row tiles of the same
+// (sequence, KV head, key split), so each K/V tile crosses HBM once for both.
+// 10 warps:
+//   warp 0     TMA producer: K tiles into a 2-slot ring, V tiles into a
+//              3-slot ring (128 keys x 128 dims, two 64-column halves each);
+//   warp 1     MMA issuer, per key tile t:  O0 += P0(t-1) V(t-1);
+//              S0(t) = Q0 K(t)^T;  O1 += P1(t-1) V(t-1);  S1(t) = Q1 K(t)^T
+//              -- each row tile has one S buffer, and tcgen05 operations of
+//              one thread run in order, so S_i(t) is written after P_i(t-1)
+//              has been read, and once S_i(t) is complete O_i holds every
+//              earlier P_i V (the softmax may rescale it at once);
+//   warps 2-5  softmax of row tile 0, warps 6-9 of row tile 1: the two
+//              warpgroups alternate with the tensor core (while one turns
+//              S_i(t) into P_i(t), the other's S or P V runs).
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Splits write
+// bf16 O (one split) or f32 partials for attn_combine_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kTile2 = 2 * kHalf;                 // one 128-row / 128-key tile: 32 KB
+constexpr int kKSlots2 = 2, kVSlots2 = 3;
+constexpr int kAttn2Smem = 2 * kTile2 + (kKSlots2 + kVSlots2) * kTile2 + 1024 + 512;
+static_assert(kAttn2Smem <= 232448, "two-tile attention exceeds shared memory");
+
+__global__ void __maxnreg__(200)
+    attn_tc2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
+  // timeline marks: 2 wait returned, 3 query and first K tile in shared
+  // memory, 4 O complete
+  DLM_TRACE_CTA(TRACE_ATTENTION);
+  const int split = blockIdx.x, pair = blockIdx.y, bg = blockIdx.z;
+  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+  const int na = p.n_active != nullptr ? __ldcg(p.n_active) : 1;
+  const bool dn = p.done != nullptr && __ldcg(p.done + b) != 0;
+  const int len_b = __ldcg(p.lens + b);
+  if (na == 0 || dn) return;
+  const int n_keys = len_b + p.C;
+  if (!DLM_IN_BOUNDS(n_keys - 1, p.Lcap, p.err)) return;
+  const int k_begin = split * p.chunk;
+  if (k_begin >= n_keys) return;
+  const int k_end = min(k_begin + p.chunk, n_keys);
+  const int n_tiles = (k_end - k_begin + kKeys - 1) / kKeys;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* qs = smem;                                   // Q0, Q1
+  uint8_t* kring = smem + 2 * kTile2;
+  uint8_t* vring = kring + kKSlots2 * kTile2;
+  uint64_t* k_full = reinterpret_cast<uint64_t*>(vring + kVSlots2 * kTile2);
+  uint64_t* k_empty = k_full + kKSlots2;
+  uint64_t* v_full = k_empty + kKSlots2;
+  uint64_t* v_empty = v_full + kVSlots2;
+  uint64_t* s_full = v_empty + kVSlots2;                // [2]
+  uint64_t* p_full = s_full + 2;                        // [2]
+  uint64_t* o_done = p_full + 2;
+  uint64_t* q_full = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < kKSlots2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kVSlots2; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(q_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  __syncthreads();
+  const int plane = b * p.Hkv + g;
+  auto issue_k = [&](int t) {
+    uint8_t* base = kring + (t % kKSlots2) * kTile2;
+    const int key0 = k_begin + t * kKeys;
+    mbar_arrive_expect_tx(&k_full[t % kKSlots2], kTile2);
+    tma_load_3d(base, &tmK, &k_full[t % kKSlots2], 0, key0, plane);
+    tma_load_3d(base + kHalf, &tmK, &k_full[t % kKSlots2], 64, key0, plane);
+  };
+  auto issue_v = [&](int t) {
+    uint8_t* base = vring + (t % kVSlots2) * kTile2;
+    const int key0 = k_begin + t * kKeys;
+    mbar_arrive_expect_tx(&v_full[t % kVSlots2], kTile2);
+    tma_load_3d(base, &tmV, &v_full[t % kVSlots2], 0, key0, plane);
+    tma_load_3d(base + kHalf, &tmV, &v_full[t % kVSlots2], 64, key0, plane);
+  };
+  // K/V tiles wholly inside the cached prefix do not depend on the previous
+  // kernel: the first ring slots' worth are issued before the wait
+  int pre = 0;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    if (p.q_tma) tma_prefetch(&tmQ);
+    while (pre < kKSlots2 && pre < n_tiles && k_begin + (pre + 1) * kKeys <= len_b) {
+      issue_k(pre);
+      issue_v(pre);
+      ++pre;
+    }
+  }
+  pdl_wait_then_release();
+  if (tid == 0) DLM_TRACE_MARK(2);
+  const int row_base = pair * 2 * kRowsCta;   // first query row of tile 0
+  if (p.q_tma) {
+    if (warp == 0 && lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * kTile2);
+      for (int i = 0; i < 2; ++i) {
+        const int z0 = b * p.C + (row_base + i * kRowsCta) / p.G;
+        tma_load_3d(qs + i * kTile2, &tmQ, q_full, 0, g * p.G, z0);
+        tma_load_3d(qs + i * kTile2 + kHalf, &tmQ, q_full, 64, g * p.G, z0);
+      }
+    }
+  } else {
+    // plain loads: 256 rows x 16 chunks of 16 bytes, rows past R zero
+    for (int idx = tid; idx < 2 * kRowsCta * 16; idx += blockDim.x) {
+      const int lr = idx >> 4, ch = idx & 15;
+      const int r = row_base + lr;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (r < p.R) {
+        const int i = r / p.G, hh = r - i * p.G;
+        val = *reinterpret_cast<const uint4*>(
+            p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8);
+      }
+      const int tile = lr >> 7, tr = lr & 127;
+      *reinterpret_cast<uint4*>(qs + tile * kTile2 + (ch >> 3) * kHalf + sw128_off(tr, ch & 7)) =
+          val;
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = pre;
+      for (int t = pre; t < n_tiles; ++t) {
+        if (t >= kKSlots2 &&
+            !mbar_wait_bounded(&k_empty[t % kKSlots2], (uint32_t)(((t / kKSlots2) & 1) ^ 1),
+                               abort_flag))
+          break;
+        if (t >= kVSlots2 &&
+            !mbar_wait_bounded(&v_empty[t % kVSlots2], (uint32_t)(((t / kVSlots2) & 1) ^ 1),
+                               abort_flag)) {
+          // K(t) is not issued either: keep the K and V counts equal
+          break;
+        }
+        issue_k(t);
+        issue_v(t);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA exits
+        for (int t = issued - 1; t >= 0 && t >= issued - kKSlots2; --t)
+          mbar_wait_bounded(&k_full[t % kKSlots2], (uint32_t)((t / kKSlots2) & 1), nullptr);
+        for (int t = issued - 1; t >= 0 && t >= issued - kVSlots2; --t)
+          mbar_wait_bounded(&v_full[t % kVSlots2], (uint32_t)((t / kVSlots2) & 1), nullptr);
+      }
+      if (p.q_tma) mbar_wait_bounded(q_full, 0, nullptr);   // the query tiles have landed
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsCta, kKeys);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kRowsCta, kDh, true);
+      auto issue_s = [&](int i, int t) {
+        const uint32_t qaddr = smem_u32(qs + i * kTile2);
+        const uint32_t kaddr = smem_u32(kring + (t % kKSlots2) * kTile2);
+        const uint32_t d = tmem_base + (uint32_t)(i * kKeys);
+#pragma unroll
+        for (int k = 0; k < kDh / 16; ++k) {
+          const uint32_t off = (uint32_t)((k >> 2) * kHalf + (k & 3) * 32);
+          umma_bf16(d, sw128_desc(qaddr + off), sw128_desc(kaddr + off), idesc_s, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[i]);
+      };
+      auto issue_pv = [&](int i, int t) {
+        const uint32_t vaddr = smem_u32(vring + (t % kVSlots2) * kTile2);
+        const uint32_t pcol = tmem_base + (uint32_t)(i * kKeys);
+        const uint32_t ocol = tmem_base + kColO + (uint32_t)(i * kDh);
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k) {
+          const uint64_t bdesc = sw128_desc_mn(vaddr + (uint32_t)(k * 2048), kHalf);
+          umma_bf16_tmem_a(ocol, pcol + (uint32_t)(k * 8), bdesc, idesc_o,
+                           (t > 0 || k > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = (!p.q_tma || mbar_wait_bounded(q_full, 0, abort_flag));
+      for (int t = 0; ok && t <= n_tiles; ++t) {
+        const int tp = t - 1;   // the previous tile, whose P V runs now
+        if (tp >= 0) {
+          if (!mbar_wait_bounded(&p_full[0], (uint32_t)(tp & 1), abort_flag) ||
+              !mbar_wait_bounded(&v_full[tp % kVSlots2], (uint32_t)((tp / kVSlots2) & 1),
+                                 abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(0, tp);
+        }
+        if (t < n_tiles) {
+          if (!mbar_wait_bounded(&k_full[t % kKSlots2], (uint32_t)((t / kKSlots2) & 1),
+                                 abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (t == 0) DLM_TRACE_MARK(3);
+          tc_fence_after();
+          issue_s(0, t);
+        }
+        if (tp >= 0) {
+          if (!mbar_wait_bounded(&p_full[1], (uint32_t)(tp & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(1, tp);
+          umma_commit(&v_empty[tp % kVSlots2]);
+        }
+        if (t < n_tiles) {
+          issue_s(1, t);
+          umma_commit(&k_empty[t % kKSlots2]);
+        }
+      }
+      // O complete (or, after an abort, every MMA issued has finished)
+      umma_commit(o_done);
+      mbar_wait_bounded(o_done, 0, nullptr);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int tile = (warp - 2) >> 2;                 // row tile of this warpgroup
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;                 // row within the tile = TMEM lane
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_col = (uint32_t)(tile * kKeys);
+    const uint32_t o_col = kColO + (uint32_t)(tile * kDh);
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      if (!mbar_wait_bounded(&s_full[tile], (uint32_t)(t & 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // two passes over S in tensor memory (64 columns live at a time): the
+      // tile maximum, then P = exp2(S * scale - m) written over S as bf16
+      // pairs; keys past the split's end (ragged last tile) count as -inf
+      const int key_base = k_begin + t * kKeys;
+      const int n_valid = min(kKeys, k_end - key_base);
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t raw[2][32];
+        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64), raw[0]);
+        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64 + 32), raw[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float v = __uint_as_float(raw[j >> 5][j & 31]);
+          mx = fmaxf(mx, h * 64 + j < n_valid ? v : -CUDART_INF_F);
+        }
+      }
+      const float m_new = fmaxf(m_run, mx * p.scale_log2);
+      const float alpha = fast_exp2(m_run - m_new);
+      float rsum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t raw[2][32];
+        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64), raw[0]);
+        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64 + 32), raw[1]);
+        tmem_wait_ld();
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int k0 = h * 64 + 2 * j;
+          const float s0 = __uint_as_float(raw[(2 * j) >> 5][(2 * j) & 31]);
+          const float s1 = __uint_as_float(raw[(2 * j + 1) >> 5][(2 * j + 1) & 31]);
+          const float e0 = k0 < n_valid ? fast_exp2(fmaf(s0, p.scale_log2, -m_new)) : 0.f;
+          const float e1 = k0 + 1 < n_valid ? fast_exp2(fmaf(s1, p.scale_log2, -m_new)) : 0.f;
+          rsum += e0 + e1;
+          w[j] = pack_bf16(e0, e1);
+        }
+        tmem_st32_u(lane_addr + s_col + (uint32_t)(h * 32), w);
+      }
+      l_run = l_run * alpha + rsum;
+      m_run = m_new;
+      // O_i holds every earlier P_i V (see the MMA order above): rescale it
+      // only when some row of the warp saw a new maximum
+      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < kDh / 32; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + o_col + (uint32_t)(c * 32), o);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] *= alpha;
+          tmem_st32(lane_addr + o_col + (uint32_t)(c * 32), o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[tile]);
+    }
+    if (ok && mbar_wait_bounded(o_done, 0, abort_flag)) {
+      tc_fence_after();
+      if (row == 0 && tile == 0) DLM_TRACE_MARK(4);
+      // O in chunks of 32 columns: bf16 rows (one split) or f32 partials
+      const int r = row_base + tile * kRowsCta + row;
+      const bool live = r < p.R;
+      const int i = r / p.G, hh = r - i * p.G;
+      __nv_bfloat16* dst = p.o + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh;
+      const size_t slot = ((size_t)bg * p.nsplit + split) * p.R + r;
+      const float inv = 1.f / l_run;
+#pragma unroll 1
+      for (int c = 0; c < kDh / 32; ++c) {
+        float ov[32];
+        tmem_ld32(lane_addr + o_col + (uint32_t)(c * 32), ov);
+        if (!live) continue;
+        if (p.nsplit == 1) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = pack_bf16(ov[8 * q4 + 0] * inv, ov[8 * q4 + 1] * inv);
+            w.y = pack_bf16(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv);
+            w.z = pack_bf16(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv);
+            w.w = pack_bf16(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv);
+            reinterpret_cast<uint4*>(dst + c * 32)[q4] = w;
+          }
+        } else {
+          float4* pd = reinterpret_cast<float4*>(p.opart + slot * kDh + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            pd[q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
+        }
+      }
+      if (live && p.nsplit > 1) p.ml[slot] = make_float2(m_run, l_run);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  if (tid == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
+}
+
 // log-sum-exp combination of the splits of one (sequence, KV head); one warp
 // per query row, lane = 4 head-dim columns.  The split weights are computed
 // in parallel (lane s holds split s), then the partial rows are read in
@@ -656,11 +1015,21 @@ cudaError_t attn_set_attributes() {
   return done;
 }
 
+cudaError_t attn2_set_attributes() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaErrorNotReady)
+    done = cudaFuncSetAttribute(attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kAttn2Smem);
+  return done;
+}
+
 cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q, void* o,
                            float* opart, float2* ml, const int32_t* lens, const uint8_t* done,
                            const int* n_active, int* err, cudaStream_t st) {
   if (cudaError_t e = attn_set_attributes(); e != cudaSuccess) return e;
+  if (ap.rows == 2 * kRowsCta)
+    if (cudaError_t e = attn2_set_attributes(); e != cudaSuccess) return e;
   AttnParams p;
   p.q = (const __nv_bfloat16*)q;
   p.o = (__nv_bfloat16*)o;
@@ -682,6 +1051,20 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
   p.Lcap = md.Lcap;
   const CUtensorMap qmap = tmQ != nullptr ? *tmQ : tmK;   // unread without q_tma
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)md.Dh));
+  if (ap.rows == 2 * kRowsCta) {
+    // two row tiles per CTA: one split writes O, more write partials
+    if (ap.cluster > 1) return cudaErrorInvalidValue;
+    dim3 grid2(ap.nsplit, (ap.rtiles + 1) / 2, ap.B * md.Hkv);
+    cudaError_t e = launch_pdl(attn_tc2_kernel, grid2, dim3(320), kAttn2Smem, st, tmK, tmV,
+                               qmap, p);
+    if (e != cudaSuccess || ap.nsplit == 1) return e;
+    const int rows_per_block = 8;
+    dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);
+    return launch_pdl(attn_combine_kernel, g2, dim3(32 * rows_per_block), 0, st,
+                      (const float*)opart, (const float2*)ml, (__nv_bfloat16*)o, lens, done,
+                      n_active, md.H, md.Hkv, ap.G, ap.C, ap.R, ap.chunk, ap.nsplit);
+  }
+  if (ap.rows != kRowsCta) return cudaErrorInvalidValue;
   dim3 grid(ap.nsplit, ap.rtiles, ap.B * md.Hkv);
   if (ap.cluster > 1) {
     // the splits of a (row tile, plane) as one cluster: no partials, no combine kernel

@@ -137,14 +137,15 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag) {
+                                                  volatile int* abort_flag,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         if (abort_flag) *abort_flag = 1;
         return false;
       }
@@ -268,6 +269,49 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint6
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// kind::mxf4nvf4 with block scaling: both operands e2m1 (format code 1),
+// K-major, e4m3 scale factors (scale format 0), one per 16 elements, f32
+// accumulation, K = 64 per instruction.  Scale-factor byte ids 0.
+__host__ __device__ constexpr uint32_t idesc_nvfp4_f32(int M, int N) {
+  return (1u << 7)                      // A format e2m1
+         | (1u << 10)                   // B format e2m1
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// D (TMEM) (+)= (A x SFA) (B x SFB), NVFP4 operands in shared memory, the
+// scale factors in tensor memory at sfa_tmem / sfb_tmem
+__device__ __forceinline__ void umma_nvfp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared-memory descriptor of 32 rows x 16 bytes stored contiguously (no
+// swizzle): 8-row groups 128 bytes apart
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // start address (16-byte units)
+  d |= (uint64_t)1 << 16;                       // leading byte offset (one 16-byte column)
+  d |= (uint64_t)(128 >> 4) << 32;              // stride byte offset: 8 rows x 16 B
+  d |= (uint64_t)1 << 46;                       // descriptor version for sm_100
+  return d;                                     // layout type 0: no swizzle
+}
+
+// 32 rows x 128 bits from shared memory into tensor memory at `taddr`,
+// the same rows written to each of the four 32-lane quadrants (lane
+// 32q + r, 4 columns, holds row r)
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,

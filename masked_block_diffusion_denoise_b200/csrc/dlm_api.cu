@@ -6,7 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -52,7 +54,12 @@ struct dlm_ctx {
   bool bf16 = true;
   // e4m3 LM head: quantised weights, their scales, the step's quantised rows
   bool lm_f8 = false;
+  // NVFP4 LM head: as above with packed e2m1 elements and, in addition, the
+  // e4m3 block scales of weights and rows in the block-scaled MMA's layout
+  bool lm_f4 = false;
   uint8_t *w_lm_q = nullptr, *yq = nullptr;
+  uint8_t *lm_sf = nullptr, *y_sf = nullptr;
+  size_t lm_sf_bytes = 0, y_sf_bytes = 0;
   float *s_lm = nullptr, *s_y = nullptr;
   size_t s_lm_count = 0;
   size_t es = 2;
@@ -91,6 +98,7 @@ struct dlm_ctx {
   cudaStream_t cap = nullptr;
   std::string msg;
   int launches = 0;
+  int withhold_gemms = 0;   // failure-detection test: GEMM launches left to starve
   // measurement hook: events around one stage
   int ev_stage = -1;
   std::vector<cudaEvent_t> ev;
@@ -226,12 +234,19 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
   if (epi == EPI_LM) {
     p.BN = mt > 1 ? 256 : 128;
     p.f8 = ctx->lm_f8 ? 1 : 0;
+    p.f4 = ctx->lm_f4 ? 1 : 0;
+    if (ctx->lm_f4) p.BN = 128;   // scale-factor columns fit tensor memory beside 2 x 128
     return p;
   }
   if (mt > 1) {
-    // tensor-bound: 256-wide tiles (less L2 traffic per flop), K not split,
-    // so the projection epilogues can be fused into the GEMM
-    p.BN = 256;
+    // tensor-bound: K not split, so the projection epilogues can be fused
+    // into the GEMM; 256-wide tiles (less shared-memory and L2 traffic per
+    // flop) unless 128-wide ones fill the SMs' waves clearly better
+    auto wave_eff = [&](int bn) {
+      const int tiles = mt * cdiv(N, bn);
+      return (double)tiles / ((double)cdiv(tiles, ctx->num_sms) * ctx->num_sms);
+    };
+    p.BN = wave_eff(128) > wave_eff(256) + 0.05 ? 128 : 256;
     return p;
   }
   // one M tile: weight-read bound; split K over as many CTAs as fit in one
@@ -244,16 +259,23 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
   return p;
 }
 
-// Split plan of the attention.  For every split count (with the smallest
-// chunk of whole 128-key tiles that gives it) the CTAs are list-scheduled in
-// launch order (split fastest) onto the SMs with a per-CTA and a per-tile
-// time; ragged prefixes (lens, host) are taken as they are.  Up to 16 splits
-// may combine inside a thread-block cluster (an exchange cost per CTA) when
-// the whole grid fits in one wave of resident clusters; otherwise splits
-// write partials for the combine kernel (a write cost per CTA, the kernel, a
-// cost per partial).  Costs in microseconds, from B200 measurements: a tile
-// takes ~1.2 us in a lone CTA and ~1.7 us when every SM streams K/V.
-AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int max_len_all) {
+// Split plan of the attention.  For each CTA shape (128 query rows, or 256
+// = two row tiles of the same KV head when it has that many rows) and every
+// split count (with the smallest chunk of whole 128-key tiles that gives it)
+// the CTAs are list-scheduled in launch order (split fastest) onto the SMs
+// with a per-CTA and a per-tile time; ragged prefixes (lens, host) are taken
+// as they are.  Up to 16 splits of 128-row CTAs may combine inside a
+// thread-block cluster (an exchange cost per CTA) when the whole grid fits in
+// one wave of resident clusters; otherwise splits write partials for the
+// combine kernel (a write cost per CTA, the kernel, a cost per partial).
+// Costs in microseconds, from B200 measurements: a 128-row tile of 128 keys
+// takes ~1.2 us in a lone CTA and ~1.7 us when every SM streams K/V; a
+// 256-row CTA reads each tile once for both row tiles.
+// max_part_slots > 0 bounds the partial row slots (B * Hkv * nsplit * R) of
+// plans that combine through the combine kernel; one split (no partials) and
+// cluster plans always qualify.
+AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int max_len_all,
+                        long max_part_slots = 0) {
   AttnPlan a{};
   a.B = B;
   a.C = C;
@@ -264,7 +286,7 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
   const int sms = std::min(std::max(ctx->num_sms, 1), 1024);
   const int max_keys = max_len_all + C;
   const int max_tiles = cdiv(max_keys, 128);
-  const double t_tile = 1.5, t_cta = 3.0, t_xchg = 1.5, t_pw = 1.5, t_comb = 4.0, t_part = 0.03;
+  const double t_xchg = 1.5, t_pw = 1.5, t_comb = 4.0, t_part = 0.03;
   double best = -1.0;
   double sm_free[1024];   // no heap allocation: this also runs inside dlm_attention_noalloc
   // diagnostic switch: DLM_ATTN_CLUSTER=0 keeps every split plan on the
@@ -274,47 +296,70 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
   // diagnostic switch: DLM_ATTN_TILES=k plans only chunks of k key tiles
   const char* ct_env = std::getenv("DLM_ATTN_TILES");
   const int only_ct = ct_env != nullptr ? std::atoi(ct_env) : 0;
-  int last_nsplit = 0;
-  for (int ct = 1; ct <= max_tiles; ++ct) {
-    if (only_ct > 0 && ct != std::min(only_ct, max_tiles)) continue;
-    const int chunk = ct * 128;
-    const int nsplit = cdiv(max_keys, chunk);
-    if (nsplit > 64) continue;   // the combine kernel holds up to 64 splits
-    if (nsplit == last_nsplit) continue;   // a larger chunk for the same split count
-    last_nsplit = nsplit;
-    const long ctas = (long)B * Hkv * a.rtiles * nsplit;
-    int cl = 1;
-    if (nsplit > 1 && nsplit <= 16 && cluster_ok) {
-      const int cap = attn_cluster_capacity(nsplit);
-      if (cap > 0 && ctas <= (long)cap * nsplit) cl = nsplit;
-    }
-    const double per_cta = t_cta + (cl > 1 ? t_xchg : (nsplit > 1 ? t_pw : 0.0));
-    // SMs as a min-heap of finish times (negated for the max-heap functions)
-    std::fill(sm_free, sm_free + sms, 0.0);
-    long partials = 0;
-    double makespan = 0.0;
-    for (int bg = 0; bg < B * Hkv; ++bg) {
-      const int keys = (lens ? lens[bg / Hkv] : max_len_all) + C;
-      for (int rt = 0; rt < a.rtiles; ++rt) {
-        for (int sp = 0; sp < nsplit; ++sp) {
-          const int k0 = sp * chunk;
-          if (k0 >= keys && cl == 1) continue;   // exits at once
-          const int tiles = k0 < keys ? cdiv(std::min(chunk, keys - k0), 128) : 0;
-          std::pop_heap(sm_free, sm_free + sms);   // earliest free SM to the back
-          sm_free[sms - 1] -= per_cta + tiles * t_tile;
-          makespan = std::max(makespan, -sm_free[sms - 1]);
-          std::push_heap(sm_free, sm_free + sms);
-          ++partials;
+  // diagnostic switch: DLM_ATTN_ROWS=128 or 256 plans only that CTA shape
+  const char* rows_env = std::getenv("DLM_ATTN_ROWS");
+  const int only_rows = rows_env != nullptr ? std::atoi(rows_env) : 0;
+  for (int rows = 128; rows <= 256; rows += 128) {
+    if (rows == 256 && a.rtiles < 2) continue;          // one row tile: nothing to pair
+    if (only_rows > 0 && rows != only_rows && !(only_rows == 256 && a.rtiles < 2)) continue;
+    const int ytiles = rows == 256 ? cdiv(a.rtiles, 2) : a.rtiles;   // CTAs per split
+    const double t_tile = rows == 256 ? 2.0 : 1.5;
+    const double t_cta = rows == 256 ? 3.5 : 3.0;
+    int last_nsplit = 0;
+    for (int ct = 1; ct <= max_tiles; ++ct) {
+      if (only_ct > 0 && ct != std::min(only_ct, max_tiles)) continue;
+      const int chunk = ct * 128;
+      const int nsplit = cdiv(max_keys, chunk);
+      if (nsplit > 64) continue;   // the combine kernel holds up to 64 splits
+      if (nsplit == last_nsplit) continue;   // a larger chunk for the same split count
+      last_nsplit = nsplit;
+      const long ctas = (long)B * Hkv * ytiles * nsplit;
+      int cl = 1;
+      if (rows == 128 && nsplit > 1 && nsplit <= 16 && cluster_ok) {
+        const int cap = attn_cluster_capacity(nsplit);
+        if (cap > 0 && ctas <= (long)cap * nsplit) cl = nsplit;
+      }
+      if (cl == 1 && nsplit > 1 && max_part_slots > 0 &&
+          (long)B * Hkv * nsplit * a.R > max_part_slots)
+        continue;   // the partials would not fit the caller's fixed scratch
+      const double per_cta =
+          t_cta + (cl > 1 ? t_xchg : (nsplit > 1 ? t_pw * rows / 128 : 0.0));
+      // SMs as a min-heap of finish times (negated for the max-heap functions)
+      std::fill(sm_free, sm_free + sms, 0.0);
+      long partials = 0;
+      double makespan = 0.0;
+      for (int bg = 0; bg < B * Hkv; ++bg) {
+        const int keys = (lens ? lens[bg / Hkv] : max_len_all) + C;
+        for (int rt = 0; rt < ytiles; ++rt) {
+          for (int sp = 0; sp < nsplit; ++sp) {
+            const int k0 = sp * chunk;
+            if (k0 >= keys && cl == 1) continue;   // exits at once
+            const int tiles = k0 < keys ? cdiv(std::min(chunk, keys - k0), 128) : 0;
+            std::pop_heap(sm_free, sm_free + sms);   // earliest free SM to the back
+            sm_free[sms - 1] -= per_cta + tiles * t_tile;
+            makespan = std::max(makespan, -sm_free[sms - 1]);
+            std::push_heap(sm_free, sm_free + sms);
+            partials += rows / 128;
+          }
         }
       }
+      const double cost = makespan + (nsplit > 1 && cl == 1 ? t_comb + t_part * partials : 0.0);
+      if (best < 0.0 || cost < best - 1e-9) {
+        best = cost;
+        a.chunk = chunk;
+        a.nsplit = nsplit;
+        a.cluster = cl;
+        a.rows = rows;
+      }
     }
-    const double cost = makespan + (nsplit > 1 && cl == 1 ? t_comb + t_part * partials : 0.0);
-    if (best < 0.0 || cost < best - 1e-9) {
-      best = cost;
-      a.chunk = chunk;
-      a.nsplit = nsplit;
-      a.cluster = cl;
-    }
+  }
+  if (best < 0.0) {
+    // nothing qualified (a forced chunk size whose partials do not fit the
+    // caller's scratch): one split of 128-row CTAs needs no partials
+    a.chunk = max_tiles * 128;
+    a.nsplit = 1;
+    a.cluster = 1;
+    a.rows = 128;
   }
   return a;
 }
@@ -444,14 +489,22 @@ SelectArgs make_select(const dlm_ctx* ctx, const dlm_sampler_params* p, int batc
 
 // one GEMM through the engine of the model's element type
 int run_gemm(dlm_ctx* ctx, const void* A, const void* B, int Brows, const GemmPlan& plan,
-             const GemmIO& io, cudaStream_t st) {
+             const GemmIO& io_in, cudaStream_t st) {
   cudaError_t e;
+  GemmIO io = io_in;
+  // the failure-detection hook applies to launches issued directly, never to
+  // a graph being captured (a captured launch would starve on every replay)
+  if (ctx->withhold_gemms > 0 && ctx->bf16 && st != ctx->cap) {
+    io.withhold_loads = 1;
+    --ctx->withhold_gemms;
+  }
   if (ctx->bf16) {
-    const bool u8 = plan.f8 != 0;
-    const CUtensorMap* ta = map2d(ctx, A, (uint64_t)ctx->Mmax, (uint64_t)plan.K,
-                                  (uint32_t)gemm_tc_a_rows(plan.M), u8);
-    const CUtensorMap* tb =
-        map2d(ctx, B, (uint64_t)Brows, (uint64_t)plan.K, (uint32_t)plan.BN, u8);
+    // 8- and 4-bit operands are mapped as bytes: K bytes (e4m3) or K / 2 (NVFP4)
+    const bool u8 = plan.f8 != 0 || plan.f4 != 0;
+    const uint64_t cols = plan.f4 ? (uint64_t)plan.K / 2 : (uint64_t)plan.K;
+    const CUtensorMap* ta =
+        map2d(ctx, A, (uint64_t)ctx->Mmax, cols, (uint32_t)gemm_tc_a_rows(plan.M), u8);
+    const CUtensorMap* tb = map2d(ctx, B, (uint64_t)Brows, cols, (uint32_t)plan.BN, u8);
     if (ta == nullptr || tb == nullptr)
       return fail(ctx, DLM_ECUDA, "cuTensorMapEncodeTiled failed");
     e = gemm_tc(*ta, *tb, plan, io, ctx->num_sms, st);
@@ -520,7 +573,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.n_active = ctx->n_active;
     io.err = ctx->err;
     io.trace_kind = TRACE_QKV_GEMM;
-    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN >= 128 && cdiv(rows, 128) > 1;
     if (fused) {
       pl.epi = EPI_QKV;
       io.done = c->done;
@@ -559,7 +612,7 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.n_active = ctx->n_active;
     io.err = ctx->err;
     io.trace_kind = TRACE_WO_GEMM;
-    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+    const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN >= 128 && cdiv(rows, 128) > 1;
     if (fused) {
       pl.epi = EPI_RESID;
       io.done = c->done;
@@ -585,7 +638,19 @@ int enqueue_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler
     io.n_active = ctx->n_active;
     io.err = ctx->err;
     io.trace_kind = TRACE_LM_HEAD;
-    if (ctx->lm_f8) {
+    if (ctx->lm_f4) {
+      // NVFP4 head: the rows are quantised first (elements, block scales, row
+      // scales); block scales enter the MMA, row scales the epilogue
+      e = quantize_rows_nvfp4(ctx->y, rows, md.d, ctx->yq, ctx->y_sf, ctx->s_y, C, c->done,
+                              ctx->n_active, st);
+      if (e != cudaSuccess) return cuda_fail(ctx, "quantize rows (NVFP4)", e);
+      ++ctx->launches;
+      io.epi.row_scale = ctx->s_y;
+      io.epi.col_scale = ctx->s_lm;
+      io.sfa = ctx->y_sf;
+      io.sfb = ctx->lm_sf;
+      if (int rc = run_gemm(ctx, ctx->yq, ctx->w_lm_q, md.V, pl, io, st)) return rc;
+    } else if (ctx->lm_f8) {
       // e4m3 head: the rows are quantised first, the scales enter the epilogue
       e = quantize_rows_e4m3(ctx->y, rows, md.d, ctx->yq, ctx->s_y, C, c->done, ctx->n_active,
                              st);
@@ -624,7 +689,7 @@ int enqueue_clean_pass(dlm_ctx* ctx, const int32_t* tokens, int batch, int C, cu
   GemmIO io;
   io.out = ctx->part;
   io.err = ctx->err;
-  const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN == 256;
+  const bool fused = ctx->bf16 && pl.splits == 1 && pl.BN >= 128 && cdiv(rows, 128) > 1;
   if (fused) {
     pl.epi = EPI_QKV;
     io.proj = proj_epi(ctx, C);
@@ -695,14 +760,19 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
     return fail(nullptr, DLM_EINVAL, "need max_batch >= 1, max_prefix >= 0, 1 <= max_canvas <= 1024");
   if (!w->emb || !w->w_q || !w->w_k || !w->w_v || !w->w_o || !w->w_lm)
     return fail(nullptr, DLM_EINVAL, "every weight pointer must be non-NULL");
-  if (d.lm_fp8 != 0 && d.lm_fp8 != 1) return fail(nullptr, DLM_EINVAL, "lm_fp8 must be 0 or 1");
-  if (d.lm_fp8 && (d.dtype != DLM_BF16 || d.d_model % 16 != 0))
-    return fail(nullptr, DLM_EINVAL, "lm_fp8 needs a bf16 model with d_model % 16 == 0");
+  if (d.lm_quant != DLM_LM_MODEL && d.lm_quant != DLM_LM_E4M3 && d.lm_quant != DLM_LM_NVFP4)
+    return fail(nullptr, DLM_EINVAL, "lm_quant must be DLM_LM_MODEL, DLM_LM_E4M3 or DLM_LM_NVFP4");
+  if (d.lm_quant == DLM_LM_E4M3 && (d.dtype != DLM_BF16 || d.d_model % 16 != 0))
+    return fail(nullptr, DLM_EINVAL, "the e4m3 LM head needs a bf16 model with d_model % 16 == 0");
+  if (d.lm_quant == DLM_LM_NVFP4 && (d.dtype != DLM_BF16 || d.d_model % 256 != 0))
+    return fail(nullptr, DLM_EINVAL,
+                "the NVFP4 LM head needs a bf16 model with d_model % 256 == 0");
 
   dlm_ctx* ctx = new dlm_ctx();
   ctx->d = d;
   ctx->bf16 = d.dtype == DLM_BF16;
-  ctx->lm_f8 = d.lm_fp8 == 1;
+  ctx->lm_f8 = d.lm_quant == DLM_LM_E4M3;
+  ctx->lm_f4 = d.lm_quant == DLM_LM_NVFP4;
   ctx->es = ctx->bf16 ? 2 : 4;
   cudaGetDevice(&ctx->dev);
   cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->dev);
@@ -754,12 +824,21 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if ((rc = dalloc(ctx, &ctx->h_stable, d.max_batch * sizeof(int32_t)))) return bail(rc);
   ctx->part_floats = part_floats_needed(ctx);
   if ((rc = dalloc(ctx, &ctx->part, ctx->part_floats * sizeof(float)))) return bail(rc);
-  if (ctx->lm_f8) {
+  if (ctx->lm_f8 || ctx->lm_f4) {
+    // one byte per element (e4m3) or two elements per byte (NVFP4)
+    const size_t row_bytes = ctx->lm_f4 ? dm / 2 : dm;
     ctx->s_lm_count = (size_t)cdiv(d.vocab, 256) * 256;   // whole tiles of either width
-    if ((rc = dalloc(ctx, &ctx->w_lm_q, (size_t)d.vocab * dm))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->w_lm_q, (size_t)d.vocab * row_bytes))) return bail(rc);
     if ((rc = dalloc(ctx, &ctx->s_lm, ctx->s_lm_count * sizeof(float)))) return bail(rc);
-    if ((rc = dalloc(ctx, &ctx->yq, ctx->Mmax * dm))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->yq, ctx->Mmax * row_bytes))) return bail(rc);
     if ((rc = dalloc(ctx, &ctx->s_y, ctx->Mmax * sizeof(float)))) return bail(rc);
+  }
+  if (ctx->lm_f4) {
+    // block scales: [row block of 128][d / 64][512 bytes]
+    ctx->lm_sf_bytes = (size_t)cdiv(d.vocab, 128) * (dm / 64) * 512;
+    ctx->y_sf_bytes = (size_t)cdiv(ctx->Mmax, 128) * (dm / 64) * 512;
+    if ((rc = dalloc(ctx, &ctx->lm_sf, ctx->lm_sf_bytes))) return bail(rc);
+    if ((rc = dalloc(ctx, &ctx->y_sf, ctx->y_sf_bytes))) return bail(rc);
   }
 
   cudaError_t e = cudaSuccess;
@@ -785,6 +864,16 @@ int dlm_create(const dlm_model_desc* desc, const dlm_weights* w, dlm_ctx** out) 
   if (d.rope_theta > 0.0f)
     ck(rope_table_init(ctx->rope, ctx->Lcap, d.head_dim, (double)d.rope_theta, nullptr),
        "rope table");
+  if (ctx->lm_f4) {
+    ck(cudaMemset(ctx->s_lm, 0, ctx->s_lm_count * sizeof(float)), "memset LM scales");
+    ck(cudaMemset(ctx->yq, 0, ctx->Mmax * dm / 2), "memset quantised rows");
+    ck(cudaMemset(ctx->s_y, 0, ctx->Mmax * sizeof(float)), "memset row scales");
+    ck(cudaMemset(ctx->lm_sf, 0, ctx->lm_sf_bytes), "memset LM block scales");
+    ck(cudaMemset(ctx->y_sf, 0, ctx->y_sf_bytes), "memset row block scales");
+    ck(quantize_rows_nvfp4(w->w_lm, d.vocab, d.d_model, ctx->w_lm_q, ctx->lm_sf, ctx->s_lm, 1,
+                           nullptr, nullptr, nullptr),
+       "quantise LM head (NVFP4)");
+  }
   if (ctx->lm_f8) {
     ck(cudaMemset(ctx->s_lm, 0, ctx->s_lm_count * sizeof(float)), "memset LM scales");
     ck(cudaMemset(ctx->yq, 0, ctx->Mmax * dm), "memset quantised rows");
@@ -891,20 +980,23 @@ int dlm_denoise_step(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   return enqueue_step(ctx, c, batch, p, stats, ap, (cudaStream_t)stream);
 }
 
-int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
-                     dlm_canvas_stats* stats, void* stream) {
-  if (ctx == nullptr) return DLM_EINVAL;
-  ctx->msg.clear();
-  if (int rc = check_params(ctx, p, batch)) return rc;
-  if (int rc = check_canvas(ctx, c, p)) return rc;
+}  // extern "C"
+
+namespace {
+
+// `n_steps` denoising steps as one CUDA graph, captured once per
+// configuration (pointers, sizes, parameters, attention plan, step count) and
+// replayed on `stream`
+int decode_steps_graph(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                       int n_steps, dlm_canvas_stats* stats, void* stream) {
   AttnPlan ap = plan_attention_cached(ctx, batch, p->canvas, max_len(ctx, batch));
   if (ctx->bf16)
     if (int rc = ensure_attn_scratch(ctx, ap)) return rc;
   // the graph bakes in pointers, sizes, parameters and the attention plan
-  std::vector<uint8_t> key(sizeof(int) * 4 + sizeof(dlm_sampler_params) + sizeof(dlm_canvas) +
+  std::vector<uint8_t> key(sizeof(int) * 5 + sizeof(dlm_sampler_params) + sizeof(dlm_canvas) +
                            sizeof(void*) * 3 + ctx->ev.size() * sizeof(cudaEvent_t));
   uint8_t* kp = key.data();
-  const int hdr[4] = {batch, ap.chunk, ap.nsplit, ctx->ev_stage};
+  const int hdr[5] = {batch, ap.chunk, ap.nsplit, ctx->ev_stage, n_steps};
   const void* ptrs[3] = {stats, ctx->opart, ctx->ml};
   std::memcpy(kp, hdr, sizeof(hdr));
   kp += sizeof(hdr);
@@ -929,7 +1021,7 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
     ctx->launches = 0;
     ctx->ev_step = 0;
     int rc = DLM_OK;
-    for (int s = 0; s < p->steps && rc == DLM_OK; ++s)
+    for (int s = 0; s < n_steps && rc == DLM_OK; ++s)
       rc = enqueue_step(ctx, c, batch, p, stats, ap, ctx->cap);
     cudaError_t ce = cudaStreamEndCapture(ctx->cap, &graph);
     if (rc != DLM_OK) {
@@ -939,7 +1031,7 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
     if (ce != cudaSuccess) return cuda_fail(ctx, "cudaStreamEndCapture", ce);
     GraphEntry g;
     g.key = key;
-    g.launches = ctx->launches / p->steps;
+    g.launches = ctx->launches / n_steps;
     ce = cudaGraphInstantiate(&g.exec, graph, 0);
     cudaGraphDestroy(graph);
     if (ce != cudaSuccess) return cuda_fail(ctx, "cudaGraphInstantiate", ce);
@@ -948,6 +1040,47 @@ int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sam
   }
   ctx->launches = ge->launches;
   CK(cudaGraphLaunch(ge->exec, (cudaStream_t)stream));
+  return DLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dlm_decode_block(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                     dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
+  return decode_steps_graph(ctx, c, batch, p, p->steps, stats, stream);
+}
+
+int dlm_decode_steps(dlm_ctx* ctx, const dlm_canvas* c, int batch, const dlm_sampler_params* p,
+                     int n_steps, dlm_canvas_stats* stats, void* stream) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (int rc = check_params(ctx, p, batch)) return rc;
+  if (int rc = check_canvas(ctx, c, p)) return rc;
+  if (n_steps < 1 || n_steps > p->steps)
+    return fail(ctx, DLM_EINVAL, "n_steps must be in [1, params->steps]");
+  return decode_steps_graph(ctx, c, batch, p, n_steps, stats, stream);
+}
+
+int dlm_attention_plan(dlm_ctx* ctx, int batch, int canvas, int* nsplit, int* chunk,
+                       int* cluster, int* rows_per_cta) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (!nsplit || !chunk || !cluster || !rows_per_cta)
+    return fail(ctx, DLM_EINVAL, "attention_plan: NULL output pointer");
+  if (!ctx->bf16) return fail(ctx, DLM_EINVAL, "attention_plan: the fp32 model has no split plan");
+  if (batch < 1 || batch > ctx->d.max_batch || canvas < 1 || canvas > ctx->d.max_canvas)
+    return fail(ctx, DLM_EINVAL, "attention_plan: batch or canvas out of range");
+  const AttnPlan ap = plan_attention_cached(ctx, batch, canvas, max_len(ctx, batch));
+  *nsplit = ap.nsplit;
+  *chunk = ap.chunk;
+  *cluster = ap.cluster;
+  *rows_per_cta = ap.rows;
   return DLM_OK;
 }
 
@@ -1065,21 +1198,30 @@ int dlm_debug_buffer(dlm_ctx* ctx, int which, void** ptr, size_t* bytes) {
     case DLM_BUF_LM_Q:
     case DLM_BUF_LM_SCALE:
     case DLM_BUF_Y_Q:
-    case DLM_BUF_Y_SCALE:
-      if (!ctx->lm_f8) return fail(ctx, DLM_EINVAL, "the context has no e4m3 LM head");
+    case DLM_BUF_Y_SCALE: {
+      if (!ctx->lm_f8 && !ctx->lm_f4)
+        return fail(ctx, DLM_EINVAL, "the context has no low-bit LM head");
+      const size_t row_bytes = ctx->lm_f4 ? dm / 2 : dm;
       if (which == DLM_BUF_LM_Q) {
         *ptr = ctx->w_lm_q;
-        *bytes = (size_t)ctx->d.vocab * dm;
+        *bytes = (size_t)ctx->d.vocab * row_bytes;
       } else if (which == DLM_BUF_LM_SCALE) {
         *ptr = ctx->s_lm;
         *bytes = ctx->s_lm_count * 4;
       } else if (which == DLM_BUF_Y_Q) {
         *ptr = ctx->yq;
-        *bytes = M * dm;
+        *bytes = M * row_bytes;
       } else {
         *ptr = ctx->s_y;
         *bytes = M * 4;
       }
+      break;
+    }
+    case DLM_BUF_LM_SF:
+    case DLM_BUF_Y_SF:
+      if (!ctx->lm_f4) return fail(ctx, DLM_EINVAL, "the context has no NVFP4 LM head");
+      *ptr = which == DLM_BUF_LM_SF ? ctx->lm_sf : ctx->y_sf;
+      *bytes = which == DLM_BUF_LM_SF ? ctx->lm_sf_bytes : ctx->y_sf_bytes;
       break;
     default: return fail(ctx, DLM_EINVAL, "unknown buffer id");
   }
@@ -1098,6 +1240,13 @@ int dlm_debug_logits(dlm_ctx* ctx, int batch, int canvas, float* logits, void* s
   GemmIO io;
   io.out = logits;
   io.err = ctx->err;
+  if (ctx->lm_f4) {
+    io.epi.row_scale = ctx->s_y;
+    io.epi.col_scale = ctx->s_lm;
+    io.sfa = ctx->y_sf;
+    io.sfb = ctx->lm_sf;
+    return run_gemm(ctx, ctx->yq, ctx->w_lm_q, ctx->d.vocab, pl, io, (cudaStream_t)stream);
+  }
   if (ctx->lm_f8) {
     io.epi.row_scale = ctx->s_y;
     io.epi.col_scale = ctx->s_lm;
@@ -1120,6 +1269,15 @@ int dlm_check(dlm_ctx* ctx, void* stream) {
 }
 
 int dlm_launches_per_step(const dlm_ctx* ctx) { return ctx ? ctx->launches : DLM_EINVAL; }
+
+int dlm_test_withhold_loads(dlm_ctx* ctx, int n_launches) {
+  if (ctx == nullptr) return DLM_EINVAL;
+  ctx->msg.clear();
+  if (n_launches < 0) return fail(ctx, DLM_EINVAL, "n_launches must be >= 0");
+  if (!ctx->bf16) return fail(ctx, DLM_EINVAL, "the fp32 model has no tensor-core GEMM");
+  ctx->withhold_gemms = n_launches;
+  return DLM_OK;
+}
 
 int dlm_set_stage_events(dlm_ctx* ctx, int stage, void* const* events, int n_pairs) {
   if (ctx == nullptr) return DLM_EINVAL;
@@ -1204,14 +1362,65 @@ static __device__ __align__(256) int g_noalloc_err[1];
 
 namespace {
 
+// Device addresses of the arrays above, looked up once per device (host code
+// must not pass the arrays' names to a kernel: those are host stand-ins).
 struct NoAllocScratch {
-  bool ready = false;
+  std::once_flag once;
+  cudaError_t status = cudaErrorNotReady;
+  const char* what = "";
   float* opart = nullptr;
   float2* ml = nullptr;
   int* err = nullptr;
+  int num_sms = 0;
 };
 constexpr int kMaxDevices = 64;
 NoAllocScratch g_noalloc[kMaxDevices];
+
+// runs once per device, with that device current
+void noalloc_setup(NoAllocScratch& sc, int dev) {
+  void* p = nullptr;
+  cudaError_t e;
+  if ((e = cudaGetSymbolAddress(&p, g_noalloc_opart)) != cudaSuccess) {
+    sc.status = e;
+    sc.what = "cudaGetSymbolAddress(partials)";
+    return;
+  }
+  sc.opart = static_cast<float*>(p);
+  if ((e = cudaGetSymbolAddress(&p, g_noalloc_ml)) != cudaSuccess) {
+    sc.status = e;
+    sc.what = "cudaGetSymbolAddress(max/sum)";
+    return;
+  }
+  sc.ml = static_cast<float2*>(p);
+  if ((e = cudaGetSymbolAddress(&p, g_noalloc_err)) != cudaSuccess) {
+    sc.status = e;
+    sc.what = "cudaGetSymbolAddress(error word)";
+    return;
+  }
+  sc.err = static_cast<int*>(p);
+  if ((e = cudaDeviceGetAttribute(&sc.num_sms, cudaDevAttrMultiProcessorCount, dev)) !=
+      cudaSuccess) {
+    sc.status = e;
+    sc.what = "cudaDeviceGetAttribute(multiprocessor count)";
+    return;
+  }
+  sc.status = cudaSuccess;
+}
+
+// the current device's scratch in *out, set up on first use; a DLM status
+int noalloc_scratch(NoAllocScratch** out) {
+  *out = nullptr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(nullptr, "cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(nullptr, DLM_EINVAL, "attention_noalloc: device index out of range");
+  NoAllocScratch& sc = g_noalloc[dev];
+  std::call_once(sc.once, noalloc_setup, std::ref(sc), dev);
+  if (sc.status != cudaSuccess) return cuda_fail(nullptr, sc.what, sc.status);
+  *out = &sc;
+  return DLM_OK;
+}
 
 }  // namespace
 
@@ -1232,32 +1441,14 @@ int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cach
     return fail(nullptr, DLM_EINVAL,
                 "attention_noalloc: need 1 <= batch <= kv_batch and max_len + canvas <= "
                 "kv_capacity");
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(nullptr, "cudaGetDevice", e);
-  if (dev < 0 || dev >= kMaxDevices)
-    return fail(nullptr, DLM_EINVAL, "attention_noalloc: device index out of range");
-  NoAllocScratch& sc = g_noalloc[dev];
-  if (!sc.ready) {
-    // host code must not pass the arrays' names to a kernel: those are host
-    // stand-ins; the device addresses come from the runtime, once per device
-    void* p = nullptr;
-    if ((e = cudaGetSymbolAddress(&p, g_noalloc_opart)) != cudaSuccess)
-      return cuda_fail(nullptr, "cudaGetSymbolAddress(partials)", e);
-    sc.opart = static_cast<float*>(p);
-    if ((e = cudaGetSymbolAddress(&p, g_noalloc_ml)) != cudaSuccess)
-      return cuda_fail(nullptr, "cudaGetSymbolAddress(max/sum)", e);
-    sc.ml = static_cast<float2*>(p);
-    if ((e = cudaGetSymbolAddress(&p, g_noalloc_err)) != cudaSuccess)
-      return cuda_fail(nullptr, "cudaGetSymbolAddress(error word)", e);
-    sc.err = static_cast<int*>(p);
-    sc.ready = true;
-  }
-  // the split plan of dlm_denoise_step for these sizes
+  NoAllocScratch* sc = nullptr;
+  if (int rc = noalloc_scratch(&sc)) return rc;
+  // the split plan of dlm_denoise_step for these sizes, restricted to plans
+  // whose partials fit the fixed array (one split needs none, so one exists)
   dlm_ctx plan_ctx;
   plan_ctx.md = ModelDims{0, n_heads, n_kv_heads, head_dim, 0, -1, -1, kv_capacity, 2};
-  cudaDeviceGetAttribute(&plan_ctx.num_sms, cudaDevAttrMultiProcessorCount, dev);
-  const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, nullptr, max_len);
+  plan_ctx.num_sms = sc->num_sms;
+  const AttnPlan ap = plan_attention(&plan_ctx, batch, canvas, nullptr, max_len, kNoAllocSlots);
   const long slots = (long)batch * n_kv_heads * ap.nsplit * ap.R;
   if (ap.nsplit > 1 && ap.cluster <= 1 && slots > kNoAllocSlots) {
     g_create_error = "attention_noalloc: the split plan needs " + std::to_string(slots) +
@@ -1271,16 +1462,30 @@ int dlm_attention_noalloc(const void* q, const void* k_cache, const void* v_cach
       !map_kv(&tmV, const_cast<void*>(v_cache), planes, kv_capacity, head_dim))
     return fail(nullptr, DLM_ECUDA, "attention_noalloc: cuTensorMapEncodeTiled failed");
   cudaStream_t st = (cudaStream_t)stream;
-  if ((e = cudaMemsetAsync(sc.err, 0, sizeof(int), st)) != cudaSuccess)
-    return cuda_fail(nullptr, "cudaMemsetAsync(error word)", e);
   CUtensorMap tmQ;
   const bool has_q = map_q(&tmQ, const_cast<void*>(q), (uint64_t)batch * canvas, n_heads,
                            head_dim, (uint32_t)(n_heads / n_kv_heads));
-  e = attention_bf16(plan_ctx.md, ap, tmK, tmV, has_q ? &tmQ : nullptr, q, o, sc.opart, sc.ml,
-                     lens, nullptr, nullptr,
-                     sc.err, st);
+  cudaError_t e = attention_bf16(plan_ctx.md, ap, tmK, tmV, has_q ? &tmQ : nullptr, q, o,
+                                 sc->opart, sc->ml, lens, nullptr, nullptr, sc->err, st);
   if (e != cudaSuccess) return cuda_fail(nullptr, "attention_noalloc launch", e);
   return DLM_OK;
+}
+
+int dlm_attention_noalloc_check(void* stream) {
+  g_create_error.clear();
+  NoAllocScratch* sc = nullptr;
+  if (int rc = noalloc_scratch(&sc)) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(nullptr, "cudaStreamSynchronize", e);
+  int word = 0;
+  if ((e = cudaMemcpy(&word, sc->err, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(nullptr, "read the no-alloc error word", e);
+  if (word == 0) return DLM_OK;
+  if ((e = cudaMemset(sc->err, 0, sizeof(int))) != cudaSuccess)
+    return cuda_fail(nullptr, "clear the no-alloc error word", e);
+  return fail(nullptr, word, word == DLM_ETIMEOUT ? "attention_noalloc: device wait timed out"
+                                                  : "attention_noalloc: device index check failed");
 }
 
 }  // extern "C"

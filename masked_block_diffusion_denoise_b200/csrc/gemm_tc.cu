@@ -57,17 +57,22 @@ struct TcCfg {
   static constexpr int kSmem = 232448;        // the opt-in maximum per block
 };
 
-__host__ __device__ constexpr int tc_stage_bytes(int BN, int a_rows) { return (BN + a_rows) * 128; }
-__host__ __device__ constexpr int tc_bar_offset(int BN, int a_rows, int stages) {
-  return stages * tc_stage_bytes(BN, a_rows) + (128 - a_rows) * 128;
+// sf: bytes of block scale factors per stage (NVFP4: 2 KB for the A rows'
+// 128-row block, 2 KB per 128 B rows), after the A tile
+__host__ __device__ constexpr int tc_stage_bytes(int BN, int a_rows, int sf = 0) {
+  return (BN + a_rows) * 128 + sf;
+}
+__host__ __device__ constexpr int tc_bar_offset(int BN, int a_rows, int stages, int sf = 0) {
+  return stages * tc_stage_bytes(BN, a_rows, sf) + (128 - a_rows) * 128;
 }
 template <int BN>
-constexpr int tc_stages(int a_rows) {
+constexpr int tc_stages(int a_rows, int sf = 0) {
   using Cfg = TcCfg<BN>;
   const int room = Cfg::kSmem - 1024 - Cfg::kBarBytes - Cfg::kXchBytes - (128 - a_rows) * 128;
-  const int n = room / tc_stage_bytes(BN, a_rows);
+  const int n = room / tc_stage_bytes(BN, a_rows, sf);
   return n < Cfg::kMaxStages ? n : Cfg::kMaxStages;
 }
+__host__ __device__ constexpr int tc_sf_bytes(int BN, bool f4) { return f4 ? 2048 * (1 + BN / 128) : 0; }
 
 struct TcParams {
   int M, N, K;
@@ -81,6 +86,15 @@ struct TcParams {
   const int* n_active;   // whole launch skipped when *n_active == 0
   int* err;
   int trace_kind;        // device timeline (DLM_TRACE builds), -1: not traced
+  // failure-detection test: the producer issues no loads, so the MMA warp's
+  // waits for them run out after wait_ns and the launch records DLM_ETIMEOUT
+  int withhold_loads;
+  uint64_t wait_ns;      // limit of the MMA warp's waits for ring stages
+  // NVFP4 operands: block scale factors of A and B in the block-scaled MMA's
+  // layout, [row block of 128][k group of 64][512 bytes]; kg = K / 64
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int kg;
 };
 
 __device__ __forceinline__ void unit_coords(const TcParams& p, int u, int& m, int& n, int& kb0,
@@ -135,13 +149,23 @@ __device__ __forceinline__ void scale_chunk(float (&v)[32], float a, const float
 
 // F8: e4m3 operands (kind::f8f6f4); a k-block is then 128 elements, the same
 // 128 bytes per row as 64 bf16 elements, so ring, swizzle and descriptors
-// are shared.
-template <int BN, int EPI, bool F8>
+// are shared.  F4: NVFP4 operands (kind::mxf4nvf4, packed e2m1, 256
+// elements per 128-byte row of a k-block) with e4m3 scale factors per 16
+// elements: each stage also carries the k-block's scale factors of the A and
+// B rows (2 KB per 128-row block), which the MMA thread copies into tensor
+// memory right before the stage's four MMAs (tcgen05 operations of one
+// thread run in order, so one scale-factor area serves every stage).
+template <int BN, int EPI, bool F8, bool F4 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcParams p) {
   using Cfg = TcCfg<BN>;
-  constexpr int kBKe = F8 ? 2 * kBK : kBK;   // elements per k-block
+  static_assert(!(F4 && (F8 || BN != 128)), "NVFP4 tiles are 128 wide");
+  constexpr int kBKe = F4 ? 4 * kBK : (F8 ? 2 * kBK : kBK);   // elements per k-block
+  constexpr int kSf = tc_sf_bytes(BN, F4);
+  constexpr uint32_t kTmemAlloc = F4 ? 512 : Cfg::kTmemCols;   // + scale-factor columns
+  constexpr uint32_t kSfaCol = 2 * BN, kSfbCol = 2 * BN + 16;
+  constexpr int kBX = F4 ? 2 * kBK : kBKe;   // TMA x coordinate (bytes for 8/4-bit) per k-block
   // timeline marks: 2 wait returned, 3 / 4 first / last ring stage full,
   // 5 first accumulator ready, 6 last tile's epilogue done
   DLM_TRACE_CTA(p.trace_kind);
@@ -149,9 +173,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = p.stages;
-  const int stage_bytes = tc_stage_bytes(BN, p.a_rows);
+  const int stage_bytes = tc_stage_bytes(BN, p.a_rows, kSf);
   const uint32_t a_bytes = (uint32_t)p.a_rows * 128u;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_bar_offset(BN, p.a_rows, stages));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_bar_offset(BN, p.a_rows, stages, kSf));
   uint64_t* empty = full + Cfg::kMaxStages;
   uint64_t* tfull = empty + Cfg::kMaxStages;
   uint64_t* tempty = tfull + 2;
@@ -179,7 +203,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, Cfg::kTmemCols);
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemAlloc);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,12 +220,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     pol_stream = l2_evict_first_policy();
     int n0, kb1, sp0;
-    if (get_unit<EPI>(p, 0, m_first, n0, kb_first, kb1, sp0)) {
+    if (!p.withhold_loads && get_unit<EPI>(p, 0, m_first, n0, kb_first, kb1, sp0)) {
       pre = min(stages, kb1 - kb_first);
       for (int s = 0; s < pre; ++s) {
         const int kb = kb_first + s;
-        mbar_expect_tx(&full[s], Cfg::kBBytes);
-        tma_load_2d_hint(smem + s * stage_bytes, &tmB, &full[s], kb * kBKe, n0 * BN, pol_stream);
+        mbar_expect_tx(&full[s], Cfg::kBBytes + (F4 ? 2048u * (BN / 128) : 0u));
+        tma_load_2d_hint(smem + s * stage_bytes, &tmB, &full[s], kb * kBX, n0 * BN, pol_stream);
+        if constexpr (F4) {
+          uint8_t* sfb_s = smem + s * stage_bytes + Cfg::kBBytes + a_bytes + 2048;
+          for (int rb = 0; rb < BN / 128; ++rb)
+            bulk_load_global(sfb_s + rb * 2048,
+                             p.sfb + ((size_t)(n0 * (BN / 128) + rb) * p.kg + 4 * kb) * 512, 2048,
+                             &full[s]);
+        }
       }
     }
   }
@@ -213,9 +244,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // always allocated, so these loads are issued even when the step turns
     // out to have nothing to do)
     for (int s = 0; s < pre; ++s) {
-      mbar_arrive_expect_tx(&full[s], a_bytes);
-      tma_load_2d(smem + s * stage_bytes + Cfg::kBBytes, &tmA, &full[s], (kb_first + s) * kBKe,
+      mbar_arrive_expect_tx(&full[s], a_bytes + (F4 ? 2048u : 0u));
+      tma_load_2d(smem + s * stage_bytes + Cfg::kBBytes, &tmA, &full[s], (kb_first + s) * kBX,
                   m_first * kBM);
+      if constexpr (F4)
+        bulk_load_global(smem + s * stage_bytes + Cfg::kBBytes + a_bytes,
+                         p.sfa + ((size_t)m_first * p.kg + 4 * (kb_first + s)) * 512, 2048,
+                         &full[s]);
     }
   }
   const bool skip = p.n_active != nullptr && *p.n_active == 0;
@@ -226,7 +261,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int s = 0; s < pre; ++s) mbar_wait_bounded(&full[s], 0u, nullptr);
   } else if (warp == 0) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    if (lane == 0 && !p.withhold_loads) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -246,8 +281,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint8_t* sb = smem + stage * stage_bytes;
             uint8_t* sa = sb + Cfg::kBBytes;
             mbar_arrive_expect_tx(&full[stage], (uint32_t)stage_bytes);
-            tma_load_2d(sa, &tmA, &full[stage], kb * kBKe, m * kBM);
-            tma_load_2d_hint(sb, &tmB, &full[stage], kb * kBKe, n * BN, pol_stream);
+            tma_load_2d(sa, &tmA, &full[stage], kb * kBX, m * kBM);
+            tma_load_2d_hint(sb, &tmB, &full[stage], kb * kBX, n * BN, pol_stream);
+            if constexpr (F4) {
+              uint8_t* sfa_s = sa + a_bytes;
+              bulk_load_global(sfa_s, p.sfa + ((size_t)m * p.kg + 4 * kb) * 512, 2048,
+                               &full[stage]);
+              for (int rb = 0; rb < BN / 128; ++rb)
+                bulk_load_global(sfa_s + 2048 + rb * 2048,
+                                 p.sfb + ((size_t)(n * (BN / 128) + rb) * p.kg + 4 * kb) * 512,
+                                 2048, &full[stage]);
+            }
           }
           ++issued;
           if (++stage == stages) {
@@ -275,7 +319,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN);
+      constexpr uint32_t idesc = F4 ? idesc_nvfp4_f32(kBM, BN)
+                                    : (F8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN));
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -287,7 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -295,10 +340,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + stage * stage_bytes);
           const uint32_t sa = sb + Cfg::kBBytes;
+          if constexpr (F4) {
+            // the k-block's scale factors into tensor memory: per MMA (64
+            // elements) 4 columns of A's and BN/32 columns of B's
+            const uint32_t sfa_s = sa + a_bytes, sfb_s = sfa_s + 2048;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              tmem_cp_32x128b_x4(tmem_base + kSfaCol + 4 * k, rows16_desc(sfa_s + k * 512));
+#pragma unroll
+              for (int rb = 0; rb < BN / 128; ++rb)
+                tmem_cp_32x128b_x4(tmem_base + kSfbCol + (BN / 32) * k + 4 * rb,
+                                   rows16_desc(sfb_s + rb * 2048 + k * 512));
+            }
+          }
           // four instructions of 32 bytes of K per 128-byte k-block
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            if constexpr (F8)
+            if constexpr (F4)
+              umma_nvfp4(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
+                         tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + (BN / 32) * k,
+                         (kb > kb0 || k > 0) ? 1u : 0u);
+            else if constexpr (F8)
               umma_e4m3(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
                         (kb > kb0 || k > 0) ? 1u : 0u);
             else
@@ -347,7 +409,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       lm_live = lm_row < p.M && (p.done == nullptr || p.done[lm_canvas] == 0);
       lm_step = lm_live ? p.epi.step[lm_canvas] : 0;
       lm_inv_t = lm_inv_temp(p.epi, lm_step);
-      if constexpr (F8) lm_a = lm_live ? p.epi.row_scale[lm_row] : 0.f;
+      if constexpr (F8 || F4) lm_a = lm_live ? p.epi.row_scale[lm_row] : 0.f;
     }
     for (int it = 0; get_unit<EPI>(p, it, m, n, kb0, kb1, split); ++it) {
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag)) break;
@@ -364,7 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float v[32];
             tmem_ld32(taddr + c, v);
             const int col0 = n * BN + c;
-            if constexpr (F8) {
+            if constexpr (F8 || F4) {
               if (p.epi.col_scale != nullptr)
                 scale_chunk(v, row < p.M ? p.epi.row_scale[row] : 0.f, p.epi.col_scale + col0);
             }
@@ -385,18 +447,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int c = cb; c < cb + kHalfN; c += 32) {
             float v[32];
             tmem_ld32(taddr + c, v);
-            if constexpr (F8) scale_chunk(v, lm_a, p.epi.col_scale + n * BN + c);
+            if constexpr (F8 || F4) scale_chunk(v, lm_a, p.epi.col_scale + n * BN + c);
             if (lm_live)
               rs_update<32>(rs, v, n * BN + c, lm_inv_t, p.epi, lm_canvas, lm_pos, lm_step);
           }
         } else if constexpr (EPI == EPI_QKV) {
-          // one 128-column head at a time: rotate pairs (j, j+64) of q and k,
-          // store q rows and the canvas K / V into the cache slots
+          // 128-column heads, each as two units of 32 rotary pairs (j, j+64),
+          // j in [32c, 32c+32): rotate q and k, store q rows and the canvas
+          // K / V into the cache slots.  The BN/64 units of a tile are split
+          // evenly between the two warpgroups.
           const ProjEpi& pe = p.proj;
           const int seq = row / pe.C, p_in = row - seq * pe.C;
           const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
+          constexpr int kUnits = BN / 128 * 2;
 #pragma unroll 1
-          for (int hc = cb / 128; hc < (cb + kHalfN) / 128; ++hc) {
+          for (int u = wg * kUnits / 2; u < (wg + 1) * kUnits / 2; ++u) {
+            const int hc = u >> 1, c = u & 1;
             const int head = (n * BN) / 128 + hc;
             bool store = live && head < pe.H + 2 * pe.Hkv;
             const int pos = store ? pe.lens[seq] + p_in : 0;
@@ -414,9 +480,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
             const bool rotate = pe.rope != nullptr && head < pe.H + pe.Hkv;
-            // rotary pairs (j, j + 64) in two chunks of 32 pairs
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
+            {
               uint32_t lo_raw[32], hi_raw[32];
               tmem_ld32_nowait(taddr + hc * 128 + c * 32, lo_raw);
               tmem_ld32_nowait(taddr + hc * 128 + 64 + c * 32, hi_raw);
@@ -512,7 +576,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    tmem_dealloc(tmem_base, kTmemAlloc);
   }
   if (threadIdx.x == 0 && *abort_flag) raise_error(p.err, DLM_ETIMEOUT);
 }
@@ -529,20 +593,20 @@ int tc_grid(int units, int m_tiles, int n_tiles, int epi, int num_sms) {
   return units < num_sms ? units : num_sms;
 }
 
-template <int BN, int EPI, bool F8 = false>
+template <int BN, int EPI, bool F8 = false, bool F4 = false>
 cudaError_t launch_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const TcParams& p,
                       int num_sms, cudaStream_t st) {
   using Cfg = TcCfg<BN>;
   static bool attr_set = false;   // per process; one device is used per process
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, F8>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, F8, F4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int grid = tc_grid(p.units, p.m_tiles, p.n_tiles, EPI, num_sms);
-  return launch_pdl(gemm_tc_kernel<BN, EPI, F8>, dim3(grid), dim3(kGemmThreads), Cfg::kSmem, st,
-                    tmA, tmB, p);
+  return launch_pdl(gemm_tc_kernel<BN, EPI, F8, F4>, dim3(grid), dim3(kGemmThreads), Cfg::kSmem,
+                    st, tmA, tmB, p);
 }
 
 }  // namespace
@@ -556,11 +620,12 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.m_tiles = (plan.M + kBM - 1) / kBM;
   p.n_tiles = (plan.N + plan.BN - 1) / plan.BN;
   p.splits = plan.splits;
-  const int kbe = plan.f8 ? 2 * kBK : kBK;   // elements per k-block
+  const int kbe = plan.f4 ? 4 * kBK : (plan.f8 ? 2 * kBK : kBK);   // elements per k-block
   p.kblocks = (plan.K + kbe - 1) / kbe;
   p.units = p.m_tiles * p.n_tiles * p.splits;
   p.a_rows = gemm_tc_a_rows(plan.M);
-  p.stages = plan.BN == 128 ? tc_stages<128>(p.a_rows) : tc_stages<256>(p.a_rows);
+  const int sf = tc_sf_bytes(plan.BN, plan.f4 != 0);
+  p.stages = plan.BN == 128 ? tc_stages<128>(p.a_rows, sf) : tc_stages<256>(p.a_rows, sf);
   p.out = io.out;
   p.part = io.part;
   p.epi = io.epi;
@@ -570,6 +635,19 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
   p.n_active = io.n_active;
   p.err = io.err;
   p.trace_kind = io.trace_kind;
+  p.withhold_loads = io.withhold_loads;
+  p.wait_ns = io.withhold_loads ? 20000000ull : kWaitLimitNs;   // 20 ms in the test
+  p.sfa = io.sfa;
+  p.sfb = io.sfb;
+  p.kg = plan.K / 64;
+  if (plan.f4) {
+    // NVFP4 operands: the LM head and its full-logit inspection, 128-wide tiles
+    if (plan.BN != 128 || plan.K % 256 != 0 || io.sfa == nullptr || io.sfb == nullptr)
+      return cudaErrorInvalidValue;
+    if (plan.epi == EPI_LM) return launch_tc<128, EPI_LM, false, true>(tmA, tmB, p, num_sms, st);
+    if (plan.epi == EPI_F32) return launch_tc<128, EPI_F32, false, true>(tmA, tmB, p, num_sms, st);
+    return cudaErrorInvalidValue;
+  }
   if (plan.f8) {
     // e4m3 operands: the LM head and its full-logit inspection only
     if (plan.epi == EPI_LM)
@@ -581,8 +659,12 @@ cudaError_t gemm_tc(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmPl
     return cudaErrorInvalidValue;
   }
   if (plan.BN == 128) {
-    return plan.epi == EPI_LM ? launch_tc<128, EPI_LM>(tmA, tmB, p, num_sms, st)
-                              : launch_tc<128, EPI_F32>(tmA, tmB, p, num_sms, st);
+    switch (plan.epi) {
+      case EPI_LM: return launch_tc<128, EPI_LM>(tmA, tmB, p, num_sms, st);
+      case EPI_QKV: return launch_tc<128, EPI_QKV>(tmA, tmB, p, num_sms, st);
+      case EPI_RESID: return launch_tc<128, EPI_RESID>(tmA, tmB, p, num_sms, st);
+      default: return launch_tc<128, EPI_F32>(tmA, tmB, p, num_sms, st);
+    }
   }
   switch (plan.epi) {
     case EPI_LM: return launch_tc<256, EPI_LM>(tmA, tmB, p, num_sms, st);

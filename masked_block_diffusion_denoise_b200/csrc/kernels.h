@@ -20,6 +20,7 @@ struct GemmPlan {
   int splits;   // K splits (EPI_F32 only)
   int epi;      // EPI_F32 / EPI_LM
   int f8 = 0;       // e4m3 operands (tcgen05 only; EPI_LM and EPI_F32)
+  int f4 = 0;       // NVFP4 operands with block scales (tcgen05, BN 128; EPI_LM, EPI_F32)
 };
 
 struct ModelDims;
@@ -73,6 +74,9 @@ struct GemmIO {
   const int* n_active = nullptr;
   int* err = nullptr;
   int trace_kind = -1;         // TraceKind of this launch, -1: not traced
+  int withhold_loads = 0;      // failure-detection test: see dlm_test_withhold_loads
+  const uint8_t* sfa = nullptr;   // NVFP4: block scales of A and B ([128-row block][K/64][512])
+  const uint8_t* sfb = nullptr;
 };
 
 // ---- gemm_tc.cu: bf16 tcgen05 GEMM ---------------------------------------
@@ -137,11 +141,20 @@ cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st);
 cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, float* scale, int C,
                                const uint8_t* done, const int* n_active, cudaStream_t st);
 
+// NVFP4 rows (bf16 input, cols % 64 == 0): packed e2m1 elements q [rows][cols/2]
+// (element 2i in the low nibble), e4m3 block scales of 16 in the block-scaled
+// MMA's layout sf [ceil(rows/128)][cols/64][512] (see the kernel), a float32
+// scale per row; rows of finished canvases are skipped
+cudaError_t quantize_rows_nvfp4(const void* x, int rows, int cols, uint8_t* q, uint8_t* sf,
+                                float* row_scale, int C, const uint8_t* done, const int* n_active,
+                                cudaStream_t st);
+
 // ---- attention.cu ------------------------------------------------------------
 struct AttnPlan {
   int B, C, G, R, rtiles;   // G = H / Hkv, R = G * C query rows per (seq, kv head)
   int chunk, nsplit;        // keys per split (multiple of 128), splits per (seq, kv head)
   int cluster = 1;          // nsplit (<= 16) when the splits combine inside a cluster
+  int rows = 128;           // query rows per CTA
 };
 
 // clusters of n (2..16) attention CTAs that fit on the device at once (0: none)

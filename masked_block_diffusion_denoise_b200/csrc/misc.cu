@@ -1,6 +1,7 @@
 // Element-wise kernels around the GEMMs: RoPE table, embedding gather, the
 // projection epilogues (split-K sum, rotary embedding, KV-cache write,
 // residual), KV copy-in and canvas initialisation.
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "kernels.h"
@@ -220,6 +221,87 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(
   if (threadIdx.x == 0) scale[r] = s;
 }
 
+// NVFP4 rows (bf16 input, cols % 64 == 0): a float32 scale per row,
+// s_r = amax(row) / (448 * 6) (1 for a zero row); per 16-element block an e4m3
+// scale e4m3(amax(block) / (6 s_r)); elements e2m1(x / (sb * s_r)), 0 in a
+// block whose scale is 0; every division and product in float32, round to
+// nearest even, saturating.  Elements are packed two per byte, element 2i
+// in the low nibble.  Block scales go to the layout the block-scaled tensor
+// core reads after a 32-row x 16-byte copy replicated to all four lane
+// quadrants: per 128-row block and 64-element k group one 512-byte chunk,
+// byte (m % 32) * 16 + (m / 32) * 4 + s for row m of the row block and the
+// s-th 16-element block of the k group.  One CTA per row, one thread per
+// block (strided).  Rows of finished canvases (row / C, when done is given)
+// are skipped.
+__global__ void __launch_bounds__(256) quantize_rows_nvfp4_kernel(
+    const __nv_bfloat16* __restrict__ x, int rows, int cols, uint8_t* __restrict__ q,
+    uint8_t* __restrict__ sf, float* __restrict__ row_scale, int C,
+    const uint8_t* __restrict__ done, const int* n_active) {
+  DLM_TRACE_CTA(TRACE_QUANTIZE);
+  pdl_wait_then_release();
+  if (threadIdx.x == 0) DLM_TRACE_MARK(2);
+  if (n_active != nullptr && *n_active == 0) return;
+  const int r = blockIdx.x;
+  if (r >= rows || (done != nullptr && done[r / C])) return;
+  const __nv_bfloat16* xr = x + (size_t)r * cols;
+  float amax = 0.f;
+  for (int i = threadIdx.x * 8; i < cols; i += blockDim.x * 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = wmax[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, wmax[w]);
+  const float sr = amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f;   // 448 * 6
+  const float six_sr = __fmul_rn(6.f, sr);
+  const int kg = cols / 64;
+  const int rb = r >> 7, m = r & 127;
+  uint8_t* qr = q + (size_t)r * (cols / 2);
+  for (int j = threadIdx.x; j < cols / 16; j += blockDim.x) {
+    float f[16];
+    const uint4* src = reinterpret_cast<const uint4*>(xr + j * 16);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 v = src[h];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[u]));
+        f[8 * h + 2 * u] = t.x;
+        f[8 * h + 2 * u + 1] = t.y;
+      }
+    }
+    float ab = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ab = fmaxf(ab, fabsf(f[e]));
+    const __nv_fp8_storage_t sbq = __nv_cvt_float_to_fp8(__fdiv_rn(ab, six_sr), __NV_SATFINITE,
+                                                         __NV_E4M3);
+    const float sbv = __half2float(__half(__nv_cvt_fp8_to_halfraw(sbq, __NV_E4M3)));
+    const float scale = __fmul_rn(sbv, sr);
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float ratio = scale > 0.f ? __fdiv_rn(f[e], scale) : 0.f;
+      const uint32_t code =
+          (uint32_t)__nv_cvt_float_to_fp4(ratio, __NV_E2M1, cudaRoundNearest) & 0xFu;
+      packed[e >> 3] |= code << (4 * (e & 7));
+    }
+    *reinterpret_cast<uint2*>(qr + j * 8) = make_uint2(packed[0], packed[1]);
+    const int g = j >> 2, sblk = j & 3;
+    sf[((size_t)rb * kg + g) * 512 + (m & 31) * 16 + (m >> 5) * 4 + sblk] = sbq;
+  }
+  if (threadIdx.x == 0) row_scale[r] = sr;
+}
+
 __global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint32_t s0,
                                    uint32_t s1, int32_t* tokens, uint8_t* committed,
                                    int32_t* step, uint8_t* done, int32_t* eos_pos,
@@ -326,6 +408,14 @@ cudaError_t quantize_rows_e4m3(const void* x, int rows, int cols, uint8_t* q, fl
   if (cols % 8 != 0) return cudaErrorInvalidValue;
   return launch_pdl(quantize_rows_kernel, dim3(rows), dim3(256), 0, st,
                     (const __nv_bfloat16*)x, rows, cols, q, scale, C, done, n_active);
+}
+
+cudaError_t quantize_rows_nvfp4(const void* x, int rows, int cols, uint8_t* q, uint8_t* sf,
+                                float* row_scale, int C, const uint8_t* done, const int* n_active,
+                                cudaStream_t st) {
+  if (cols % 64 != 0) return cudaErrorInvalidValue;
+  return launch_pdl(quantize_rows_nvfp4_kernel, dim3(rows), dim3(256), 0, st,
+                    (const __nv_bfloat16*)x, rows, cols, q, sf, row_scale, C, done, n_active);
 }
 
 cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st) {

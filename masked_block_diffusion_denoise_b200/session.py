@@ -109,7 +109,8 @@ class Session:
                               shape.vocab, DLM_BF16 if shape.dtype == "bf16" else DLM_F32,
                               float(shape.rope_theta), shape.mask_id, shape.eos_id,
                               max_batch, max_prefix, max_canvas,
-                              1 if getattr(shape, "lm_fp8", False) else 0)
+                              2 if getattr(shape, "lm_nvfp4", False)
+                              else (1 if getattr(shape, "lm_fp8", False) else 0))
         wts = dlm_weights(*(self.w[k].data_ptr() for k in
                             ("emb", "w_q", "w_k", "w_v", "w_o", "w_lm")))
         torch.cuda.synchronize(self.device)

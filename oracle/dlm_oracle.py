@@ -294,6 +294,23 @@ def dequantize_rows_nvfp4(q, sb, sr) -> np.ndarray:
     return q * s
 
 
+def quantize_rows_nvfp4_blocked(x, rows_per_block: int = 4096):
+    """quantize_rows_nvfp4 over row blocks (rows are independent), keeping
+    the elements as float32 (every e2m1 value is exact there) to bound
+    memory for large matrices."""
+    x = np.asarray(x)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), dtype=np.float32)
+    sb = np.empty((rows, cols // NVFP4_BLOCK), dtype=F64)
+    sr = np.empty(rows, dtype=np.float32)
+    for r0 in range(0, rows, rows_per_block):
+        qb_, sbb_, srb_ = quantize_rows_nvfp4(x[r0:r0 + rows_per_block])
+        q[r0:r0 + rows_per_block] = qb_
+        sb[r0:r0 + rows_per_block] = sbb_
+        sr[r0:r0 + rows_per_block] = srb_
+    return q, sb, sr
+
+
 def nvfp4_dot(qa, sba, sra, qb, sbb, srb) -> np.ndarray:
     """Rows of A times rows of B, both NVFP4 along the reduction axis, the way
     a block-scaled product runs: per block the exact sum of element products
@@ -310,6 +327,22 @@ def nvfp4_dot(qa, sba, sra, qb, sbb, srb) -> np.ndarray:
     return (blk * w).sum(axis=2) * (np.asarray(sra, F64)[:, None] * np.asarray(srb, F64)[None, :])
 
 
+def nvfp4_head_logits(qa, sba, sra, qb, sbb, srb, rows_per_block: int = 4096) -> np.ndarray:
+    """The NVFP4 LM head: per pair of rows the block-scaled sum of nvfp4_dot
+    without the row scales, times the two row scales' product rounded to
+    float32 (READING, as for the e4m3 head: one float32 factor per logit).
+    B is processed in row blocks to bound memory."""
+    ra = np.asarray(qa).shape[0]
+    out = np.empty((ra, np.asarray(qb).shape[0]), dtype=F64)
+    ones_a = np.ones(ra)
+    for r0 in range(0, out.shape[1], rows_per_block):
+        sl = slice(r0, r0 + rows_per_block)
+        blk = nvfp4_dot(qa, sba, ones_a, qb[sl], sbb[sl], np.ones(len(srb[sl])))
+        f = (np.asarray(sra, np.float32)[:, None] * np.asarray(srb[sl], np.float32)[None, :])
+        out[:, sl] = blk * f.astype(np.float32).astype(F64)
+    return out
+
+
 @dataclass
 class ModelDims:
     d_model: int
@@ -322,12 +355,13 @@ class ModelDims:
     mask_id: int = 100
     eos_id: int = 11
     lm_fp8: bool = False      # LM head with e4m3 weights and activations
+    lm_nvfp4: bool = False    # LM head with NVFP4 weights and activations
 
     @classmethod
     def of(cls, shape) -> "ModelDims":
         return cls(shape.d_model, shape.n_heads, shape.n_kv_heads, shape.head_dim,
                    shape.vocab, shape.dtype, shape.rope_theta, shape.mask_id, shape.eos_id,
-                   bool(getattr(shape, "lm_fp8", False)))
+                   bool(getattr(shape, "lm_fp8", False)), bool(getattr(shape, "lm_nvfp4", False)))
 
 
 class OracleModel:
@@ -353,6 +387,8 @@ class OracleModel:
         self.w_lm = conv(weights["w_lm"])
         if dims.lm_fp8:
             self.lm_q, self.lm_scale = quantize_rows_e4m3(self.w_lm)
+        if dims.lm_nvfp4:
+            self.lm_q4, self.lm_sb, self.lm_sr = quantize_rows_nvfp4_blocked(self.w_lm)
         self.store = round_to_bf16 if dims.dtype == "bf16" else round_to_f32
         self.k_cache: Dict[int, np.ndarray] = {}
         self.v_cache: Dict[int, np.ndarray] = {}
@@ -421,6 +457,11 @@ class OracleModel:
         return self.store(x + o @ self.w_o.T)
 
     def logits(self, y: np.ndarray) -> np.ndarray:
+        if self.dims.lm_nvfp4:
+            # the NVFP4 head: both operands quantised per row (e2m1 elements,
+            # e4m3 block scales of 16, a float32 row scale)
+            qy, sby, sry = quantize_rows_nvfp4(y)
+            return nvfp4_head_logits(qy, sby, sry, self.lm_q4, self.lm_sb, self.lm_sr)
         if self.dims.lm_fp8:
             # the e4m3 head: both operands quantised per row, the products
             # summed exactly, then one float32 factor a_r * s_v per logit

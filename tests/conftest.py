@@ -22,3 +22,15 @@ def golden_lines(name):
             line = line.split("#", 1)[0].strip()
             if line:
                 yield line.split()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Near ties counted by the GPU parity tests: positions whose candidate
+    differs from the oracle's float64 argmax only within the near-tie gap."""
+    mod = sys.modules.get("gpu_util")
+    ties = getattr(mod, "NEAR_TIES", None) if mod is not None else None
+    if not ties:
+        return
+    terminalreporter.section("near ties (GPU parity)")
+    for name, (n, m) in sorted(ties.items()):
+        terminalreporter.write_line("near-ties %s: %d of %d positions compared" % (name, n, m))

@@ -17,8 +17,8 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
-from gpu_util import (abs_terms, assert_storage_close, lib_params, make_pair, near_tie_ok,
-                      oracle_params, state_from, to64)
+from gpu_util import (abs_terms, assert_storage_close, check_one_step, lib_params, make_pair,
+                      oracle_params, record_near_ties, to64)
 from oracle import dlm_oracle as O
 import workloads as W
 
@@ -28,118 +28,7 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU-only ho
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 from masked_block_diffusion_denoise_b200 import (DLM_BUF_CAND, DLM_BUF_CONF, DLM_BUF_ENTROPY,
-                                                 DLM_BUF_K_CACHE, DLM_BUF_O, DLM_BUF_Q,
-                                                 DLM_BUF_V_CACHE, DLM_BUF_X, DLM_BUF_Y)
-
-
-# ---------------------------------------------------------------------------
-# stage-by-stage check of one step
-# ---------------------------------------------------------------------------
-
-def check_one_step(sess, om, wl, cv, p_lib, p_or, *, rows_sample=None, heads_sample=None,
-                   full_logits=True, report=None):
-    sh = wl.shape
-    B, C = cv.tokens.shape
-    M = B * C
-    dt = torch.bfloat16 if sh.dtype == "bf16" else torch.float32
-    pre = cv.numpy()
-    sess.step(cv, p_lib)
-    sess.check()
-    post = cv.numpy()
-    active = [b for b in range(B) if not pre["done"][b]]
-    x = to64(sess.buffer(DLM_BUF_X, (M, sh.d_model), dt))
-    q = to64(sess.buffer(DLM_BUF_Q, (M, sh.n_heads, sh.head_dim), dt))
-    o = to64(sess.buffer(DLM_BUF_O, (M, sh.n_heads * sh.head_dim), dt))
-    y = to64(sess.buffer(DLM_BUF_Y, (M, sh.d_model), dt))
-    Lcap = sess.max_prefix + sess.max_canvas
-    kc = sess.buffer(DLM_BUF_K_CACHE, (sess.max_batch, sh.n_kv_heads, Lcap, sh.head_dim), dt)
-    vc = sess.buffer(DLM_BUF_V_CACHE, (sess.max_batch, sh.n_kv_heads, Lcap, sh.head_dim), dt)
-    cand = sess.buffer(DLM_BUF_CAND, (M,), torch.int32).cpu().numpy()
-    conf = sess.buffer(DLM_BUF_CONF, (M,), torch.float32).cpu().numpy()
-    ent = sess.buffer(DLM_BUF_ENTROPY, (M,), torch.float32).cpu().numpy()
-    logits = sess.logits(B, C).cpu().numpy() if full_logits else None
-    near_ties = 0
-    for b in active:
-        r0 = b * C
-        rows = np.arange(C) if rows_sample is None else np.asarray(rows_sample)
-        L = om.kv_len(b)
-        # a1 embedding: exact
-        assert np.array_equal(x[r0 + rows], om.embed(pre["tokens"][b][rows])), "embed"
-        # a2 projections + RoPE from the GPU's x
-        qo, ko, vo = om.project_qkv(x[r0 + rows], L + rows)
-        xr = x[r0 + rows]
-        half = sh.head_dim // 2
-        rot = lambda t: np.concatenate([t[..., :half] + t[..., half:]] * 2, axis=-1)
-        tq = rot(abs_terms(xr, om.w_q).reshape(qo.shape))
-        tk = rot(abs_terms(xr, om.w_k).reshape(ko.shape))
-        tv = abs_terms(xr, om.w_v).reshape(vo.shape)
-        assert_storage_close(q[r0 + rows], qo, sh.dtype, what="q", terms=tq)
-        kg = to64(kc[b, :, L:L + C]).transpose(1, 0, 2)
-        vg = to64(vc[b, :, L:L + C]).transpose(1, 0, 2)
-        assert_storage_close(kg[rows], ko, sh.dtype, what="canvas k", terms=tk)
-        assert_storage_close(vg[rows], vo, sh.dtype, what="canvas v", terms=tv)
-        # a3 attention from the GPU's q, k, v
-        qb = q[r0:r0 + C]
-        oo = om.attend(b, qb, kg, vg)
-        err = np.abs(o[r0:r0 + C] - oo)
-        if heads_sample is not None:
-            cols = np.concatenate([np.arange(h * sh.head_dim, (h + 1) * sh.head_dim)
-                                   for h in heads_sample])
-            err = err[:, cols]
-        assert err.max() < 2e-2, "attention max abs err %g" % err.max()
-        if report is not None:
-            report.setdefault("attn_max_err", []).append(float(err.max()))
-        # a4 output projection + residual from the GPU's x and o
-        yo = om.out_proj(x[r0 + rows], o[r0 + rows])
-        assert_storage_close(y[r0 + rows], yo, sh.dtype, what="y",
-                             terms=np.abs(xr) + abs_terms(o[r0 + rows], om.w_o))
-        # a5/a6 scores
-        if p_or.entropy_bound >= 0 or p_or.temperature > 0:
-            continue   # sampling modes are checked in their own test
-        mask = sh.mask_id if p_or.corruption == "mask" else -1
-        if logits is not None:
-            lg = logits[r0:r0 + C]
-            lo = om.logits(y[r0:r0 + C])
-            assert np.abs(lg - lo).max() < 2e-3 * max(1.0, np.abs(lo).max()), "logits"
-            c32, f32, h32, _ = O.scores(lg.astype(np.float32), mask)
-            assert np.array_equal(cand[r0:r0 + C], c32), "cand from identical logits"
-            assert np.abs(conf[r0:r0 + C] - f32).max() < 1e-3, "confidence"
-            assert np.abs(ent[r0:r0 + C] - h32).max() < 1e-3, "entropy"
-            c64, _, _, z = O.scores(lo, mask)
-            for i in range(C):
-                if cand[r0 + i] != c64[i]:
-                    assert near_tie_ok(z[i], int(cand[r0 + i]), int(c64[i]), 1e-3), \
-                        "argmax flip outside a near tie"
-                    near_ties += 1
-        else:
-            for i in rows:
-                lo = om.logits(y[r0 + i:r0 + i + 1])
-                c64, f64, h64, z = O.scores(lo, mask)
-                if cand[r0 + i] != c64[0]:
-                    assert near_tie_ok(z[0], int(cand[r0 + i]), int(c64[0]), 1e-3)
-                    near_ties += 1
-                else:
-                    assert abs(conf[r0 + i] - f64[0]) < 1e-3
-                assert abs(ent[r0 + i] - h64[0]) < 1e-3
-    # a7 selection on the GPU's own cand / conf / H: bit-exact
-    st = state_from(pre)
-    stats = [O.CanvasStats() for _ in range(B)]
-    for b in range(B):
-        O.select_canvas(st, b, cand[b * C:(b + 1) * C], conf[b * C:(b + 1) * C],
-                        ent[b * C:(b + 1) * C], p_or, vocab=sh.vocab, mask_id=sh.mask_id,
-                        eos_id=sh.eos_id, stats=stats[b])
-    assert np.array_equal(st.tokens, post["tokens"]), "tokens after commit"
-    assert np.array_equal(st.committed, post["committed"]), "commit mask"
-    assert np.array_equal(st.step, post["step"]) and np.array_equal(st.done, post["done"])
-    assert np.array_equal(st.eos_pos, post["eos_pos"])
-    dstats = post["stats"] - pre["stats"]
-    for b in range(B):
-        assert list(dstats[b]) == [stats[b].steps_used, stats[b].committed_by_sampler,
-                                   stats[b].forced_at_budget, stats[b].eos_autofill,
-                                   stats[b].frozen, stats[b].edited]
-    if report is not None:
-        report["near_ties"] = report.get("near_ties", 0) + near_ties
-    return pre, post
+                                                 DLM_BUF_K_CACHE, DLM_BUF_V_CACHE, DLM_BUF_Y)
 
 
 SMALL = {
@@ -163,6 +52,13 @@ SMALL = {
                                          canvas=64, steps=4, quota=0, prefix_len=(64, 300),
                                          prefix_cap=320, vocab=3000, lm_fp8=True,
                                          corruption="uniform"),
+    # NVFP4 LM head, one M tile, ragged vocabulary
+    "small_nvfp4": W.small_workload("small_nvfp4", steps=6, quota=0, lm_nvfp4=True, seed=4),
+    # NVFP4 LM head over two M tiles, d 512 (two k-blocks), uniform corruption
+    "small_nvfp4_mtiles": W.small_workload("small_nvfp4_mtiles", d_model=512, n_heads=8,
+                                           n_kv_heads=2, batch=4, canvas=64, steps=4, quota=0,
+                                           prefix_len=(64, 300), prefix_cap=320, vocab=3000,
+                                           lm_nvfp4=True, corruption="uniform"),
 }
 
 
@@ -183,7 +79,8 @@ def test_small_block_stagewise(name):
             if post["done"].all():
                 break
         assert cv.numpy()["done"].all()
-        print(name, report)
+        record_near_ties("small_block_stagewise[%s]" % name, report.get("near_ties", 0),
+                         report.get("compared", 0))
     finally:
         sess.close()
 
@@ -202,6 +99,40 @@ def test_attention_split_paths(cluster, monkeypatch):
         p_lib, p_or = lib_params(wl), oracle_params(wl)
         sess.init(cv, p_lib)
         check_one_step(sess, om, wl, cv, p_lib, p_or)
+    finally:
+        sess.close()
+
+
+@pytest.mark.parametrize("heads,canvas,tiles", [
+    ((8, 2), 64, None),    # G 4, 256 rows: one CTA per KV head, planner's splits
+    ((8, 2), 64, 2),       # the same with 256-key splits: partials + combine kernel
+    ((8, 2), 96, 3),       # 384 rows: the second CTA holds one live row tile
+    ((4, 4), 256, None),   # G 1 (encoder-decoder grouping), 256 canvas positions
+    ((6, 2), 96, None),    # G 3 does not divide 128: query tiles by plain loads
+])
+def test_attention_two_row_tiles(heads, canvas, tiles, monkeypatch):
+    """The 256-row attention CTA (two 128-row query tiles of one KV head
+    share every K/V tile), forced with DLM_ATTN_ROWS=256, on ragged prefixes,
+    within 2e-2 of the float64 attention over the GPU's own q, k, v."""
+    from masked_block_diffusion_denoise_b200 import dlm_attention_plan
+    monkeypatch.setenv("DLM_ATTN_ROWS", "256")
+    if tiles is not None:
+        monkeypatch.setenv("DLM_ATTN_TILES", str(tiles))
+    H, Hkv = heads
+    wl = W.small_workload("two_tiles", n_heads=H, n_kv_heads=Hkv, batch=3, canvas=canvas,
+                          steps=2, quota=0, prefix_len=(20, 1500), prefix_cap=1600, seed=8)
+    sess, om, _ = make_pair(wl)
+    try:
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib, p_or = lib_params(wl), oracle_params(wl)
+        sess.init(cv, p_lib)
+        plan = dlm_attention_plan(sess.ctx, wl.batch, wl.canvas)
+        assert plan["rows_per_cta"] == 256, plan
+        if tiles is not None:
+            assert plan["nsplit"] > 1 and plan["chunk"] == 128 * tiles, plan
+        report = {}
+        check_one_step(sess, om, wl, cv, p_lib, p_or, report=report)
+        assert max(report["attn_max_err"]) < 2e-2
     finally:
         sess.close()
 
@@ -464,7 +395,65 @@ def test_fp8_quantisation_bit_exact():
         sess.close()
 
 
-@pytest.mark.parametrize("name", ["8b_b1", "encdec", "8b_b1_fp8"])
+E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _decode_e2m1_pairs(packed: np.ndarray, cols: int) -> np.ndarray:
+    """[rows][cols/2] bytes, element 2i in the low nibble -> values"""
+    b = packed.astype(np.int64)
+    nib = np.stack([b & 0xF, b >> 4], axis=-1).reshape(b.shape[0], cols)
+    return np.where(nib & 8, -1.0, 1.0) * E2M1[nib & 7]
+
+
+def _block_scales_from_mma_layout(sf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """e4m3 block scales stored per 128-row block and 64-element k group in
+    512-byte chunks, byte (m % 32) * 16 + (m / 32) * 4 + s -> [rows][cols/16]"""
+    kg = cols // 64
+    r = np.arange(rows)[:, None]
+    j = np.arange(cols // 16)[None, :]
+    m = r % 128
+    idx = ((r // 128) * kg + j // 4) * 512 + (m % 32) * 16 + (m // 32) * 4 + j % 4
+    return torch.from_numpy(sf[idx].astype(np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def test_nvfp4_quantisation_bit_exact():
+    """The NVFP4 copies of the LM head's weights and of a step's input rows --
+    e2m1 elements, e4m3 block scales in the block-scaled MMA's layout and
+    float32 row scales -- equal the oracle's quantisation exactly."""
+    wl = SMALL["small_nvfp4_mtiles"]
+    sess, om, _ = make_pair(wl)
+    try:
+        from masked_block_diffusion_denoise_b200 import (DLM_BUF_LM_Q, DLM_BUF_LM_SCALE,
+                                                         DLM_BUF_LM_SF, DLM_BUF_Y_Q,
+                                                         DLM_BUF_Y_SCALE, DLM_BUF_Y_SF)
+        sh = wl.shape
+        V, d = sh.vocab, sh.d_model
+        lm_q = sess.buffer(DLM_BUF_LM_Q, (V, d // 2), torch.uint8).cpu().numpy()
+        assert np.array_equal(_decode_e2m1_pairs(lm_q, d), om.lm_q4)
+        kgb = -(-V // 128) * (d // 64) * 512
+        lm_sf = sess.buffer(DLM_BUF_LM_SF, (kgb,), torch.uint8).cpu().numpy()
+        assert np.array_equal(_block_scales_from_mma_layout(lm_sf, V, d), om.lm_sb)
+        sr = sess.buffer(DLM_BUF_LM_SCALE, (V,), torch.float32).cpu().numpy()
+        assert np.array_equal(sr, om.lm_sr)
+        cv = sess.new_canvas(wl.batch, wl.canvas)
+        p_lib = lib_params(wl)
+        sess.init(cv, p_lib)
+        sess.step(cv, p_lib)
+        sess.check()
+        M = wl.batch * wl.canvas
+        y = to64(sess.buffer(DLM_BUF_Y, (M, d), torch.bfloat16))
+        ref_q, ref_sb, ref_sr = O.quantize_rows_nvfp4(y)
+        yq = sess.buffer(DLM_BUF_Y_Q, (M, d // 2), torch.uint8).cpu().numpy()
+        assert np.array_equal(_decode_e2m1_pairs(yq, d), ref_q)
+        ysf = sess.buffer(DLM_BUF_Y_SF, (-(-M // 128) * (d // 64) * 512,), torch.uint8)
+        assert np.array_equal(_block_scales_from_mma_layout(ysf.cpu().numpy(), M, d), ref_sb)
+        ys = sess.buffer(DLM_BUF_Y_SCALE, (M,), torch.float32).cpu().numpy()
+        assert np.array_equal(ys, ref_sr)
+    finally:
+        sess.close()
+
+
+@pytest.mark.parametrize("name", ["8b_b1", "encdec", "8b_b1_fp8", "8b_b1_nvfp4"])
 def test_full_size_step_sampled(name):
     wl = W.WORKLOADS[name]
     sess, om, _ = make_pair(wl)
@@ -473,6 +462,10 @@ def test_full_size_step_sampled(name):
         p_lib, p_or = lib_params(wl), oracle_params(wl)
         sess.init(cv, p_lib)
         rows = np.array([0, 5, wl.canvas - 1])
-        check_one_step(sess, om, wl, cv, p_lib, p_or, rows_sample=rows, full_logits=False)
+        report = {}
+        check_one_step(sess, om, wl, cv, p_lib, p_or, rows_sample=rows, full_logits=False,
+                       report=report)
+        record_near_ties("full_size_step_sampled[%s]" % name, report.get("near_ties", 0),
+                         report.get("compared", 0))
     finally:
         sess.close()

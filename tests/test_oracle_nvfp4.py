@@ -113,3 +113,32 @@ def test_block_scaled_dot_equals_the_dequantised_product():
 def test_columns_must_fill_blocks():
     with pytest.raises(ValueError):
         O.quantize_rows_nvfp4(np.ones((2, 24), np.float32))
+
+
+def test_blocked_quantisation_equals_whole_matrix():
+    """Rows are independent: quantising in row blocks gives the same codes,
+    block scales and row scales as one call over the whole matrix."""
+    r = np.random.default_rng(21)
+    x = r.standard_normal((37, 96)).astype(np.float32) * 0.02
+    q, sb, sr = O.quantize_rows_nvfp4(x)
+    qb, sbb, srb = O.quantize_rows_nvfp4_blocked(x, rows_per_block=8)
+    assert np.array_equal(qb, q) and np.array_equal(sbb, sb) and np.array_equal(srb, sr)
+
+
+def test_head_logits_equal_dequantised_product_with_f32_row_factor():
+    """The NVFP4 head's logits: the block-scaled sums times the two row
+    scales' product rounded to float32 -- equal to the product of the rows
+    dequantised without their row scales, times that factor."""
+    r = np.random.default_rng(22)
+    a = r.standard_normal((5, 64)).astype(np.float32)
+    b = r.standard_normal((33, 64)).astype(np.float32) * 0.02
+    qa, sba, sra = O.quantize_rows_nvfp4(a)
+    qb, sbb, srb = O.quantize_rows_nvfp4(b)
+    got = O.nvfp4_head_logits(qa, sba, sra, qb, sbb, srb, rows_per_block=7)
+    da = O.dequantize_rows_nvfp4(qa, sba, np.ones(5))
+    db = O.dequantize_rows_nvfp4(qb, sbb, np.ones(33))
+    f = (sra[:, None] * srb[None, :]).astype(np.float32).astype(np.float64)
+    want = (da @ db.T) * f
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+    # and it stays within float32 rounding of the f64 row-scale product
+    assert np.allclose(got, O.nvfp4_dot(qa, sba, sra, qb, sbb, srb), rtol=2 ** -23)

@@ -61,6 +61,7 @@ class ModelShape:
     mask_id: int = 100
     eos_id: int = 11
     lm_fp8: bool = False           # LM head in e4m3 (weights and its input rows)
+    lm_nvfp4: bool = False         # LM head in NVFP4 (e2m1, e4m3 block scales of 16)
 
     @property
     def q_dim(self) -> int:
@@ -130,21 +131,27 @@ WORKLOADS: Dict[str, Workload] = {
                           t_max=0.8, t_min=0.4),
 }
 # the same workloads with the e4m3 LM head (online FP8 weight quantisation)
+# and with the NVFP4 LM head (4-bit weights, the Blackwell low-bit path)
 for _name in ("8b_b1", "batched", "encdec"):
     _w = WORKLOADS[_name]
     WORKLOADS[_name + "_fp8"] = _w.replace(name=_name + "_fp8",
                                            shape=dataclasses.replace(_w.shape, lm_fp8=True))
+for _name in ("8b_b1", "longctx"):
+    _w = WORKLOADS[_name]
+    WORKLOADS[_name + "_nvfp4"] = _w.replace(name=_name + "_nvfp4",
+                                             shape=dataclasses.replace(_w.shape, lm_nvfp4=True))
 
 
 def small_workload(name: str = "small", *, d_model=256, n_heads=4, n_kv_heads=2,
                    head_dim=128, vocab=4096 + 96, batch=2, canvas=32, steps=8,
                    prefix_len=(200, 333), prefix_cap=384, dtype="bf16", lm_fp8=False,
-                   **kw) -> Workload:
+                   lm_nvfp4=False, **kw) -> Workload:
     """A reduced workload that the oracle finishes in seconds; by default the
     vocabulary, prefix lengths and canvas are not multiples of the kernels'
     tile sizes, so every tiling has a ragged tail."""
     shape = ModelShape(d_model=d_model, n_heads=n_heads, n_kv_heads=n_kv_heads,
-                       head_dim=head_dim, vocab=vocab, dtype=dtype, lm_fp8=lm_fp8)
+                       head_dim=head_dim, vocab=vocab, dtype=dtype, lm_fp8=lm_fp8,
+                       lm_nvfp4=lm_nvfp4)
     return Workload(name, shape, batch=batch, canvas=canvas, steps=steps,
                     prefix_len=prefix_len, prefix_cap=prefix_cap, **kw)
 
