@@ -33,6 +33,7 @@ L2 flush is needed between steps.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -327,11 +328,12 @@ def kernel_figures(r, pk, n_blocks):
         n_full = min(n_full, max(1, -(-slot // max(1, wl.quota_eff))))
     mean = {k: statistics.mean(v[:n_full]) for k, v in times.items()}
     lm_fp8 = bool(getattr(sh, "lm_fp8", False))
+    lm_nvfp4 = bool(getattr(sh, "lm_nvfp4", False))
     es = 2 if sh.dtype == "bf16" else 4
     shape = RL.StepShape(sh.d_model, sh.n_heads, sh.n_kv_heads, sh.head_dim, sh.vocab, es,
                          wl.canvas, r.lens)
-    work = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 else 256,
-                        lm_elem_bytes=1 if lm_fp8 else 0)
+    work = RL.step_work(shape, lm_tile=128 if wl.batch * wl.canvas <= 128 or lm_nvfp4 else 256,
+                        lm_elem_bytes=1 if lm_fp8 else 0, lm_nvfp4=lm_nvfp4)
     out = {"stages_us": {k: round(v, 2) for k, v in mean.items()},
            "steps_averaged": n_full, "step_algorithmic_bytes": work["step"]["bytes"]}
     if sh.dtype != "bf16":
@@ -342,11 +344,14 @@ def kernel_figures(r, pk, n_blocks):
         ach, peak, unit, bound = work["lm_head"]["bytes"] / lm_s / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
         src = " hbm_gbs"
     else:
-        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * (2 if lm_fp8 else 1)
+        ratio = 4 if lm_nvfp4 else (2 if lm_fp8 else 1)
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * ratio
         ach, unit, bound = work["lm_head"]["flop"] / lm_s / 1e12, "TFLOP/s", "tensor"
-        src = " bf16_tflops_sustained" + (" x 2 (e4m3 : bf16 nominal ratio)" if lm_fp8 else "")
+        src = " bf16_tflops_sustained" + (
+            " x %d (%s : bf16 nominal ratio)" % (ratio, "nvfp4" if lm_nvfp4 else "e4m3")
+            if ratio > 1 else "")
     roof = {"kernel": "gemm_tc_kernel<EPI_LM%s> (LM head + fused vocab reduction)"
-                      % (", e4m3" if lm_fp8 else ""),
+                      % (", nvfp4" if lm_nvfp4 else (", e4m3" if lm_fp8 else "")),
             "bound": bound, "achieved": round(ach, 1), "peak": peak, "unit": unit,
             "frac": round(ach / peak, 4), "traffic": _ncu_traffic(wl.name),
             "peak_source": pk.get("source", "measured") + src,
@@ -463,7 +468,8 @@ def run_ours(a):
             "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": Wm,
             "ms_per_step": round(ms_max / K, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("bf16, LM head e4m3" if getattr(sh, "lm_fp8", False) else "bf16")
+            "dtype": ("bf16, LM head nvfp4" if getattr(sh, "lm_nvfp4", False) else
+                      ("bf16, LM head e4m3" if getattr(sh, "lm_fp8", False) else "bf16"))
                      if sh.dtype == "bf16" else "f32",
             "data": "synthetic: seeded random-init weights N(0,0.02), embeddings and prefix "
                     "K/V N(0,1), all-mask canvas",
@@ -497,7 +503,8 @@ def run_ours(a):
         pg.destroy_process_group()
 
 
-CONFIG_WORKLOADS = ["tiny", "8b_b1", "batched", "longctx", "encdec", "encdec_eb"]
+CONFIG_WORKLOADS = ["tiny", "8b_b1", "batched", "longctx", "encdec", "encdec_eb",
+                    "8b_b1_fp8", "8b_b1_nvfp4"]
 
 
 def measure_configs(skip, device, pk):
@@ -512,7 +519,8 @@ def measure_configs(skip, device, pk):
             out[name] = "the headline line"
             continue
         wl = W.WORKLOADS[name]
-        key = (wl.shape, wl.seed)
+        # the low-bit LM-head variants share the model's weights
+        key = (dataclasses.replace(wl.shape, lm_fp8=False, lm_nvfp4=False), wl.seed)
         if key not in uploads:
             from masked_block_diffusion_denoise_b200.session import host_to_device
             uploads.clear()

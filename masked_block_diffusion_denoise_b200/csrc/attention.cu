@@ -71,6 +71,18 @@ static_assert(kRecvOff + (kRowsCta + kMaxCluster) * kXoRowBytes <= kStages * kSt
               "exchange areas exceed the K/V ring");
 static_assert(kXoRowBytes % 16 == 0 && kRecvOff % 16 == 0, "bulk copies need 16-byte units");
 
+// maximum of a thread's 128 scores as eight independent chains and a tree
+// (a single chain of 128 dependent maxima would be latency, not throughput)
+__device__ __forceinline__ float row_max128(const float (&sv)[kKeys]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = sv[k];
+#pragma unroll
+  for (int j = 8; j < kKeys; ++j) m[j & 7] = fmaxf(m[j & 7], sv[j]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
 //   warp 0     TMA producer: 128-key K and V tiles (two 64-column halves each,
 //              128-byte swizzle) into a 3-stage ring;
@@ -317,18 +329,18 @@ __global__ void __launch_bounds__(192, 1)
           if (key_base + j >= k_end) sv[j] = -CUDART_INF_F;
       }
       // maximum on the raw scores (the scale is positive), then one FFMA per score
-      float mx = -CUDART_INF_F;
-#pragma unroll
-      for (int j = 0; j < kKeys; ++j) mx = fmaxf(mx, sv[j]);
+      const float mx = row_max128(sv);
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const float alpha = fast_exp2(m_run - m_new);
-      float rsum = 0.f;
+      // eight independent partial sums (no 128-long dependency chain)
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < kKeys; ++j) {
         const float e = fast_exp2(fmaf(sv[j], p.scale_log2, -m_new));
         sv[j] = e;
-        rsum += e;
+        rs[j & 7] += e;
       }
+      const float rsum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       l_run = l_run * alpha + rsum;
       m_run = m_new;
       // P(t) in bf16, two keys per 32-bit TMEM column, over the S(t) columns
@@ -504,32 +516,43 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------------------
 // Two query-row tiles per CTA (256 rows): when a KV head has at least 256
 // query rows (G * C >= 256), one CTA takes two 128-row tiles of the same
-// (sequence, KV head, key split), so each K/V tile crosses HBM once for both.
-// 10 warps:
-//   warp 0     TMA producer: K tiles into a 2-slot ring, V tiles into a
+// (sequence, KV head, key split), so each K/V tile is brought in once for
+// both and the two softmax warpgroups keep the exponent units busy while
+// the tensor core works for the other.  12 warps in three warpgroups:
+//   warps 0-3  softmax of row tile 0, warps 4-7 of row tile 1: thread =
+//              query row = TMEM lane; the 128 scores of a key tile are read
+//              from tensor memory once and kept in registers (the warpgroups
+//              raise their register limit to 224, setmaxnreg);
+//   warp 8     TMA producer: K tiles into a 2-slot ring, V tiles into a
 //              3-slot ring (128 keys x 128 dims, two 64-column halves each);
-//   warp 1     MMA issuer, per key tile t:  O0 += P0(t-1) V(t-1);
-//              S0(t) = Q0 K(t)^T;  O1 += P1(t-1) V(t-1);  S1(t) = Q1 K(t)^T
-//              -- each row tile has one S buffer, and tcgen05 operations of
-//              one thread run in order, so S_i(t) is written after P_i(t-1)
-//              has been read, and once S_i(t) is complete O_i holds every
-//              earlier P_i V (the softmax may rescale it at once);
-//   warps 2-5  softmax of row tile 0, warps 6-9 of row tile 1: the two
-//              warpgroups alternate with the tensor core (while one turns
-//              S_i(t) into P_i(t), the other's S or P V runs).
+//   warp 9     MMA issuer, polling without blocking: for each row tile i it
+//              issues O_i += P_i(t) V(t) as soon as P_i(t) and V(t) are there
+//              and S_i(t+1) = Q_i K(t+1)^T right after (one S buffer per row
+//              tile: tcgen05 operations of one thread run in order, so S_i(t+1)
+//              is written after P_i(t) has been read, and once S_i(t+1) is
+//              complete O_i holds every earlier P_i V, which the softmax may
+//              then rescale); a row tile never waits for the other;
+//   warps 10-11 idle (they complete the third warpgroup for setmaxnreg).
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).  Splits write
 // bf16 O (one split) or f32 partials for attn_combine_kernel.
 // ---------------------------------------------------------------------------
 constexpr int kTile2 = 2 * kHalf;                 // one 128-row / 128-key tile: 32 KB
 constexpr int kKSlots2 = 2, kVSlots2 = 3;
+constexpr int kAttn2Threads = 384;
 constexpr int kAttn2Smem = 2 * kTile2 + (kKSlots2 + kVSlots2) * kTile2 + 1024 + 512;
 static_assert(kAttn2Smem <= 232448, "two-tile attention exceeds shared memory");
+// register split: 384 threads launch with 168 registers each (64512); the
+// third warpgroup gives back 112 per thread, the softmax warpgroups take 56
+constexpr int kAttn2RegsSoftmax = 224, kAttn2RegsOther = 56;
+static_assert(kAttn2RegsSoftmax * 256 + kAttn2RegsOther * 128 <= 168 * kAttn2Threads,
+              "register split exceeds the launch's registers");
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kAttn2Threads, 1)
     attn_tc2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
   // timeline marks: 2 wait returned, 3 query and first K tile in shared
-  // memory, 4 O complete
+  // memory, 4 O complete, 5 row tile 0's softmax of key tile 1 begins, 6 its
+  // last key tile's P is written, 7 the producer has issued its last tile
   DLM_TRACE_CTA(TRACE_ATTENTION);
   const int split = blockIdx.x, pair = blockIdx.y, bg = blockIdx.z;
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
@@ -562,6 +585,7 @@ __global__ void __maxnreg__(200)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int kProducer = 8, kMma = 9;
   if (tid == 0) {
     for (int i = 0; i < kKSlots2; ++i) {
       mbar_init(&k_full[i], 1);
@@ -580,7 +604,7 @@ __global__ void __maxnreg__(200)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == kMma) tmem_alloc(tmem_slot, kTmemCols);
   __syncthreads();
   const int plane = b * p.Hkv + g;
   auto issue_k = [&](int t) {
@@ -600,7 +624,7 @@ __global__ void __maxnreg__(200)
   // K/V tiles wholly inside the cached prefix do not depend on the previous
   // kernel: the first ring slots' worth are issued before the wait
   int pre = 0;
-  if (warp == 0 && lane == 0) {
+  if (warp == kProducer && lane == 0) {
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
     if (p.q_tma) tma_prefetch(&tmQ);
@@ -614,7 +638,7 @@ __global__ void __maxnreg__(200)
   if (tid == 0) DLM_TRACE_MARK(2);
   const int row_base = pair * 2 * kRowsCta;   // first query row of tile 0
   if (p.q_tma) {
-    if (warp == 0 && lane == 0) {
+    if (warp == kProducer && lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * kTile2);
       for (int i = 0; i < 2; ++i) {
         const int z0 = b * p.C + (row_base + i * kRowsCta) / p.G;
@@ -633,8 +657,8 @@ __global__ void __maxnreg__(200)
         val = *reinterpret_cast<const uint4*>(
             p.q + ((size_t)(b * p.C + i) * p.H + (g * p.G + hh)) * kDh + ch * 8);
       }
-      const int tile = lr >> 7, tr = lr & 127;
-      *reinterpret_cast<uint4*>(qs + tile * kTile2 + (ch >> 3) * kHalf + sw128_off(tr, ch & 7)) =
+      const int tl = lr >> 7, tr = lr & 127;
+      *reinterpret_cast<uint4*>(qs + tl * kTile2 + (ch >> 3) * kHalf + sw128_off(tr, ch & 7)) =
           val;
     }
   }
@@ -643,8 +667,11 @@ __global__ void __maxnreg__(200)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
+  // the register split heads each warpgroup's branch (every warp of the
+  // warpgroup executes it)
+  if (warp >= kProducer) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAttn2RegsOther));
+  if (warp == kProducer) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int issued = pre;
@@ -655,14 +682,13 @@ __global__ void __maxnreg__(200)
           break;
         if (t >= kVSlots2 &&
             !mbar_wait_bounded(&v_empty[t % kVSlots2], (uint32_t)(((t / kVSlots2) & 1) ^ 1),
-                               abort_flag)) {
-          // K(t) is not issued either: keep the K and V counts equal
-          break;
-        }
+                               abort_flag))
+          break;   // K(t) is not issued either: the K and V counts stay equal
         issue_k(t);
         issue_v(t);
         ++issued;
       }
+      DLM_TRACE_MARK(7);
       if (*abort_flag) {
         // let the copies already in flight land before the CTA exits
         for (int t = issued - 1; t >= 0 && t >= issued - kKSlots2; --t)
@@ -672,7 +698,7 @@ __global__ void __maxnreg__(200)
       }
       if (p.q_tma) mbar_wait_bounded(q_full, 0, nullptr);   // the query tiles have landed
     }
-  } else if (warp == 1) {
+  } else if (warp == kMma) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRowsCta, kKeys);
@@ -699,50 +725,63 @@ __global__ void __maxnreg__(200)
                            (t > 0 || k > 0) ? 1u : 0u);
         }
       };
-      bool ok = (!p.q_tma || mbar_wait_bounded(q_full, 0, abort_flag));
-      for (int t = 0; ok && t <= n_tiles; ++t) {
-        const int tp = t - 1;   // the previous tile, whose P V runs now
-        if (tp >= 0) {
-          if (!mbar_wait_bounded(&p_full[0], (uint32_t)(tp & 1), abort_flag) ||
-              !mbar_wait_bounded(&v_full[tp % kVSlots2], (uint32_t)((tp / kVSlots2) & 1),
-                                 abort_flag)) {
-            ok = false;
+      // s_next[i]: next S tile of row tile i; pv_next[i]: next P V tile.
+      // S_i(t) may be issued once P_i(t-1) V has been (s_next == pv_next);
+      // a K slot is released when both row tiles' S of it are issued, a V
+      // slot when both P V are.  A row tile is at most one phase ahead of
+      // any barrier it tests (its S(t) needs its S(t-2), whose K slot phase
+      // came first; its P V(t) needs the V slot's previous phase done), so
+      // the non-blocking parity tests cannot alias.
+      int s_next[2] = {0, 0}, pv_next[2] = {0, 0};
+      bool ok = !p.q_tma || mbar_wait_bounded(q_full, 0, abort_flag);
+      uint64_t t_idle = 0;
+      for (uint32_t spin = 0; ok && (pv_next[0] < n_tiles || pv_next[1] < n_tiles); ++spin) {
+        bool progress = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int ts = s_next[i];
+          if (ts < n_tiles && ts == pv_next[i] &&
+              mbar_test_wait(&k_full[ts % kKSlots2], (uint32_t)((ts / kKSlots2) & 1))) {
+            if (ts == 0 && i == 0) DLM_TRACE_MARK(3);
+            tc_fence_after();
+            issue_s(i, ts);
+            s_next[i] = ts + 1;
+            progress = true;
+            // K(ts) is free once both row tiles' S(ts) have been issued
+            if (s_next[0] > ts && s_next[1] > ts) umma_commit(&k_empty[ts % kKSlots2]);
+          }
+          const int tp = pv_next[i];
+          if (tp < s_next[i] && mbar_test_wait(&p_full[i], (uint32_t)(tp & 1)) &&
+              mbar_test_wait(&v_full[tp % kVSlots2], (uint32_t)((tp / kVSlots2) & 1))) {
+            tc_fence_after();
+            issue_pv(i, tp);
+            pv_next[i] = tp + 1;
+            progress = true;
+            if (pv_next[0] > tp && pv_next[1] > tp) umma_commit(&v_empty[tp % kVSlots2]);
+          }
+        }
+        if (progress) {
+          t_idle = 0;
+        } else if ((spin & 255u) == 0) {
+          if (*abort_flag) break;
+          const uint64_t now = global_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitLimitNs) {
+            *abort_flag = 1;
             break;
           }
-          tc_fence_after();
-          issue_pv(0, tp);
-        }
-        if (t < n_tiles) {
-          if (!mbar_wait_bounded(&k_full[t % kKSlots2], (uint32_t)((t / kKSlots2) & 1),
-                                 abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (t == 0) DLM_TRACE_MARK(3);
-          tc_fence_after();
-          issue_s(0, t);
-        }
-        if (tp >= 0) {
-          if (!mbar_wait_bounded(&p_full[1], (uint32_t)(tp & 1), abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(1, tp);
-          umma_commit(&v_empty[tp % kVSlots2]);
-        }
-        if (t < n_tiles) {
-          issue_s(1, t);
-          umma_commit(&k_empty[t % kKSlots2]);
         }
       }
       // O complete (or, after an abort, every MMA issued has finished)
       umma_commit(o_done);
       mbar_wait_bounded(o_done, 0, nullptr);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kAttn2RegsSoftmax));
     // ---------------- softmax warpgroups ----------------
-    const int tile = (warp - 2) >> 2;                 // row tile of this warpgroup
+    const int tile = warp >> 2;                       // row tile of this warpgroup
     const int quad = warp & 3;
     const int row = quad * 32 + lane;                 // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -755,51 +794,48 @@ __global__ void __maxnreg__(200)
         ok = false;
         break;
       }
+      if (t == 1 && tile == 0 && row == 0) DLM_TRACE_MARK(5);
       tc_fence_after();
-      // two passes over S in tensor memory (64 columns live at a time): the
-      // tile maximum, then P = exp2(S * scale - m) written over S as bf16
-      // pairs; keys past the split's end (ragged last tile) count as -inf
-      const int key_base = k_begin + t * kKeys;
-      const int n_valid = min(kKeys, k_end - key_base);
-      float mx = -CUDART_INF_F;
+      float sv[kKeys];
+      {
+        uint32_t raw[kKeys / 32][32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t raw[2][32];
-        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64), raw[0]);
-        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64 + 32), raw[1]);
+        for (int c = 0; c < kKeys / 32; ++c)
+          tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(c * 32), raw[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float v = __uint_as_float(raw[j >> 5][j & 31]);
-          mx = fmaxf(mx, h * 64 + j < n_valid ? v : -CUDART_INF_F);
-        }
+        for (int c = 0; c < kKeys / 32; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(raw[c][j]);
       }
+      const int key_base = k_begin + t * kKeys;
+      if (key_base + kKeys > k_end) {   // ragged last tile (warp-uniform): mask past the end
+#pragma unroll
+        for (int j = 0; j < kKeys; ++j)
+          if (key_base + j >= k_end) sv[j] = -CUDART_INF_F;
+      }
+      const float mx = row_max128(sv);
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const float alpha = fast_exp2(m_run - m_new);
-      float rsum = 0.f;
+      // eight independent partial sums (no 128-long dependency chain)
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t raw[2][32];
-        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64), raw[0]);
-        tmem_ld32_nowait(lane_addr + s_col + (uint32_t)(h * 64 + 32), raw[1]);
-        tmem_wait_ld();
-        uint32_t w[32];
+      for (int c = 0; c < kKeys / 32; ++c) {
+        uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int k0 = h * 64 + 2 * j;
-          const float s0 = __uint_as_float(raw[(2 * j) >> 5][(2 * j) & 31]);
-          const float s1 = __uint_as_float(raw[(2 * j + 1) >> 5][(2 * j + 1) & 31]);
-          const float e0 = k0 < n_valid ? fast_exp2(fmaf(s0, p.scale_log2, -m_new)) : 0.f;
-          const float e1 = k0 + 1 < n_valid ? fast_exp2(fmaf(s1, p.scale_log2, -m_new)) : 0.f;
-          rsum += e0 + e1;
+        for (int j = 0; j < 16; ++j) {
+          const float e0 = fast_exp2(fmaf(sv[32 * c + 2 * j], p.scale_log2, -m_new));
+          const float e1 = fast_exp2(fmaf(sv[32 * c + 2 * j + 1], p.scale_log2, -m_new));
+          rs[j & 7] += e0 + e1;
           w[j] = pack_bf16(e0, e1);
         }
-        tmem_st32_u(lane_addr + s_col + (uint32_t)(h * 32), w);
+        tmem_st16_u(lane_addr + s_col + (uint32_t)(c * 16), w);
       }
+      const float rsum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       l_run = l_run * alpha + rsum;
       m_run = m_new;
-      // O_i holds every earlier P_i V (see the MMA order above): rescale it
-      // only when some row of the warp saw a new maximum
+      // O_i holds every earlier P_i V (see the MMA issuer): rescale it only
+      // when some row of the warp saw a new maximum
       if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < kDh / 32; ++c) {
@@ -814,6 +850,7 @@ __global__ void __maxnreg__(200)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[tile]);
+      if (t == n_tiles - 1 && tile == 0 && row == 0) DLM_TRACE_MARK(6);
     }
     if (ok && mbar_wait_bounded(o_done, 0, abort_flag)) {
       tc_fence_after();
@@ -853,7 +890,7 @@ __global__ void __maxnreg__(200)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMma) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -1055,8 +1092,8 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
     // two row tiles per CTA: one split writes O, more write partials
     if (ap.cluster > 1) return cudaErrorInvalidValue;
     dim3 grid2(ap.nsplit, (ap.rtiles + 1) / 2, ap.B * md.Hkv);
-    cudaError_t e = launch_pdl(attn_tc2_kernel, grid2, dim3(320), kAttn2Smem, st, tmK, tmV,
-                               qmap, p);
+    cudaError_t e = launch_pdl(attn_tc2_kernel, grid2, dim3(kAttn2Threads), kAttn2Smem, st, tmK,
+                               tmV, qmap, p);
     if (e != cudaSuccess || ap.nsplit == 1) return e;
     const int rows_per_block = 8;
     dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);

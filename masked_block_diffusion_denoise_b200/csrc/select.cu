@@ -9,6 +9,10 @@
 // EntropyBoundScheduler), the course "Diffusion LLMs" section 12 (confidence
 // order, ties to the lower position) and the Nemotron guide, section 6 (the
 // last step fills every remaining mask).
+#include <algorithm>
+
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 
 namespace dlm {
@@ -137,6 +141,11 @@ __device__ int eos_fill(int32_t* tok, uint8_t* com, int C, int eos_id, int* e_s,
   return e < C ? e : -1;
 }
 
+// One canvas per CTA, or, when the partials are given and the canvas is
+// longer than 32 positions, one canvas per thread-block cluster of kcl CTAs:
+// CTA r of the cluster reduces rows [r * rows_per, (r + 1) * rows_per) and
+// writes their candidates, confidences and entropies into the shared memory
+// of the cluster's first CTA, which then selects for the whole canvas.
 __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __restrict__ tokens,
                               uint8_t* __restrict__ committed, int32_t* __restrict__ step,
                               uint8_t* __restrict__ done, int32_t* __restrict__ eos_pos,
@@ -144,7 +153,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
                               const float* __restrict__ part, int n_part, int stage_bytes,
                               int32_t* __restrict__ cand, float* __restrict__ conf,
                               float* __restrict__ ent, dlm_canvas_stats* stats,
-                              const int* n_active, int* err) {
+                              const int* n_active, int* err, int kcl, int rows_per) {
   // timeline marks: 2 wait returned, 3 rows reduced, 4 keys sorted, 5 done
   DLM_TRACE_CTA(TRACE_COMMIT);
   // Inside a step (partials given) the direct predecessor is the LM head,
@@ -168,11 +177,13 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
     __syncthreads();
   }
   if (!early) pdl_wait_then_release();
-  const int b = blockIdx.x;
+  const int rank = kcl > 1 ? (int)cooperative_groups::this_cluster().block_rank() : 0;
+  const int b = blockIdx.x / kcl;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int i = threadIdx.x;
   const int C = a.C;
   const size_t base = (size_t)b * C;
+  const int r0 = rank * rows_per, r1 = min(C, r0 + rows_per);   // this CTA's rows
   // the active count, this canvas's flag and state in one round trip; the
   // state goes to registers and reaches shared memory after the reduction
   const int na = n_active != nullptr ? __ldcg(n_active) : 1;
@@ -180,7 +191,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   const int s = __ldcg(step + b);
   int32_t tok_r = 0;
   uint8_t com_r = 0;
-  if (i < C) {
+  if (rank == 0 && i < C) {
     tok_r = __ldcg(tokens + base + i);
     com_r = __ldcg(committed + base + i);
   }
@@ -191,8 +202,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   __shared__ int32_t stable_s;
   __shared__ dlm_canvas_stats st0;
   const bool stopping = a.stop_entropy > 0.f;
-  if (stopping && i < C) prev_s[i] = __ldcg(prev_cand + base + i);
-  if (i == 0) {
+  if (rank == 0 && stopping && i < C) prev_s[i] = __ldcg(prev_cand + base + i);
+  if (rank == 0 && i == 0) {
     if (stopping) stable_s = __ldcg(stable + b);
     if (stats != nullptr) {
       const int32_t* sp = reinterpret_cast<const int32_t*>(stats + b);
@@ -206,12 +217,16 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
   }
   if (early) pdl_wait_then_release();
   if (threadIdx.x == 0) DLM_TRACE_MARK(2);
+  // uniform over a cluster: its CTAs share the canvas
   if (na == 0 || dn) return;
+  // this CTA's slice of the partials (stage_bytes is the largest slice)
+  const int slice_bytes = (r1 - r0) * kLmFields * n_part * (int)sizeof(float);
   if (staged && i == 0) {
-    mbar_arrive_expect_tx(&stage_bar, (uint32_t)stage_bytes);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(part + base * kLmFields * (size_t)n_part);
-    for (int off = 0; off < stage_bytes; off += kStageChunk)
-      bulk_load_global(stage_raw + off, src + off, (uint32_t)min(kStageChunk, stage_bytes - off),
+    mbar_arrive_expect_tx(&stage_bar, (uint32_t)slice_bytes);
+    const uint8_t* src =
+        reinterpret_cast<const uint8_t*>(part + (base + r0) * kLmFields * (size_t)n_part);
+    for (int off = 0; off < slice_bytes; off += kStageChunk)
+      bulk_load_global(stage_raw + off, src + off, (uint32_t)min(kStageChunk, slice_bytes - off),
                        &stage_bar);
   }
   __shared__ unsigned long long keys[kMaxC];
@@ -227,13 +242,28 @@ __global__ void __launch_bounds__(1024) commit_kernel(SelectArgs a, int32_t* __r
       raise_error(err, DLM_ETIMEOUT);
       mbar_wait_bounded(&stage_bar, 0, nullptr);   // the copies land before the CTA exits
     }
-    // a6: the cross-tile reduction of this canvas's rows, one warp per row
-    for (int r = warp; r < C; r += nw) {
+    // a6: the cross-tile reduction of this CTA's rows, one warp per row; the
+    // results go to the cluster's first CTA (this CTA without a cluster)
+    int32_t* cand_l = cand_s;
+    float *conf_l = conf_s, *ent_l = ent_s;
+    if (kcl > 1) {
+      cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+      cand_l = cl.map_shared_rank(cand_s, 0);
+      conf_l = cl.map_shared_rank(conf_s, 0);
+      ent_l = cl.map_shared_rank(ent_s, 0);
+    }
+    for (int r = r0 + warp; r < r1; r += nw) {
       const size_t row = base + r;
-      const float* pr = staged ? reinterpret_cast<const float*>(stage_raw) + r * kLmFields * n_part
-                               : part + row * kLmFields * (size_t)n_part;
-      reduce_row(pr, n_part, lane, cand + row, conf + row, ent + row,
-                 cand_s + r, conf_s + r, ent_s + r);
+      const float* pr = staged
+                            ? reinterpret_cast<const float*>(stage_raw) + (r - r0) * kLmFields * n_part
+                            : part + row * kLmFields * (size_t)n_part;
+      reduce_row(pr, n_part, lane, cand + row, conf + row, ent + row, cand_l + r, conf_l + r,
+                 ent_l + r);
+    }
+    if (kcl > 1) {
+      // every row of the canvas is in the first CTA's shared memory
+      cooperative_groups::this_cluster().sync();
+      if (rank != 0) return;
     }
   } else if (i < C) {
     cand_s[i] = cand[base + i];
@@ -443,21 +473,50 @@ cudaError_t commit_step(const SelectArgs& a, int32_t* tokens, uint8_t* committed
   while (P < a.C) P <<= 1;
   if (P > kMaxC) return cudaErrorInvalidValue;
   if (part != nullptr) P = 1024;   // 32 warps for the row reductions
-  // the partials of a canvas go through shared memory when they fit and
-  // every canvas's block starts on a 16-byte boundary
+  // with partials, a canvas of more than 32 positions is reduced by a
+  // cluster of up to 8 CTAs (an even number of rows each)
+  int kcl = 1, rows_per = a.C;
+  if (part != nullptr && a.C > 32) {
+    kcl = std::min(8, (a.C + 31) / 32);
+    rows_per = (a.C + kcl - 1) / kcl;
+    rows_per += rows_per & 1;
+    kcl = (a.C + rows_per - 1) / rows_per;
+  }
+  // a slice's partials go through shared memory when the largest fits and
+  // every slice starts on a 16-byte boundary
   int stage_bytes = 0;
   if (part != nullptr) {
-    const long long bytes = (long long)a.C * kLmFields * n_part * (long long)sizeof(float);
-    if (bytes <= kStageMax && bytes % 16 == 0) stage_bytes = (int)bytes;
+    const long long row_bytes = (long long)kLmFields * n_part * (long long)sizeof(float);
+    const long long bytes = rows_per * row_bytes;
+    if (bytes <= kStageMax && bytes % 16 == 0 && (a.C * row_bytes) % 16 == 0)
+      stage_bytes = (int)bytes;
   }
   static cudaError_t attr = cudaErrorNotReady;   // per process; one device per process
   if (attr == cudaErrorNotReady)
     attr = cudaFuncSetAttribute(commit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kStageMax);
   if (attr != cudaSuccess) return attr;
-  return launch_pdl(commit_kernel, dim3(a.B), dim3(P), (size_t)stage_bytes, st, a, tokens,
-                    committed, step, done, eos_pos, prev_cand, stable, part, n_part, stage_bytes,
-                    cand, conf, ent, stats, n_active, err);
+  if (kcl == 1)
+    return launch_pdl(commit_kernel, dim3(a.B), dim3(P), (size_t)stage_bytes, st, a, tokens,
+                      committed, step, done, eos_pos, prev_cand, stable, part, n_part,
+                      stage_bytes, cand, conf, ent, stats, n_active, err, 1, rows_per);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * kcl);
+  cfg.blockDim = dim3(P);
+  cfg.dynamicSmemBytes = (size_t)stage_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)kcl;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, commit_kernel, a, tokens, committed, step, done, eos_pos,
+                            prev_cand, stable, part, n_part, stage_bytes, cand, conf, ent, stats,
+                            n_active, err, kcl, rows_per);
 }
 
 }  // namespace dlm

@@ -75,11 +75,14 @@ class StepShape:
 
 
 def step_work(s: StepShape, lm_tile: int = 128, part_bytes: int = 24,
-              lm_elem_bytes: int = 0) -> Dict[str, Dict[str, float]]:
+              lm_elem_bytes: int = 0, lm_nvfp4: bool = False) -> Dict[str, Dict[str, float]]:
     """Algorithmic bytes and flops of each stage of one denoise step.
     lm_elem_bytes = 1: the e4m3 LM head (one-byte weights and input rows, a
     float32 scale per vocabulary row and per input row, and the quantisation
-    of the input rows); 0: the head in the model's element type."""
+    of the input rows); lm_nvfp4: the NVFP4 head (half a byte per element,
+    one e4m3 scale per 16 elements, a float32 scale per row, for weights and
+    input rows, and the quantisation of the input rows); otherwise the head
+    in the model's element type."""
     e = s.elem_bytes
     M, d, V = s.rows, s.d_model, s.vocab
     qd, kvd = s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
@@ -102,7 +105,11 @@ def step_work(s: StepShape, lm_tile: int = 128, part_bytes: int = 24,
         "reduce": {"bytes": float(M * ntiles * part_bytes + 12 * M), "flop": 0.0},
         "commit": {"bytes": float(M * (4 + 1 + 4 + 4 + 4) * 2), "flop": 0.0},
     }
-    if lm_elem_bytes == 1:
+    if lm_nvfp4:
+        q4 = lambda rows: rows * d / 2 + rows * d / 16 + 4 * rows
+        out["lm_head"]["bytes"] = float(q4(V) + q4(M) + M * ntiles * part_bytes)
+        out["quantize"]["bytes"] = float(M * d * e + q4(M))
+    elif lm_elem_bytes == 1:
         out["lm_head"]["bytes"] = float(V * d + M * d + 4 * V + 4 * M + M * ntiles * part_bytes)
         out["quantize"]["bytes"] = float(M * d * e + M * d + 4 * M)
     out["step"] = {"bytes": sum(v["bytes"] for v in out.values()),
