@@ -405,6 +405,13 @@ int dlm_trace_clear(void);
  * DLM_EINVAL for n_launches < 0 or an fp32 context. */
 int dlm_test_withhold_loads(dlm_ctx *ctx, int n_launches);
 
+/* Test hook for the attention kernels' polynomial exponential (part of
+ * every key tile's exponentials are computed on the FMA pipe instead of the
+ * exponential unit): out[i] = 2^x[i] by Cody-Waite range reduction and a
+ * cubic on [-1/2, 1/2] (maximum relative error 7.5e-5 for -125 <= x <= 8; 0
+ * below -125).  x, out: device float [n].  DLM_EINVAL for NULL or n < 0. */
+int dlm_test_exp2(const float *x, float *out, int n, void *stream);
+
 /* Number of kernel launches one dlm_denoise_step made for this batch and
  * configuration (the last one issued), for launch accounting. */
 int dlm_launches_per_step(const dlm_ctx *ctx);

@@ -28,7 +28,7 @@ __all__ = [
     "DLM_STAGE_ATTENTION", "DLM_STAGE_WO", "DLM_STAGE_LM_HEAD", "DLM_STAGE_COMMIT",
     "DLM_NUM_STAGES", "dlm_attention_noalloc", "dlm_attention_noalloc_check",
     "dlm_trace_layout", "dlm_trace_read", "dlm_trace_clear", "dlm_decode_steps",
-    "dlm_attention_plan", "dlm_test_withhold_loads",
+    "dlm_attention_plan", "dlm_test_withhold_loads", "dlm_test_exp2",
 ]
 
 DLM_OK, DLM_EINVAL, DLM_ENOMEM, DLM_ECUDA, DLM_ECAP, DLM_ETIMEOUT, DLM_EBOUNDS, DLM_ESTATE = \
@@ -124,6 +124,7 @@ _SIGS = {
     "dlm_check": (_I, [_P, _P]),
     "dlm_launches_per_step": (_I, [_P]),
     "dlm_test_withhold_loads": (_I, [_P, _I]),
+    "dlm_test_exp2": (_I, [_P, _P, _I, _P]),
     "dlm_trace_layout": (_I, [ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "dlm_trace_read": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_size_t]),
     "dlm_trace_clear": (_I, []),
@@ -312,6 +313,14 @@ def dlm_check(ctx, stream=None) -> int:
 
 def dlm_launches_per_step(ctx) -> int:
     return _check(ctx, lib().dlm_launches_per_step(ctx))
+
+
+def dlm_test_exp2(x, out, n: int, stream=None) -> int:
+    """out = 2^x by the attention kernels' polynomial exponential (test hook)."""
+    rc = lib().dlm_test_exp2(_ptr(x), _ptr(out), n, _stream(stream))
+    if rc != DLM_OK:
+        raise DlmError(rc, lib().dlm_last_error(None).decode())
+    return rc
 
 
 def dlm_test_withhold_loads(ctx, n_launches: int) -> int:

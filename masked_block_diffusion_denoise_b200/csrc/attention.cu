@@ -19,6 +19,9 @@
 // (log-sum-exp).
 #include <math_constants.h>
 
+#include <cstdlib>
+#include <cstring>
+
 #include <cooperative_groups.h>
 
 #include "kernels.h"
@@ -41,6 +44,13 @@ constexpr int kStageBytes = 4 * kHalf;        // K and V tiles, two halves each:
 constexpr int kAttnSmem = kQBytes + kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 512;           // S/P double buffer (2 x 128) + O (128)
 constexpr uint32_t kColO = 256;
+// Online softmax with a lagging reference maximum: a row's reference moves
+// to its new maximum only when that exceeds the reference by more than
+// kRescaleLog2 (log2 units), so P = exp2(s - reference) stays below 2^8 and
+// O is rescaled in tensor memory only when a row of the warp moves -- rarely
+// after the first key tile.  Exact for any reference: the final O / l, and a
+// split's (O, m, l) for the combine, do not depend on where it sat.
+constexpr float kRescaleLog2 = 8.0f;
 
 struct AttnParams {
   const __nv_bfloat16* q;
@@ -94,6 +104,7 @@ __device__ __forceinline__ float row_max128(const float (&sv)[kKeys]) {
 //              when a row's maximum moved, rescales O in TMEM.
 // tcgen05 operations of the issuing thread run in order, so S(t+2) cannot
 // overwrite P(t) before P(t) V(t) has read it.
+template <bool POLY>
 __global__ void __launch_bounds__(192, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
@@ -329,14 +340,18 @@ __global__ void __launch_bounds__(192, 1)
           if (key_base + j >= k_end) sv[j] = -CUDART_INF_F;
       }
       // maximum on the raw scores (the scale is positive), then one FFMA per score
-      const float mx = row_max128(sv);
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const float alpha = fast_exp2(m_run - m_new);
+      const float mx = row_max128(sv) * p.scale_log2;
+      const bool move = __any_sync(0xffffffffu, mx > m_run + kRescaleLog2);
+      const float m_new = move ? fmaxf(m_run, mx) : m_run;
+      const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;
       // eight independent partial sums (no 128-long dependency chain)
+      // POLY: 3 of every 8 exponentials on the FMA pipe (exp2_poly), the
+      // rest on the exponential unit
       float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < kKeys; ++j) {
-        const float e = fast_exp2(fmaf(sv[j], p.scale_log2, -m_new));
+        const float x = fmaf(sv[j], p.scale_log2, -m_new);
+        const float e = POLY && (j & 7) >= 5 ? exp2_poly(x) : fast_exp2(x);
         sv[j] = e;
         rs[j & 7] += e;
       }
@@ -351,9 +366,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int j = 0; j < 32; ++j) w[j] = pack_bf16(sv[64 * c + 2 * j], sv[64 * c + 2 * j + 1]);
         tmem_st32_u(lane_addr + (uint32_t)(buf * kKeys + c * 32), w);
       }
-      // rescale O only when some row of the warp saw a new maximum; O must
-      // first hold every earlier P V
-      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      // rescale O only when the warp's reference moved; O must first hold
+      // every earlier P V
+      if (t > 0 && move) {
         if (!mbar_wait_bounded(pv_done, (uint32_t)((t - 1) & 1), abort_flag)) {
           ok = false;
           break;
@@ -547,6 +562,7 @@ constexpr int kAttn2RegsSoftmax = 224, kAttn2RegsOther = 56;
 static_assert(kAttn2RegsSoftmax * 256 + kAttn2RegsOther * 128 <= 168 * kAttn2Threads,
               "register split exceeds the launch's registers");
 
+template <bool POLY>
 __global__ void __launch_bounds__(kAttn2Threads, 1)
     attn_tc2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const AttnParams p) {
@@ -760,6 +776,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
             if (pv_next[0] > tp && pv_next[1] > tp) umma_commit(&v_empty[tp % kVSlots2]);
           }
         }
+        if (!progress) {
+          // nothing ready: sleep on the row tile that has waited longest for
+          // its P (briefly, so the other one is not kept waiting), instead of
+          // spinning on the issue slots the softmax warps of this SM
+          // sub-partition need
+          const int w = pv_next[0] <= pv_next[1] ? 0 : 1;
+          if (pv_next[w] < s_next[w])
+            mbar_try_wait_hint(&p_full[w], (uint32_t)(pv_next[w] & 1), 200u);
+        }
         if (progress) {
           t_idle = 0;
         } else if ((spin & 255u) == 0) {
@@ -814,9 +839,10 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         for (int j = 0; j < kKeys; ++j)
           if (key_base + j >= k_end) sv[j] = -CUDART_INF_F;
       }
-      const float mx = row_max128(sv);
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const float alpha = fast_exp2(m_run - m_new);
+      const float mx = row_max128(sv) * p.scale_log2;
+      const bool move = __any_sync(0xffffffffu, mx > m_run + kRescaleLog2);
+      const float m_new = move ? fmaxf(m_run, mx) : m_run;
+      const float alpha = move ? fast_exp2(m_run - m_new) : 1.f;
       // eight independent partial sums (no 128-long dependency chain)
       float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -824,8 +850,11 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float e0 = fast_exp2(fmaf(sv[32 * c + 2 * j], p.scale_log2, -m_new));
-          const float e1 = fast_exp2(fmaf(sv[32 * c + 2 * j + 1], p.scale_log2, -m_new));
+          // POLY: pairs 10..15 of every 16 (3 in 8 exponentials) on the FMA pipe
+          const float x0 = fmaf(sv[32 * c + 2 * j], p.scale_log2, -m_new);
+          const float x1 = fmaf(sv[32 * c + 2 * j + 1], p.scale_log2, -m_new);
+          const float e0 = POLY && j >= 10 ? exp2_poly(x0) : fast_exp2(x0);
+          const float e1 = POLY && j >= 10 ? exp2_poly(x1) : fast_exp2(x1);
           rs[j & 7] += e0 + e1;
           w[j] = pack_bf16(e0, e1);
         }
@@ -835,8 +864,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       l_run = l_run * alpha + rsum;
       m_run = m_new;
       // O_i holds every earlier P_i V (see the MMA issuer): rescale it only
-      // when some row of the warp saw a new maximum
-      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      // when the warp's reference moved
+      if (t > 0 && move) {
 #pragma unroll
         for (int c = 0; c < kDh / 32; ++c) {
           float o[32];
@@ -1038,35 +1067,40 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(int H, int Hkv, int C, in
 
 }  // namespace
 
-// the attention kernel's function attributes: its shared memory, and
-// clusters of up to 16 CTAs (beyond the portable 8), once per process
-cudaError_t attn_set_attributes() {
+// diagnostic switch: DLM_ATTN_POLY=1 computes 3 of every 8 of the softmax's
+// exponentials with exp2_poly on the FMA pipe instead of the exponential unit
+bool attn_poly() {
+  const char* e = std::getenv("DLM_ATTN_POLY");
+  return e != nullptr && std::strcmp(e, "1") == 0;
+}
+
+// the attention kernels' function attributes: shared memory, and clusters of
+// up to 16 CTAs (beyond the portable 8) for the 128-row kernel, once per
+// process
+template <bool POLY>
+cudaError_t attn_set_attributes_t() {
   static cudaError_t done = cudaErrorNotReady;
   if (done == cudaErrorNotReady) {
-    done = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    done = cudaFuncSetAttribute(attn_tc_kernel<POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kAttnSmem);
     if (done == cudaSuccess)
-      done = cudaFuncSetAttribute(attn_tc_kernel,
+      done = cudaFuncSetAttribute(attn_tc_kernel<POLY>,
                                   cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (done == cudaSuccess)
+      done = cudaFuncSetAttribute(attn_tc2_kernel<POLY>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kAttn2Smem);
   }
   return done;
 }
+cudaError_t attn_set_attributes() { return attn_set_attributes_t<false>(); }
 
-cudaError_t attn2_set_attributes() {
-  static cudaError_t done = cudaErrorNotReady;
-  if (done == cudaErrorNotReady)
-    done = cudaFuncSetAttribute(attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kAttn2Smem);
-  return done;
-}
-
-cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
-                           const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q, void* o,
-                           float* opart, float2* ml, const int32_t* lens, const uint8_t* done,
-                           const int* n_active, int* err, cudaStream_t st) {
-  if (cudaError_t e = attn_set_attributes(); e != cudaSuccess) return e;
-  if (ap.rows == 2 * kRowsCta)
-    if (cudaError_t e = attn2_set_attributes(); e != cudaSuccess) return e;
+template <bool POLY>
+cudaError_t attention_bf16_t(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q,
+                             void* o, float* opart, float2* ml, const int32_t* lens,
+                             const uint8_t* done, const int* n_active, int* err,
+                             cudaStream_t st) {
+  if (cudaError_t e = attn_set_attributes_t<POLY>(); e != cudaSuccess) return e;
   AttnParams p;
   p.q = (const __nv_bfloat16*)q;
   p.o = (__nv_bfloat16*)o;
@@ -1092,8 +1126,8 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
     // two row tiles per CTA: one split writes O, more write partials
     if (ap.cluster > 1) return cudaErrorInvalidValue;
     dim3 grid2(ap.nsplit, (ap.rtiles + 1) / 2, ap.B * md.Hkv);
-    cudaError_t e = launch_pdl(attn_tc2_kernel, grid2, dim3(kAttn2Threads), kAttn2Smem, st, tmK,
-                               tmV, qmap, p);
+    cudaError_t e = launch_pdl(attn_tc2_kernel<POLY>, grid2, dim3(kAttn2Threads), kAttn2Smem, st,
+                               tmK, tmV, qmap, p);
     if (e != cudaSuccess || ap.nsplit == 1) return e;
     const int rows_per_block = 8;
     dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);
@@ -1120,15 +1154,27 @@ cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtens
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmK, tmV, qmap, p);
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel<POLY>, tmK, tmV, qmap, p);
   }
-  cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kAttnSmem, st, tmK, tmV, qmap, p);
+  cudaError_t e =
+      launch_pdl(attn_tc_kernel<POLY>, grid, dim3(192), kAttnSmem, st, tmK, tmV, qmap, p);
   if (e != cudaSuccess || ap.nsplit == 1) return e;
   const int rows_per_block = 8;
   dim3 g2(ap.B * md.Hkv, (ap.R + rows_per_block - 1) / rows_per_block);
   return launch_pdl(attn_combine_kernel, g2, dim3(32 * rows_per_block), 0, st,
                     (const float*)opart, (const float2*)ml, (__nv_bfloat16*)o, lens, done,
                     n_active, md.H, md.Hkv, ap.G, ap.C, ap.R, ap.chunk, ap.nsplit);
+}
+
+cudaError_t attention_bf16(const ModelDims& md, const AttnPlan& ap, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const CUtensorMap* tmQ, const void* q, void* o,
+                           float* opart, float2* ml, const int32_t* lens, const uint8_t* done,
+                           const int* n_active, int* err, cudaStream_t st) {
+  return attn_poly()
+             ? attention_bf16_t<true>(md, ap, tmK, tmV, tmQ, q, o, opart, ml, lens, done,
+                                      n_active, err, st)
+             : attention_bf16_t<false>(md, ap, tmK, tmV, tmQ, q, o, opart, ml, lens, done,
+                                       n_active, err, st);
 }
 
 int attn_cluster_capacity(int n) {
@@ -1157,7 +1203,7 @@ int attn_cluster_capacity(int n) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int num = 0;
-  if (cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&num, attn_tc_kernel<false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     num = 0;
   }

@@ -240,13 +240,16 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
   }
   if (mt > 1) {
     // tensor-bound: K not split, so the projection epilogues can be fused
-    // into the GEMM; 256-wide tiles (less shared-memory and L2 traffic per
-    // flop) unless 128-wide ones fill the SMs' waves clearly better
+    // into the GEMM; 256-wide tiles: a 128 x 128 MMA step needs the whole
+    // shared-memory bandwidth (measured ~6 against ~10 TFLOP/s per SM for
+    // 128 x 256), so 128-wide tiles pay only when 256-wide ones leave most
+    // SMs idle (fewer tiles than SMs and a clearly better fill)
     auto wave_eff = [&](int bn) {
       const int tiles = mt * cdiv(N, bn);
       return (double)tiles / ((double)cdiv(tiles, ctx->num_sms) * ctx->num_sms);
     };
-    p.BN = wave_eff(128) > wave_eff(256) + 0.05 ? 128 : 256;
+    const bool under_one_wave = mt * cdiv(N, 256) < ctx->num_sms;
+    p.BN = under_one_wave && wave_eff(128) > wave_eff(256) + 0.05 ? 128 : 256;
     return p;
   }
   // one M tile: weight-read bound; split K over as many CTAs as fit in one
@@ -269,8 +272,9 @@ GemmPlan plan_gemm(const dlm_ctx* ctx, int M, int N, int K, int epi) {
 // one wave of resident clusters; otherwise splits write partials for the
 // combine kernel (a write cost per CTA, the kernel, a cost per partial).
 // Costs in microseconds, from B200 measurements: a 128-row tile of 128 keys
-// takes ~1.2 us in a lone CTA and ~1.7 us when every SM streams K/V; a
-// 256-row CTA reads each tile once for both row tiles.
+// takes ~1.2 us in a lone CTA and ~1.6 us when every SM streams K/V; a
+// 256-row CTA reads each tile once for both row tiles (L2 already catches the
+// second 128-row tile's reads) and takes ~2.65 us per tile pair.
 // max_part_slots > 0 bounds the partial row slots (B * Hkv * nsplit * R) of
 // plans that combine through the combine kernel; one split (no partials) and
 // cluster plans always qualify.
@@ -303,8 +307,11 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
     if (rows == 256 && a.rtiles < 2) continue;          // one row tile: nothing to pair
     if (only_rows > 0 && rows != only_rows && !(only_rows == 256 && a.rtiles < 2)) continue;
     const int ytiles = rows == 256 ? cdiv(a.rtiles, 2) : a.rtiles;   // CTAs per split
-    const double t_tile = rows == 256 ? 2.0 : 1.5;
-    const double t_cta = rows == 256 ? 3.5 : 3.0;
+    // measured (device timeline): a 128-row tile ~1.2 us alone, ~1.6 us with
+    // every SM streaming; a 256-row tile pair ~2.65 us -- the same per-row
+    // rate, so the wider CTA wins only where it saves CTAs
+    const double t_tile = rows == 256 ? 2.9 : 1.5;
+    const double t_cta = rows == 256 ? 4.0 : 3.0;
     int last_nsplit = 0;
     for (int ct = 1; ct <= max_tiles; ++ct) {
       if (only_ct > 0 && ct != std::min(only_ct, max_tiles)) continue;
@@ -1269,6 +1276,16 @@ int dlm_check(dlm_ctx* ctx, void* stream) {
 }
 
 int dlm_launches_per_step(const dlm_ctx* ctx) { return ctx ? ctx->launches : DLM_EINVAL; }
+
+int dlm_test_exp2(const float* x, float* out, int n, void* stream) {
+  g_create_error.clear();
+  if (x == nullptr || out == nullptr || n < 0)
+    return fail(nullptr, DLM_EINVAL, "test_exp2: NULL pointer or n < 0");
+  if (n == 0) return DLM_OK;
+  cudaError_t e = exp2_poly_apply(x, out, n, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(nullptr, "test_exp2 launch", e);
+  return DLM_OK;
+}
 
 int dlm_test_withhold_loads(dlm_ctx* ctx, int n_launches) {
   if (ctx == nullptr) return DLM_EINVAL;

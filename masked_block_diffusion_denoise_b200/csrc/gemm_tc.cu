@@ -455,18 +455,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // 128-column heads, each as two units of 32 rotary pairs (j, j+64),
           // j in [32c, 32c+32): rotate q and k, store q rows and the canvas
           // K / V into the cache slots.  The BN/64 units of a tile are split
-          // evenly between the two warpgroups.
+          // evenly between the two warpgroups.  The row's cache slot is read
+          // once per tile, and each unit's cos/sin (16-byte loads) are in
+          // flight while its accumulator columns come out of tensor memory.
           const ProjEpi& pe = p.proj;
           const int seq = row / pe.C, p_in = row - seq * pe.C;
           const bool live = row < p.M && (p.done == nullptr || p.done[seq] == 0);
+          const int pos = live ? pe.lens[seq] + p_in : 0;
+          const bool pos_ok = live && DLM_IN_BOUNDS(pos, pe.Lcap, p.err);
           constexpr int kUnits = BN / 128 * 2;
 #pragma unroll 1
           for (int u = wg * kUnits / 2; u < (wg + 1) * kUnits / 2; ++u) {
             const int hc = u >> 1, c = u & 1;
             const int head = (n * BN) / 128 + hc;
-            bool store = live && head < pe.H + 2 * pe.Hkv;
-            const int pos = store ? pe.lens[seq] + p_in : 0;
-            if (store && !DLM_IN_BOUNDS(pos, pe.Lcap, p.err)) store = false;
+            const bool store = pos_ok && head < pe.H + 2 * pe.Hkv;
             __nv_bfloat16* dst = nullptr;
             if (store) {
               if (head < pe.H) {
@@ -479,42 +481,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                       (((size_t)seq * pe.Hkv + (head - pe.H - pe.Hkv)) * pe.Lcap + pos) * 128;
               }
             }
-            const bool rotate = pe.rope != nullptr && head < pe.H + pe.Hkv;
-            {
-              uint32_t lo_raw[32], hi_raw[32];
-              tmem_ld32_nowait(taddr + hc * 128 + c * 32, lo_raw);
-              tmem_ld32_nowait(taddr + hc * 128 + 64 + c * 32, hi_raw);
+            const bool rotate = store && pe.rope != nullptr && head < pe.H + pe.Hkv;
+            // two halves of 16 pairs
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+              const int j0 = c * 32 + h * 16;   // first pair of this half
+              float4 cs[8];                     // cos/sin of its 16 pairs, two a load
+              if (rotate) {
+                const float4* src = reinterpret_cast<const float4*>(pe.rope + (size_t)pos * 64 + j0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) cs[j] = src[j];
+              }
+              uint32_t lo_raw[16], hi_raw[16];
+              tmem_ld16_nowait(taddr + hc * 128 + j0, lo_raw);
+              tmem_ld16_nowait(taddr + hc * 128 + 64 + j0, hi_raw);
               tmem_wait_ld();
               if (store) {
-                float lo[32], hi[32];
+                float lo[16], hi[16];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < 16; ++j) {
                   lo[j] = __uint_as_float(lo_raw[j]);
                   hi[j] = __uint_as_float(hi_raw[j]);
                 }
                 if (rotate) {
-                  const float2* cs = pe.rope + (size_t)pos * 64 + c * 32;
 #pragma unroll
-                  for (int j = 0; j < 32; ++j) {
-                    const float2 r = cs[j];
+                  for (int j = 0; j < 16; ++j) {
+                    const float2 r = (j & 1) ? make_float2(cs[j >> 1].z, cs[j >> 1].w)
+                                             : make_float2(cs[j >> 1].x, cs[j >> 1].y);
                     const float a = lo[j], b2 = hi[j];
                     lo[j] = a * r.x - b2 * r.y;
                     hi[j] = b2 * r.x + a * r.y;
                   }
                 }
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  uint4 w, u;
+                for (int q4 = 0; q4 < 2; ++q4) {
+                  uint4 w, v;
                   w.x = pack_bf16(lo[8 * q4 + 0], lo[8 * q4 + 1]);
                   w.y = pack_bf16(lo[8 * q4 + 2], lo[8 * q4 + 3]);
                   w.z = pack_bf16(lo[8 * q4 + 4], lo[8 * q4 + 5]);
                   w.w = pack_bf16(lo[8 * q4 + 6], lo[8 * q4 + 7]);
-                  u.x = pack_bf16(hi[8 * q4 + 0], hi[8 * q4 + 1]);
-                  u.y = pack_bf16(hi[8 * q4 + 2], hi[8 * q4 + 3]);
-                  u.z = pack_bf16(hi[8 * q4 + 4], hi[8 * q4 + 5]);
-                  u.w = pack_bf16(hi[8 * q4 + 6], hi[8 * q4 + 7]);
-                  reinterpret_cast<uint4*>(dst + c * 32)[q4] = w;
-                  reinterpret_cast<uint4*>(dst + 64 + c * 32)[q4] = u;
+                  v.x = pack_bf16(hi[8 * q4 + 0], hi[8 * q4 + 1]);
+                  v.y = pack_bf16(hi[8 * q4 + 2], hi[8 * q4 + 3]);
+                  v.z = pack_bf16(hi[8 * q4 + 4], hi[8 * q4 + 5]);
+                  v.w = pack_bf16(hi[8 * q4 + 6], hi[8 * q4 + 7]);
+                  reinterpret_cast<uint4*>(dst + j0)[q4] = w;
+                  reinterpret_cast<uint4*>(dst + 64 + j0)[q4] = v;
                 }
               }
             }

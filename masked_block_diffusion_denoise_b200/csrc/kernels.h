@@ -149,6 +149,9 @@ cudaError_t quantize_rows_nvfp4(const void* x, int rows, int cols, uint8_t* q, u
                                 float* row_scale, int C, const uint8_t* done, const int* n_active,
                                 cudaStream_t st);
 
+// out[i] = exp2_poly(x[i]) (the attention's exponential on the FMA pipe)
+cudaError_t exp2_poly_apply(const float* x, float* out, int n, cudaStream_t st);
+
 // ---- attention.cu ------------------------------------------------------------
 struct AttnPlan {
   int B, C, G, R, rtiles;   // G = H / Hkv, R = G * C query rows per (seq, kv head)

@@ -302,6 +302,12 @@ __global__ void __launch_bounds__(256) quantize_rows_nvfp4_kernel(
   if (threadIdx.x == 0) row_scale[r] = sr;
 }
 
+// test hook: the attention's polynomial exp2 on given arguments
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = exp2_poly(x[i]);
+}
+
 __global__ void canvas_init_kernel(int C, int V, int mask_id, int uniform, uint32_t s0,
                                    uint32_t s1, int32_t* tokens, uint8_t* committed,
                                    int32_t* step, uint8_t* done, int32_t* eos_pos,
@@ -416,6 +422,11 @@ cudaError_t quantize_rows_nvfp4(const void* x, int rows, int cols, uint8_t* q, u
   if (cols % 64 != 0) return cudaErrorInvalidValue;
   return launch_pdl(quantize_rows_nvfp4_kernel, dim3(rows), dim3(256), 0, st,
                     (const __nv_bfloat16*)x, rows, cols, q, sf, row_scale, C, done, n_active);
+}
+
+cudaError_t exp2_poly_apply(const float* x, float* out, int n, cudaStream_t st) {
+  exp2_poly_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, out, n);
+  return cudaGetLastError();
 }
 
 cudaError_t add_len_all(int32_t* lens, int B, int n, cudaStream_t st) {

@@ -23,7 +23,7 @@ def _library():
 def header_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(dlm_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(dlm_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary():
