@@ -81,16 +81,25 @@ static_assert(kRecvOff + (kRowsCta + kMaxCluster) * kXoRowBytes <= kStages * kSt
               "exchange areas exceed the K/V ring");
 static_assert(kXoRowBytes % 16 == 0 && kRecvOff % 16 == 0, "bulk copies need 16-byte units");
 
-// maximum of a thread's 128 scores as eight independent chains and a tree
-// (a single chain of 128 dependent maxima would be latency, not throughput)
+// three-input maximum (sm_100 max.f32 with three operands)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// maximum of a thread's 128 scores as eight independent chains of
+// three-input maxima and a tree (a single chain of 128 dependent maxima
+// would be latency, not throughput)
 __device__ __forceinline__ float row_max128(const float (&sv)[kKeys]) {
   float m[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m[k] = sv[k];
+  for (int k = 0; k < 8; ++k) m[k] = fmaxf(sv[k], sv[k + 8]);
 #pragma unroll
-  for (int j = 8; j < kKeys; ++j) m[j & 7] = fmaxf(m[j & 7], sv[j]);
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
-               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+  for (int j = 16; j < kKeys; j += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = fmax3(m[k], sv[j + k], sv[j + 8 + k]);
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // One CTA per (key split, 128-query-row tile, sequence x KV head), 6 warps:
@@ -141,9 +150,12 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* ring = smem + kQBytes;
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* s_full = kv_empty + kStages;   // [2]: S(t) in TMEM buffer t % 2
+  // [2]: P(t) in TMEM buffer t % 2.  One barrier per buffer keeps the softmax
+  // at most one phase ahead of the issuer: it can arrive for t + 2 only after
+  // S(t + 2), which is issued after P(t) V(t)
   uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 1;
+  uint64_t* pv_done = p_full + 2;
   uint64_t* mma_done = pv_done + 1;
   uint64_t* q_full = mma_done + 1;
   uint64_t* rx = q_full + 1;   // cluster exchange: the peers' rows have landed
@@ -156,8 +168,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
-    mbar_init(p_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+    }
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
     mbar_init(q_full, 1);
@@ -288,7 +302,7 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
           issue_s(t1);
         }
-        if (!mbar_wait_bounded(p_full, (uint32_t)(t & 1), abort_flag)) {
+        if (!mbar_wait_bounded(&p_full[t & 1], (uint32_t)((t >> 1) & 1), abort_flag)) {
           ok = false;
           break;
         }
@@ -386,12 +400,13 @@ __global__ void __launch_bounds__(192, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[buf]);
     }
+    // every MMA has completed (a one-phase barrier: no parity can alias, as
+    // a wait on pv_done for the last tile could while P(t-1) V(t-1) runs)
     float ov[kDh];
     bool have = false;
-    if (ok && n_tiles > 0 &&
-        mbar_wait_bounded(pv_done, (uint32_t)((n_tiles - 1) & 1), abort_flag)) {
+    if (ok && n_tiles > 0 && mbar_wait_bounded(mma_done, 0, abort_flag)) {
       tc_fence_after();
       have = true;
       if (row == 0) DLM_TRACE_MARK(4);

@@ -290,7 +290,10 @@ AttnPlan plan_attention(const dlm_ctx* ctx, int B, int C, const int* lens, int m
   const int sms = std::min(std::max(ctx->num_sms, 1), 1024);
   const int max_keys = max_len_all + C;
   const int max_tiles = cdiv(max_keys, 128);
-  const double t_xchg = 1.5, t_pw = 1.5, t_comb = 4.0, t_part = 0.03;
+  // the combine kernel: ~30 us after the attention for the batched shape's
+  // 512 partial row tiles (device timeline), against the same attention with
+  // one split and no partials
+  const double t_xchg = 1.5, t_pw = 1.5, t_comb = 4.0, t_part = 0.05;
   double best = -1.0;
   double sm_free[1024];   // no heap allocation: this also runs inside dlm_attention_noalloc
   // diagnostic switch: DLM_ATTN_CLUSTER=0 keeps every split plan on the

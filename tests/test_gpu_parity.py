@@ -85,12 +85,16 @@ def test_small_block_stagewise(name):
         sess.close()
 
 
-@pytest.mark.parametrize("cluster", ["1", "0"])
-def test_attention_split_paths(cluster, monkeypatch):
+@pytest.mark.parametrize("cluster,tiles", [("1", None), ("0", None), ("0", 1)])
+def test_attention_split_paths(cluster, tiles, monkeypatch):
     """The split-KV attention both ways: splits combined inside a thread-block
     cluster, and splits written as partials for the combine kernel
-    (DLM_ATTN_CLUSTER=0); ragged prefixes leave some splits without keys."""
+    (DLM_ATTN_CLUSTER=0; also with 128-key splits, one per key tile); ragged
+    prefixes leave some splits without keys.  Two steps each."""
     monkeypatch.setenv("DLM_ATTN_CLUSTER", cluster)
+    if tiles is not None:
+        monkeypatch.setenv("DLM_ATTN_TILES", str(tiles))
+    from masked_block_diffusion_denoise_b200 import dlm_attention_plan
     wl = W.small_workload("split_paths", n_heads=8, n_kv_heads=2, batch=3, canvas=16, steps=2,
                           quota=0, prefix_len=(20, 1500), prefix_cap=1600, seed=6)
     sess, om, _ = make_pair(wl)
@@ -98,7 +102,13 @@ def test_attention_split_paths(cluster, monkeypatch):
         cv = sess.new_canvas(wl.batch, wl.canvas)
         p_lib, p_or = lib_params(wl), oracle_params(wl)
         sess.init(cv, p_lib)
-        check_one_step(sess, om, wl, cv, p_lib, p_or)
+        plan = dlm_attention_plan(sess.ctx, wl.batch, wl.canvas)
+        if cluster == "0":
+            assert plan["cluster"] == 1, plan
+        if tiles is not None:
+            assert plan["chunk"] == 128 and plan["nsplit"] >= 4, plan
+        for _ in range(2):
+            check_one_step(sess, om, wl, cv, p_lib, p_or)
     finally:
         sess.close()
 
