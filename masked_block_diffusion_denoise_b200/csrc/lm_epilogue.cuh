@@ -71,6 +71,67 @@ __device__ __forceinline__ float lm_inv_temp(const LmEpi& e, int step) {
   return 1.f;
 }
 
+// three-input maximum (sm_100 max.f32 with three operands)
+__device__ __forceinline__ float lm_max3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
+// Greedy fold of a chunk with no excluded column (the common case: every
+// chunk but the one holding the mask id and the vocabulary's ragged end).
+// The same state as the general path below, with less work per logit, which
+// matters on a power-capped GPU where the epilogue's instructions take power
+// from the tensor cores: the chunk maximum by three-input maxima; the
+// argmax searched only when the chunk beats the row's best (first
+// occurrence, as the general path); then per logit one FFMA (x = z log2 e -
+// m log2 e), one exponential, one add for s and one FFMA for the entropy
+// term, summed in base 2 and scaled by ln 2 once per chunk.
+template <int N>
+__device__ __forceinline__ void rs_update_greedy_clean(RowState& r, const float (&v)[N],
+                                                       int col0) {
+  static_assert(N % 4 == 0, "chunks of 4k logits");
+  float mx[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+  for (int j = 4; j + 8 <= N; j += 8)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx[k] = lm_max3(mx[k], v[j + k], v[j + 4 + k]);
+  if constexpr (N % 8 == 0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], v[N - 4 + k]);
+  }
+  const float cmax = fmaxf(lm_max3(mx[0], mx[1], mx[2]), mx[3]);
+  if (!(cmax > -CUDART_INF_F)) return;   // no finite logit (as the general path)
+  if (cmax > r.g) {   // columns arrive in increasing order: on equal values the earlier wins
+    int carg = 0;
+#pragma unroll
+    for (int j = N - 1; j >= 0; --j) carg = v[j] == cmax ? j : carg;
+    r.g = cmax;
+    r.zw = cmax;
+    r.idx = col0 + carg;
+  }
+  if (cmax > r.m) {
+    if (r.m != -CUDART_INF_F) {
+      const float a = __expf(r.m - cmax);
+      r.t = (r.t + r.s * (r.m - cmax)) * a;
+      r.s *= a;
+    }
+    r.m = cmax;
+  }
+  constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+  const float m2 = r.m * kLog2e;
+  float s4[4] = {0.f, 0.f, 0.f, 0.f}, t4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float x = fmaf(v[j], kLog2e, -m2);   // (z - m) log2 e
+    const float ex = fast_exp2(x);
+    s4[j & 3] += ex;
+    t4[j & 3] = fmaf(ex, x, t4[j & 3]);
+  }
+  r.s += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  r.t = fmaf((t4[0] + t4[1]) + (t4[2] + t4[3]), kLn2, r.t);
+}
+
 // Fold N consecutive logits (columns col0 .. col0+N-1, col0 % 4 == 0) of one
 // row into the row state.  canvas / pos / step locate the row for the
 // sampling counter.
@@ -78,6 +139,10 @@ template <int N>
 __device__ __forceinline__ void rs_update(RowState& r, const float (&v)[N], int col0,
                                           float inv_t, const LmEpi& e, int canvas, int pos,
                                           int step) {
+  if (e.mode == LM_GREEDY && col0 + N <= e.V && (unsigned)(e.mask_id - col0) >= (unsigned)N) {
+    rs_update_greedy_clean<N>(r, v, col0);
+    return;
+  }
   float z[N];
   float cmax = -CUDART_INF_F;
   int carg = 0;
