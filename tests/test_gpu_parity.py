@@ -52,6 +52,12 @@ SMALL = {
                                          canvas=64, steps=4, quota=0, prefix_len=(64, 300),
                                          prefix_cap=320, vocab=3000, lm_fp8=True,
                                          corruption="uniform"),
+    # two M tiles, 256-wide LM tiles, vocabulary 20440 = 80 tiles (the last
+    # ragged): on 148 SMs 74 CTAs share each M tile and 6 of them take a
+    # second tile
+    "small_lm_tail": W.small_workload("small_lm_tail", n_heads=8, n_kv_heads=2, batch=4,
+                                      canvas=64, steps=3, quota=0, prefix_len=(64, 300),
+                                      prefix_cap=320, vocab=20440, seed=7),
     # NVFP4 LM head, one M tile, ragged vocabulary
     "small_nvfp4": W.small_workload("small_nvfp4", steps=6, quota=0, lm_nvfp4=True, seed=4),
     # NVFP4 LM head over two M tiles, d 512 (two k-blocks), uniform corruption
